@@ -1,0 +1,40 @@
+"""CPU oracle for content-adaptive block-sparse tile attention.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the library imports this package; only
+``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg use
+it.  It is a plain, slow, fp64 restatement of the method, written so that a
+reader can check it step by step against the source it cites.
+
+Sources (cited by page title and section):
+
+* "NABLA: Neighborhood Adaptive Block-Level Attention" (gist.science
+  explanation of arXiv 2507.13546), section "Méthodologie : NABLA":
+  token reordering ("Fractal Flattening"), block mean-pooling
+  ("Sous-échantillonnage"), the reduced attention map ("Attention Réduite"),
+  the per-row CDF threshold ("Seuil CDF"), expansion of the block mask
+  ("Expansion") and the union with Sliding Tile Attention ("Intégration
+  Hybride avec STA"); the lay section "L'ancienne solution" describes STA as
+  a tile attending to itself and the immediately adjacent tiles.
+* "AB-Attention accélère la génération vidéo…" (news.hamidun.com), section
+  "Les trois techniques": the kernel gathers the selected key/value blocks
+  by index, which is why the mask is also emitted as per-row index lists.
+
+Readings adopted where the pages are silent or garbled are listed in the
+module docstring of ``oracle.nabla``.
+"""
+from .nabla import (  # noqa: F401
+    Geometry,
+    bf16_bits_to_f64,
+    tile_reorder,
+    tile_unreorder,
+    block_mean_pool,
+    pooled_score_map,
+    cdf_select_row,
+    cdf_select,
+    sta_mask,
+    build_block_mask,
+    mask_to_lists,
+    masked_attention,
+    dense_attention,
+    kept_pair_flops,
+)
