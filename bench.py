@@ -1,0 +1,342 @@
+"""Benchmark of the block-sparse tile attention path on B200.
+
+One step = one pass of the whole path over one batch of the Wan-like 480p
+latent workload (B=1, H=40, D=128, token grid 21x32x56 in 1x8x8 tiles,
+N=37632, 588 blocks; CDF threshold p=0.9; seeded synthetic q/k/v):
+    tile_reorder(q, k, v) -> build_block_mask -> block_sparse_attn -> tile_unreorder(o)
+
+`value` = kept-block TFLOP/s of the whole step (4*D*64*64 FLOP per kept
+block pair, summed over heads, divided by the step time) with inputs resident
+in HBM; `e2e` = the same metric with pinned-host inputs copied in and the
+output copied back inside the timed region.  Inputs (385 MB per tensor) are
+larger than the 126 MB L2, so no flush is needed between steps.
+
+Multi-GPU (torchrun): every rank runs its own independent Wan-sized problem
+(weak scaling, no collective on the data path); the time is the max over
+ranks.  `--impl reference` times the CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import dbst_synth as S  # noqa: E402
+
+METRIC = "sparse-attn ms/call & TFLOP/s on kept blocks (N=32760,H=40,D=128,bf16)"
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d["bf16_tflops"], d["bf16_tflops_sustained"], "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def workload_desc(w: S.Workload, p: float) -> str:
+    return (f"{w.name}-like latent: B={w.B} H={w.H} D={w.D} grid={w.grid[0]}x{w.grid[1]}x{w.grid[2]} "
+            f"(N={w.N}, {w.NB} blocks of {w.tile[0]}x{w.tile[1]}x{w.tile[2]}), p={p}, "
+            f"sta_radius={w.sta_radius}")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample(w: S.Workload, p: float, budget_s: float, seed: int = 7):
+    """Time the CPU oracle on a bounded sample of the workload.
+
+    Sample: a few heads; for each, the full oracle mask (pool, reduced map,
+    CDF selection) and the masked attention of randomly chosen query blocks,
+    until ~budget_s seconds of CPU work.  Returns (kept-block TFLOP/s, seconds,
+    description).
+    """
+    import dataclasses
+    import oracle as O
+    rng = np.random.default_rng(seed)
+    g1 = O.Geometry(1, 1, w.D, *w.grid, *w.tile)
+    scale = 1.0 / math.sqrt(w.D)
+    flops = 0.0
+    elapsed = 0.0
+    heads_done, rows_done = 0, 0
+    h = 0
+    while elapsed < budget_s and h < w.H:
+        q, k, v = S.make_qkv(w, heads=range(h, h + 1), batches=range(1))
+        t0 = time.perf_counter()
+        qt, kt, vt = (O.tile_reorder(a, g1) for a in (q, k, v))
+        mask = O.build_block_mask(qt, kt, g1, p, w.sta_radius)
+        elapsed += time.perf_counter() - t0
+        heads_done += 1
+        order = rng.permutation(g1.NB)
+        for i in order:
+            if elapsed >= budget_s:
+                break
+            t0 = time.perf_counter()
+            O.masked_attention(qt, kt, vt, mask, 64, scale, rows=[(0, 0, int(i))])
+            elapsed += time.perf_counter() - t0
+            flops += 4.0 * w.D * 64 * 64 * float(mask[0, 0, i].sum())
+            rows_done += 1
+        h += 1
+    desc = (f"oracle (numpy fp64) on {heads_done} head(s): full mask build per head + masked attention of "
+            f"{rows_done} random query blocks; kept-block FLOPs of those blocks / CPU seconds")
+    return flops / elapsed / 1e12, elapsed, desc
+
+
+def run_reference(args, w, p):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    vals, secs = [], []
+    desc = ""
+    for step in range(args.warmup + args.steps):
+        v, s, desc = oracle_sample(w, p, budget_s=args.ref_budget, seed=100 + step)
+        if step >= args.warmup:
+            vals.append(v)
+            secs.append(s)
+    value = statistics.mean(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(secs),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": workload_desc(w, p), "sample": "bounded oracle sample"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="wan")
+    ap.add_argument("--p", type=float, default=None)
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--ref-budget", type=float, default=10.0, help="seconds of oracle work per reference step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = S.workload(args.workload)
+    p = args.p if args.p is not None else w.p_list[0]
+    if args.impl == "reference":
+        return run_reference(args, w, p)
+
+    import torch
+    import torch.distributed as dist
+    import dynamic_block_sparse_tile_b200 as dbst
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    dbst.load()
+    g = dbst.Geom.make(w.B, w.H, w.D, w.grid, w.tile)
+    q_h, k_h, v_h = S.make_qkv(w)
+    to_t = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)   # noqa: E731
+    host = [to_t(a).pin_memory() for a in (q_h, k_h, v_h)]
+    del q_h, k_h, v_h
+    q, k, v = (t.cuda() for t in host)
+    qt, kt, vt, ot, o = (torch.empty_like(q) for _ in range(5))
+    bits = torch.empty((g.B, g.H, g.NB, g.NW), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((g.B, g.H, g.NB), dtype=torch.int32, device="cuda")
+    idx = torch.empty((g.B, g.H, g.NB, g.NB), dtype=torch.int16, device="cuda")
+    ws = torch.empty(dbst.mask_workspace_bytes(g), dtype=torch.uint8, device="cuda")
+    lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device="cuda")
+    o_host = torch.empty_like(host[0]).pin_memory()
+    stream = torch.cuda.current_stream()
+    launches_per_step = 8   # 3 reorder + pool + logits + select + attention + unreorder
+
+    ev = {}
+
+    def step(timed_parts: bool):
+        dbst.tile_reorder(q, g, out=qt)
+        dbst.tile_reorder(k, g, out=kt)
+        dbst.tile_reorder(v, g, out=vt)
+        if timed_parts:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        dbst.build_block_mask(qt, kt, g, p, w.sta_radius, workspace=ws, out=(bits, cnt, idx))
+        if timed_parts:
+            e1 = torch.cuda.Event(enable_timing=True)
+            e1.record(stream)
+        dbst.block_sparse_attn(qt, kt, vt, g, cnt, idx, 0.0, want_lse=True, out=ot, lse=lse)
+        if timed_parts:
+            e2 = torch.cuda.Event(enable_timing=True)
+            e2.record(stream)
+            ev.setdefault("parts", []).append((e0, e1, e2))
+        dbst.tile_unreorder(ot, g, out=o)
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    dbst.get_error()
+    kept_pairs = int(cnt.sum().item())
+    kept_frac = kept_pairs / (g.B * g.H * g.NB * g.NB)
+    flops = 4.0 * w.D * 64 * 64 * kept_pairs
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        step(True)
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    dbst.get_error()
+    ms_total = start.elapsed_time(end)
+    mask_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev["parts"])
+    attn_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev["parts"])
+
+    # end to end: pinned host inputs -> device -> path -> output back to pinned host
+    def e2e_step():
+        for src, dst in zip(host, (q, k, v)):
+            dst.copy_(src, non_blocking=True)
+        step(False)
+        o_host.copy_(o, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    s2 = torch.cuda.Event(enable_timing=True)
+    e2 = torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e2.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = s2.elapsed_time(e2)
+    dbst.get_error()
+
+    t = torch.tensor([ms_total, e2e_ms, attn_ms, mask_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total, e2e_ms, attn_ms, mask_ms = (float(x) for x in t.tolist())
+    ms_step = ms_total / args.steps
+    value = world * flops / (ms_step * 1e-3) / 1e12
+    e2e_value = world * flops / (e2e_ms / args.steps * 1e-3) / 1e12
+
+    hbm, bf16, bf16_sus, src = peaks()
+    attn_tflops = flops / (attn_ms * 1e-3) / 1e12
+    mask_bytes = 2 * w.B * w.H * w.N * w.D * 2
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_desc(w, p), "kept_fraction": kept_frac, "kept_block_pairs": kept_pairs,
+                   "l2": "inputs (385 MB per tensor) larger than L2; no flush", "parallelism": f"dp{world} (independent problems)"},
+        "sparse_attn_ms_per_call": attn_ms, "sparse_attn_tflops": attn_tflops,
+        "mask_build_ms_per_call": mask_ms, "mask_build_gbs": mask_bytes / (mask_ms * 1e-3) / 1e9,
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": bf16, "unit": "TFLOP/s",
+                     "frac": attn_tflops / bf16, "traffic": None,
+                     "peak_source": f"{src} bf16 burst; frac of sustained {attn_tflops / bf16_sus:.3f}",
+                     "kernel": "sparse_attn_kernel<128>"},
+        "mask_roofline": {"bound": "hbm", "achieved": mask_bytes / (mask_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                          "frac": mask_bytes / (mask_ms * 1e-3) / 1e9 / hbm},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "ms_per_step": e2e_ms / args.steps,
+                "h2d_bytes_per_step": 3 * host[0].numel() * 2, "d2h_bytes_per_step": o_host.numel() * 2},
+        "clocks": clk, "gpu_launches": launches_per_step * args.steps,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        cv, cs, desc = oracle_sample(w, p, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": cv, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                                "sample": desc}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

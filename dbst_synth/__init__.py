@@ -84,7 +84,7 @@ WORKLOADS: List[Workload] = [
     Workload("small", 1, B=1, H=8, D=64, grid=(8, 16, 16), tile=(1, 8, 8),
              alpha=0.7, beta=0.3, f_rms=2.0, kmax=3, p_list=(0.8, 0.9, 0.95), sta_radius=1),
     Workload("wan", 2, B=1, H=40, D=128, grid=(21, 32, 56), tile=(1, 8, 8),
-             alpha=0.5, beta=0.5, f_rms=2.0, kmax=3, p_list=(0.9,), sta_radius=-1,
+             alpha=0.5, beta=0.5, f_rms=2.54, kmax=3, p_list=(0.9,), sta_radius=-1,
              unpadded=(21, 30, 52)),
     Workload("hunyuan", 3, B=1, H=24, D=128, grid=(34, 48, 80), tile=(2, 4, 8),
              alpha=0.4, beta=0.6, f_rms=2.0, kmax=3, p_list=(0.9,), sta_radius=1,

@@ -1,0 +1,206 @@
+"""Python binding of libdbst.so: block-sparse tile attention on B200 (sm_100a).
+
+Argument marshalling only.  Every step of the path runs in the library's CUDA
+kernels; there is no CPU or PyTorch fallback, and importing a function whose
+library is missing raises immediately.  Tensors are torch CUDA tensors
+(device memory and streams come from PyTorch); each call is enqueued on the
+current torch stream.
+
+Layouts follow ``include/dbst.h``: q, k, v, o are bf16 ``[B, H, N, D]``
+contiguous, raster order ``n = (t*Y + y)*X + x`` or tile order.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+__all__ = ["Geom", "DbstError", "lib_path", "load", "tile_reorder", "tile_unreorder", "mask_workspace_bytes",
+           "build_block_mask", "mask_from_bits", "block_sparse_attn", "dense_attn", "get_error", "EXPORTS"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libdbst.so")
+
+# Every symbol declared in include/dbst.h.
+EXPORTS = ("dbst_status_string", "dbst_tile_reorder", "dbst_tile_unreorder", "dbst_mask_workspace_bytes",
+           "dbst_build_block_mask", "dbst_mask_from_bits", "dbst_block_sparse_attn", "dbst_dense_attn",
+           "dbst_get_error")
+
+DBST_OK, DBST_EINVAL, DBST_ECUDA, DBST_ETIMEOUT, DBST_EBOUNDS = 0, 1, 2, 3, 4
+
+
+class DbstError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {_status_string(status)} (status {status})")
+        self.status = status
+
+
+class Geom(ctypes.Structure):
+    """Mirror of ``dbst_geom``: batch, heads, head dim, token grid, tile shape."""
+    _fields_ = [(n, ctypes.c_int) for n in ("B", "H", "D", "T", "Y", "X", "tt", "ty", "tx")]
+
+    @classmethod
+    def make(cls, B: int, H: int, D: int, grid: Sequence[int], tile: Sequence[int]) -> "Geom":
+        return cls(B, H, D, *grid, *tile)
+
+    @property
+    def N(self) -> int:
+        return self.T * self.Y * self.X
+
+    @property
+    def NB(self) -> int:
+        return self.N // 64
+
+    @property
+    def NW(self) -> int:
+        return (self.NB + 31) // 32
+
+
+_lib = None
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load() -> ctypes.CDLL:
+    """Load libdbst.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"{_LIB_PATH} is missing: build it with `python -m dynamic_block_sparse_tile_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, gp, i32, f32 = ctypes.c_void_p, ctypes.POINTER(Geom), ctypes.c_int, ctypes.c_float
+    lib.dbst_status_string.argtypes, lib.dbst_status_string.restype = [i32], ctypes.c_char_p
+    for name in ("dbst_tile_reorder", "dbst_tile_unreorder"):
+        getattr(lib, name).argtypes = [vp, vp, gp, vp]
+        getattr(lib, name).restype = i32
+    lib.dbst_mask_workspace_bytes.argtypes, lib.dbst_mask_workspace_bytes.restype = [gp], ctypes.c_size_t
+    lib.dbst_build_block_mask.argtypes = [vp, vp, gp, f32, i32, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.dbst_build_block_mask.restype = i32
+    lib.dbst_mask_from_bits.argtypes, lib.dbst_mask_from_bits.restype = [vp, gp, vp, vp, vp], i32
+    lib.dbst_block_sparse_attn.argtypes = [vp, vp, vp, gp, vp, vp, f32, vp, vp, vp]
+    lib.dbst_block_sparse_attn.restype = i32
+    lib.dbst_dense_attn.argtypes, lib.dbst_dense_attn.restype = [vp, vp, vp, gp, f32, vp, vp, vp], i32
+    lib.dbst_get_error.argtypes, lib.dbst_get_error.restype = [vp], i32
+    _lib = lib
+    return lib
+
+
+def _status_string(status: int) -> str:
+    try:
+        return load().dbst_status_string(status).decode()
+    except Exception:
+        return "unknown"
+
+
+def _check(status: int, what: str) -> None:
+    if status != DBST_OK:
+        raise DbstError(status, what)
+
+
+def _stream() -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _need(t: torch.Tensor, dtype: torch.dtype, shape: Tuple[int, ...], name: str) -> None:
+    if not t.is_cuda or t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{name}: expected contiguous CUDA {dtype} {tuple(shape)}, got "
+                         f"{t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def _qkv_shape(g: Geom) -> Tuple[int, int, int, int]:
+    return (g.B, g.H, g.N, g.D)
+
+
+def tile_reorder(x: torch.Tensor, g: Geom, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Raster -> tile order (``dbst_tile_reorder``)."""
+    _need(x, torch.bfloat16, _qkv_shape(g), "x")
+    out = torch.empty_like(x) if out is None else out
+    _need(out, torch.bfloat16, _qkv_shape(g), "out")
+    _check(load().dbst_tile_reorder(_ptr(x), _ptr(out), ctypes.byref(g), _stream()), "dbst_tile_reorder")
+    return out
+
+
+def tile_unreorder(y: torch.Tensor, g: Geom, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Tile -> raster order (``dbst_tile_unreorder``)."""
+    _need(y, torch.bfloat16, _qkv_shape(g), "y")
+    out = torch.empty_like(y) if out is None else out
+    _need(out, torch.bfloat16, _qkv_shape(g), "out")
+    _check(load().dbst_tile_unreorder(_ptr(y), _ptr(out), ctypes.byref(g), _stream()), "dbst_tile_unreorder")
+    return out
+
+
+def mask_workspace_bytes(g: Geom) -> int:
+    return int(load().dbst_mask_workspace_bytes(ctypes.byref(g)))
+
+
+def build_block_mask(q_tiled: torch.Tensor, k_tiled: torch.Tensor, g: Geom, p: float, sta_radius: int = -1,
+                     workspace: Optional[torch.Tensor] = None, out=None):
+    """Adaptive block mask (``dbst_build_block_mask``) -> (mask_bits, kv_count, kv_idx)."""
+    _need(q_tiled, torch.bfloat16, _qkv_shape(g), "q_tiled")
+    _need(k_tiled, torch.bfloat16, _qkv_shape(g), "k_tiled")
+    dev = q_tiled.device
+    if out is None:
+        bits = torch.empty((g.B, g.H, g.NB, g.NW), dtype=torch.int32, device=dev)
+        cnt = torch.empty((g.B, g.H, g.NB), dtype=torch.int32, device=dev)
+        idx = torch.empty((g.B, g.H, g.NB, g.NB), dtype=torch.int16, device=dev)
+    else:
+        bits, cnt, idx = out
+    nbytes = mask_workspace_bytes(g)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    _check(load().dbst_build_block_mask(_ptr(q_tiled), _ptr(k_tiled), ctypes.byref(g), float(p), int(sta_radius),
+                                        _ptr(bits), _ptr(cnt), _ptr(idx), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(), _stream()),
+           "dbst_build_block_mask")
+    return bits, cnt, idx
+
+
+def mask_from_bits(bits: torch.Tensor, g: Geom):
+    """Caller-supplied bitmask -> (kv_count, kv_idx) (``dbst_mask_from_bits``)."""
+    _need(bits, torch.int32, (g.B, g.H, g.NB, g.NW), "bits")
+    cnt = torch.empty((g.B, g.H, g.NB), dtype=torch.int32, device=bits.device)
+    idx = torch.empty((g.B, g.H, g.NB, g.NB), dtype=torch.int16, device=bits.device)
+    _check(load().dbst_mask_from_bits(_ptr(bits), ctypes.byref(g), _ptr(cnt), _ptr(idx), _stream()),
+           "dbst_mask_from_bits")
+    return cnt, idx
+
+
+def block_sparse_attn(q, k, v, g: Geom, kv_count, kv_idx, scale: float = 0.0, want_lse: bool = True,
+                      out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None):
+    """Attention over kept blocks (``dbst_block_sparse_attn``) -> (o, lse or None)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, _qkv_shape(g), n)
+    _need(kv_count, torch.int32, (g.B, g.H, g.NB), "kv_count")
+    _need(kv_idx, torch.int16, (g.B, g.H, g.NB, g.NB), "kv_idx")
+    o = torch.empty_like(q) if out is None else out
+    if want_lse and lse is None:
+        lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device=q.device)
+    _check(load().dbst_block_sparse_attn(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(g), _ptr(kv_count),
+                                         _ptr(kv_idx), float(scale), _ptr(o), _ptr(lse if want_lse else None),
+                                         _stream()), "dbst_block_sparse_attn")
+    return o, (lse if want_lse else None)
+
+
+def dense_attn(q, k, v, g: Geom, scale: float = 0.0, want_lse: bool = True):
+    """Dense attention over all tokens (``dbst_dense_attn``) -> (o, lse or None)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, _qkv_shape(g), n)
+    o = torch.empty_like(q)
+    lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device=q.device) if want_lse else None
+    _check(load().dbst_dense_attn(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(g), float(scale), _ptr(o), _ptr(lse),
+                                  _stream()), "dbst_dense_attn")
+    return o, lse
+
+
+def get_error() -> None:
+    """Synchronise the current stream and raise if a kernel recorded an error."""
+    _check(load().dbst_get_error(_stream()), "device")

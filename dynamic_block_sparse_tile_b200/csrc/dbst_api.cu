@@ -1,0 +1,309 @@
+// C ABI of libdbst.so: argument validation, launch configuration, TMA
+// descriptors and the device error word.  Every check runs on the host
+// before anything is enqueued.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/dbst.h"
+#include "attn.cuh"
+#include "mask.cuh"
+#include "ptx.cuh"
+#include "reorder.cuh"
+
+namespace {
+
+constexpr int kMaxNB = 4096;   // selection and list kernels keep one row on chip
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape checks shared by every entry point.
+bool geom_ok(const dbst_geom* g) {
+  if (!g) return false;
+  if (g->B < 1 || g->H < 1) return false;
+  if (g->D != 64 && g->D != 128) return false;
+  if (g->T < 1 || g->Y < 1 || g->X < 1 || g->tt < 1 || g->ty < 1 || g->tx < 1) return false;
+  if (static_cast<long long>(g->tt) * g->ty * g->tx != 64) return false;
+  if (g->T % g->tt || g->Y % g->ty || g->X % g->tx) return false;
+  const long long N = static_cast<long long>(g->T) * g->Y * g->X;
+  if (N / 64 > kMaxNB) return false;
+  const long long rows = N * g->B * g->H;
+  if (rows >= (1ll << 31)) return false;   // TMA row coordinates are int32
+  return true;
+}
+
+long long tokens(const dbst_geom* g) { return static_cast<long long>(g->T) * g->Y * g->X; }
+int nblocks(const dbst_geom* g) { return static_cast<int>(tokens(g) / 64); }
+long long bh_count(const dbst_geom* g) { return static_cast<long long>(g->B) * g->H; }
+
+int sm_count() {
+  static int n = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      n = 148;
+  });
+  return n;
+}
+
+dbst::TileGeo tile_geo(const dbst_geom* g) {
+  dbst::TileGeo t;
+  t.N = static_cast<int>(tokens(g));
+  t.X = g->X;
+  t.Y = g->Y;
+  t.tt = g->tt;
+  t.ty = g->ty;
+  t.tx = g->tx;
+  t.nX = g->X / g->tx;
+  t.nY = g->Y / g->ty;
+  return t;
+}
+
+dbst_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? DBST_OK : DBST_ECUDA;
+}
+
+dbst_status permute(const void* src, void* dst, const dbst_geom* g, void* stream, int to_tiled) {
+  if (!geom_ok(g) || !src || !dst || !aligned16(src) || !aligned16(dst)) return DBST_EINVAL;
+  const long long rows = bh_count(g) * tokens(g);
+  const long long bytes = rows * g->D * 2;
+  const char* a = static_cast<const char*>(src);
+  const char* b = static_cast<const char*>(dst);
+  if (a < b + bytes && b < a + bytes) return DBST_EINVAL;   // overlapping buffers
+  auto s = static_cast<cudaStream_t>(stream);
+  const long long chunks = rows * (g->D / 8);
+  long long grid = (chunks + 255) / 256;
+  const long long cap = static_cast<long long>(sm_count()) * 16;
+  if (grid > cap) grid = cap;
+  const auto* in = static_cast<const uint4*>(src);
+  auto* out = static_cast<uint4*>(dst);
+  if (g->D == 128)
+    dbst::tile_permute_kernel<4><<<static_cast<int>(grid), 256, 0, s>>>(in, out, tile_geo(g), rows, to_tiled);
+  else
+    dbst::tile_permute_kernel<3><<<static_cast<int>(grid), 256, 0, s>>>(in, out, tile_geo(g), rows, to_tiled);
+  return launch_status();
+}
+
+size_t align_up(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct MaskWorkspace {
+  size_t qp, kp, s, total;
+};
+MaskWorkspace mask_workspace(const dbst_geom* g) {
+  const size_t nb = static_cast<size_t>(nblocks(g));
+  const size_t bh = static_cast<size_t>(bh_count(g));
+  MaskWorkspace w;
+  w.qp = 0;
+  w.kp = align_up(bh * nb * g->D * sizeof(double));
+  w.s = w.kp + align_up(bh * nb * g->D * sizeof(double));
+  w.total = w.s + align_up(bh * nb * nb * sizeof(double));
+  return w;
+}
+
+// ---- TMA descriptors: a [rows, D] bf16 matrix, 64 x 64 boxes, 128-byte swizzle
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_tmap(CUtensorMap* m, const void* base, long long rows, int D) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D>
+dbst_status launch_attn(const void* q, const void* k, const void* v, const dbst_geom* g, const int32_t* cnt,
+                        const int16_t* idx, float scale, void* o, float* lse, cudaStream_t s) {
+  const long long rows = bh_count(g) * tokens(g);
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, rows, D) || !make_tmap(&tk, k, rows, D) || !make_tmap(&tv, v, rows, D)) return DBST_ECUDA;
+  dbst::AttnParams p;
+  p.kv_count = cnt;
+  p.kv_idx = idx;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.NB = nblocks(g);
+  p.N = static_cast<int>(tokens(g));
+  const float sc = scale > 0.0f ? scale : 1.0f / std::sqrt(static_cast<float>(D));
+  p.scale_log2 = sc * 1.4426950408889634f;
+  const int smem = dbst::AttnSmem::kBytes + 1024;
+  static std::once_flag once;
+  static cudaError_t attr = cudaSuccess;
+  std::call_once(once, [&] {
+    attr = cudaFuncSetAttribute(dbst::sparse_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  if (attr != cudaSuccess) return DBST_ECUDA;
+  const long long grid = bh_count(g) * p.NB;
+  if (grid >= (1ll << 31)) return DBST_EINVAL;
+  dbst::sparse_attn_kernel<D><<<static_cast<unsigned>(grid), 256, smem, s>>>(tq, tk, tv, p);
+  return launch_status();
+}
+
+dbst_status attn_common(const void* q, const void* k, const void* v, const dbst_geom* g, const int32_t* cnt,
+                        const int16_t* idx, float scale, void* o, float* lse, void* stream) {
+  if (!geom_ok(g) || !q || !k || !v || !o) return DBST_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return DBST_EINVAL;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return DBST_EINVAL;
+  if (!(std::isfinite(scale))) return DBST_EINVAL;
+  auto s = static_cast<cudaStream_t>(stream);
+  return g->D == 128 ? launch_attn<128>(q, k, v, g, cnt, idx, scale, o, lse, s)
+                     : launch_attn<64>(q, k, v, g, cnt, idx, scale, o, lse, s);
+}
+
+template <int NPT>
+void launch_select(const double* S, const dbst::SelectGeo& sg, long long rows, uint32_t* bits, int32_t* cnt,
+                   int16_t* idx, cudaStream_t s) {
+  dbst::select_kernel<NPT><<<static_cast<unsigned>(rows), 256, 0, s>>>(S, sg, bits, cnt, idx);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dbst_status_string(int status) {
+  switch (status) {
+    case DBST_OK: return "ok";
+    case DBST_EINVAL: return "invalid argument";
+    case DBST_ECUDA: return "CUDA error";
+    case DBST_ETIMEOUT: return "device wait timed out";
+    case DBST_EBOUNDS: return "index list entry out of range";
+    default: return "unknown status";
+  }
+}
+
+dbst_status dbst_tile_reorder(const void* x, void* y, const dbst_geom* g, void* stream) {
+  return permute(x, y, g, stream, 1);
+}
+
+dbst_status dbst_tile_unreorder(const void* y, void* x, const dbst_geom* g, void* stream) {
+  return permute(y, x, g, stream, 0);
+}
+
+size_t dbst_mask_workspace_bytes(const dbst_geom* g) {
+  if (!geom_ok(g)) return 0;
+  return mask_workspace(g).total;
+}
+
+dbst_status dbst_build_block_mask(const void* q_tiled, const void* k_tiled, const dbst_geom* g, float p,
+                                  int sta_radius, uint32_t* mask_bits, int32_t* kv_count, int16_t* kv_idx,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  if (!geom_ok(g) || !q_tiled || !k_tiled || !mask_bits || !kv_count || !kv_idx || !workspace) return DBST_EINVAL;
+  if (!aligned16(q_tiled) || !aligned16(k_tiled) || !aligned16(mask_bits) || !aligned16(kv_count) ||
+      !aligned16(kv_idx) || !aligned16(workspace))
+    return DBST_EINVAL;
+  if (!(p > 0.0f && p <= 1.0f)) return DBST_EINVAL;   // also rejects NaN
+  const MaskWorkspace w = mask_workspace(g);
+  if (workspace_bytes < w.total) return DBST_EINVAL;
+  auto s = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  double* qp = reinterpret_cast<double*>(ws + w.qp);
+  double* kp = reinterpret_cast<double*>(ws + w.kp);
+  double* S = reinterpret_cast<double*>(ws + w.s);
+  const int NB = nblocks(g);
+  const long long bh = bh_count(g);
+  const long long nblk = bh * NB;
+
+  {  // 1. block mean-pool of q and k
+    long long grid = (2 * nblk * 32 + 255) / 256;
+    const long long cap = static_cast<long long>(sm_count()) * 8;
+    if (grid > cap) grid = cap;
+    const auto* qa = static_cast<const uint4*>(q_tiled);
+    const auto* ka = static_cast<const uint4*>(k_tiled);
+    if (g->D == 128)
+      dbst::pool_kernel<128><<<static_cast<unsigned>(grid), 256, 0, s>>>(qa, ka, qp, kp, nblk);
+    else
+      dbst::pool_kernel<64><<<static_cast<unsigned>(grid), 256, 0, s>>>(qa, ka, qp, kp, nblk);
+    if (cudaGetLastError() != cudaSuccess) return DBST_ECUDA;
+  }
+  {  // 2. pooled logits (float64)
+    const double scale = 1.0 / std::sqrt(static_cast<double>(g->D));
+    dim3 grid((NB + 63) / 64, (NB + 63) / 64, static_cast<unsigned>(bh));
+    if (bh > 65535) return DBST_EINVAL;
+    if (g->D == 128)
+      dbst::pooled_logits_kernel<128><<<grid, 256, 0, s>>>(qp, kp, S, NB, scale);
+    else
+      dbst::pooled_logits_kernel<64><<<grid, 256, 0, s>>>(qp, kp, S, NB, scale);
+    if (cudaGetLastError() != cudaSuccess) return DBST_ECUDA;
+  }
+  {  // 3. softmax + CDF selection + sliding-tile union + lists
+    dbst::SelectGeo sg;
+    sg.NB = NB;
+    sg.NW = (NB + 31) / 32;
+    sg.nX = g->X / g->tx;
+    sg.nY = g->Y / g->ty;
+    sg.sta_radius = sta_radius;
+    sg.p = static_cast<double>(p);
+    const long long rows = nblk;
+    if (NB <= 256) launch_select<1>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
+    else if (NB <= 512) launch_select<2>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
+    else if (NB <= 1024) launch_select<4>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
+    else if (NB <= 2048) launch_select<8>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
+    else launch_select<16>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
+  }
+  return launch_status();
+}
+
+dbst_status dbst_mask_from_bits(const uint32_t* bits, const dbst_geom* g, int32_t* kv_count, int16_t* kv_idx,
+                                void* stream) {
+  if (!geom_ok(g) || !bits || !kv_count || !kv_idx) return DBST_EINVAL;
+  if (!aligned16(bits) || !aligned16(kv_count) || !aligned16(kv_idx)) return DBST_EINVAL;
+  const int NB = nblocks(g);
+  const long long rows = bh_count(g) * NB;
+  long long grid = (rows * 32 + 255) / 256;
+  const long long cap = static_cast<long long>(sm_count()) * 8;
+  if (grid > cap) grid = cap;
+  dbst::bits_to_lists_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      bits, NB, (NB + 31) / 32, rows, kv_count, kv_idx);
+  return launch_status();
+}
+
+dbst_status dbst_block_sparse_attn(const void* q, const void* k, const void* v, const dbst_geom* g,
+                                   const int32_t* kv_count, const int16_t* kv_idx, float scale, void* o, float* lse,
+                                   void* stream) {
+  if (!kv_count || !kv_idx) return DBST_EINVAL;
+  if (!aligned16(kv_count) || !aligned16(kv_idx)) return DBST_EINVAL;
+  return attn_common(q, k, v, g, kv_count, kv_idx, scale, o, lse, stream);
+}
+
+dbst_status dbst_dense_attn(const void* q, const void* k, const void* v, const dbst_geom* g, float scale, void* o,
+                            float* lse, void* stream) {
+  return attn_common(q, k, v, g, nullptr, nullptr, scale, o, lse, stream);
+}
+
+dbst_status dbst_get_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DBST_ECUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, dbst::g_error_word, sizeof(word)) != cudaSuccess) return DBST_ECUDA;
+  if (word != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(dbst::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return DBST_ECUDA;
+  }
+  if (cudaGetLastError() != cudaSuccess) return DBST_ECUDA;
+  if (word == dbst::kErrTimeout) return DBST_ETIMEOUT;
+  if (word == dbst::kErrBounds) return DBST_EBOUNDS;
+  return word ? DBST_ECUDA : DBST_OK;
+}
+
+}  // extern "C"

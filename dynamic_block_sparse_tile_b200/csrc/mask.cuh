@@ -1,0 +1,362 @@
+// Adaptive block mask: block mean-pool, pooled score map, per-row CDF
+// selection, sliding-tile union and index-list expansion (NABLA page,
+// "Construction de Masque Adaptatif" and "Intégration Hybride avec STA").
+//
+// Precision: the pooled means are exact (64 bf16 values summed in float64),
+// the pooled logits, softmax and cumulative masses are float64, so the kept
+// set agrees with a float64 reference except where a cumulative mass sits
+// within rounding of p.
+#pragma once
+#include <cstdint>
+#include "ptx.cuh"
+
+namespace dbst {
+
+// ---------------------------------------------------------------------------
+// Block mean-pool: one warp per 64-token block; out[blk][c] = mean (float64).
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) pool_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
+                                                   double* __restrict__ qp, double* __restrict__ kp,
+                                                   long long nblocks) {
+  constexpr int CPR = D / 8;            // 16-byte chunks per token row
+  constexpr int RPW = 32 / CPR;         // token rows covered by one warp pass
+  const int lane = threadIdx.x & 31;
+  const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  const int ch = lane % CPR;
+  const int r0 = lane / CPR;
+  for (long long w = warp; w < 2 * nblocks; w += nwarps) {
+    const bool isk = w >= nblocks;
+    const long long b = isk ? w - nblocks : w;
+    const uint4* src = (isk ? k : q) + b * 64 * CPR;
+    double acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.0;
+#pragma unroll 8
+    for (int r = r0; r < 64; r += RPW) {
+      const uint4 v = ld_stream(src + r * CPR + ch);
+      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[2 * e] += static_cast<double>(__uint_as_float(u[e] << 16));
+        acc[2 * e + 1] += static_cast<double>(__uint_as_float(u[e] & 0xFFFF0000u));
+      }
+    }
+#pragma unroll
+    for (int off = CPR; off < 32; off <<= 1) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+    }
+    if (r0 == 0) {
+      double* out = (isk ? kp : qp) + b * D + ch * 8;
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        double2 pr = make_double2(acc[e] * (1.0 / 64.0), acc[e + 1] * (1.0 / 64.0));
+        reinterpret_cast<double2*>(out)[e / 2] = pr;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Pooled logits S[bh][i][j] = scale * <Qp_i, Kp_j> in float64.
+// 64 x 64 output tile per CTA, 256 threads, 4 x 4 outputs per thread.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) pooled_logits_kernel(const double* __restrict__ qp,
+                                                            const double* __restrict__ kp,
+                                                            double* __restrict__ S, int NB, double scale) {
+  constexpr int KC = 16;
+  __shared__ double As[KC][64 + 1];
+  __shared__ double Bs[KC][64 + 1];
+  const int bh = blockIdx.z;
+  const int i0 = blockIdx.y * 64, j0 = blockIdx.x * 64;
+  const double* Q = qp + static_cast<long long>(bh) * NB * D;
+  const double* K = kp + static_cast<long long>(bh) * NB * D;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  double acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+  for (int c0 = 0; c0 < D; c0 += KC) {
+    // 64 rows x 16 columns of each operand: 1024 values, 4 per thread
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int idx = threadIdx.x + e * 256;
+      const int row = idx / KC, col = idx % KC;
+      As[col][row] = (i0 + row < NB) ? Q[static_cast<long long>(i0 + row) * D + c0 + col] : 0.0;
+      Bs[col][row] = (j0 + row < NB) ? K[static_cast<long long>(j0 + row) * D + c0 + col] : 0.0;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int c = 0; c < KC; ++c) {
+      double a[4], b[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        a[e] = As[c][ty + 16 * e];
+        b[e] = Bs[c][tx + 16 * e];
+      }
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) acc[x][y] = fma(a[x], b[y], acc[x][y]);
+    }
+    __syncthreads();
+  }
+  double* out = S + static_cast<long long>(bh) * NB * NB;
+#pragma unroll
+  for (int x = 0; x < 4; ++x) {
+    const int i = i0 + ty + 16 * x;
+    if (i >= NB) continue;
+#pragma unroll
+    for (int y = 0; y < 4; ++y) {
+      const int j = j0 + tx + 16 * y;
+      if (j < NB) out[static_cast<long long>(i) * NB + j] = acc[x][y] * scale;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Per-row softmax + CDF selection + STA union + list expansion.
+// One CTA (256 threads) per row; thread t owns key blocks j = t + 256*u.
+// ---------------------------------------------------------------------------
+struct SelectGeo {
+  int NB, NW;          // blocks per (b,h); 32-bit mask words per row
+  int nX, nY;          // tile grid (for the sliding-tile neighbourhood)
+  int sta_radius;      // < 0: none
+  double p;            // CDF threshold; >= 1 keeps all
+};
+
+__device__ __forceinline__ double block_reduce_max(double v, double* red) {
+  for (int off = 16; off > 0; off >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, off));
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  double r = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) r = fmax(r, red[i]);
+  return r;
+}
+__device__ __forceinline__ double block_reduce_sum(double v, double* red) {
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  double r = 0.0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) r += red[i];
+  return r;
+}
+
+template <int NPT>
+__global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ S, SelectGeo g,
+                                                     uint32_t* __restrict__ bits, int32_t* __restrict__ count,
+                                                     int16_t* __restrict__ idx) {
+  __shared__ double red[8];
+  __shared__ double hist[256];
+  __shared__ int hcnt[256];
+  __shared__ unsigned long long s_prefix;
+  __shared__ int s_state;            // 0 searching, 1 threshold found, 2 keep all
+  __shared__ int s_shift;
+  __shared__ double s_above;
+  __shared__ int wcount[128 + 1];
+
+  const long long row = blockIdx.x;
+  const int i = static_cast<int>(row % g.NB);
+  const double* srow = S + row * g.NB;
+  const int t = threadIdx.x;
+
+  double a[NPT];
+  unsigned long long key[NPT];
+  double mx = -INFINITY;
+#pragma unroll
+  for (int u = 0; u < NPT; ++u) {
+    const int j = t + 256 * u;
+    a[u] = (j < g.NB) ? srow[j] : -INFINITY;
+    mx = fmax(mx, a[u]);
+  }
+  mx = block_reduce_max(mx, red);
+  double sum = 0.0;
+#pragma unroll
+  for (int u = 0; u < NPT; ++u) {
+    const int j = t + 256 * u;
+    a[u] = (j < g.NB) ? exp(a[u] - mx) : 0.0;
+    sum += a[u];
+  }
+  sum = block_reduce_sum(sum, red);
+#pragma unroll
+  for (int u = 0; u < NPT; ++u) {
+    const int j = t + 256 * u;
+    a[u] = a[u] / sum;
+    // descending A (top 48 bits of the non-negative double), ties -> lower j first
+    key[u] = (j < g.NB) ? (((static_cast<unsigned long long>(__double_as_longlong(a[u])) >> 16) << 16) |
+                           static_cast<unsigned long long>(0xFFFF - j))
+                        : 0ull;
+  }
+
+  // Radix select, most significant byte first: find the key of the k*-th
+  // largest element, i.e. the first element at which the cumulative mass of
+  // all larger keys plus its own reaches p.
+  if (t == 0) {
+    s_prefix = 0ull;
+    s_above = 0.0;
+    s_state = (g.p >= 1.0) ? 2 : 0;
+    s_shift = 64;
+  }
+  __syncthreads();
+  for (int shift = 56; shift >= 0 && s_state == 0; shift -= 8) {
+    hist[t] = 0.0;
+    hcnt[t] = 0;
+    __syncthreads();
+    const unsigned long long pre = s_prefix;
+#pragma unroll
+    for (int u = 0; u < NPT; ++u) {
+      const int j = t + 256 * u;
+      if (j < g.NB && (shift == 56 || (key[u] >> (shift + 8)) == pre)) {
+        const int d = static_cast<int>((key[u] >> shift) & 0xFF);
+        atomicAdd(&hist[d], a[u]);
+        atomicAdd(&hcnt[d], 1);
+      }
+    }
+    __syncthreads();
+    if (t < 32) {
+      // lane l scans bins 255-8l .. 248-8l (descending); suffix mass from the top
+      double m[8];
+      double local = 0.0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        m[e] = hist[255 - 8 * t - e];
+        local += m[e];
+      }
+      double incl = local;   // inclusive scan over lanes (lane 0 = highest bins)
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const double o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (t >= off) incl += o;
+      }
+      const double excl = incl - local;
+      const double need = g.p - s_above;
+      const unsigned ball = __ballot_sync(0xffffffffu, incl >= need);
+      if (ball == 0u) {
+        if (t == 0) s_state = 2;               // total mass below p (rounding): keep every block
+      } else {
+        const int L = __ffs(ball) - 1;
+        if (t == L) {
+          double cum = excl;
+          int e = 0;
+          for (; e < 8; ++e) {
+            if (cum + m[e] >= need) break;
+            cum += m[e];
+          }
+          if (e == 8) e = 7;
+          const int d = 255 - 8 * t - e;
+          s_above += cum;
+          s_prefix = (s_prefix << 8) | static_cast<unsigned long long>(d);
+          s_shift = shift;
+          if (hcnt[d] <= 1) s_state = 1;
+        }
+      }
+    }
+    __syncthreads();
+  }
+  const int state = s_state;
+  const unsigned long long pre = s_prefix;
+  const int shf = s_shift;
+
+  // tile coordinates of the query block (for the sliding-tile neighbourhood)
+  const int qx = i % g.nX, qy = (i / g.nX) % g.nY, qt = i / (g.nX * g.nY);
+  const int lane = t & 31, warp = t >> 5;
+  uint32_t words[NPT];
+  int mycount = 0;
+#pragma unroll
+  for (int u = 0; u < NPT; ++u) {
+    const int j = t + 256 * u;
+    bool keep = false;
+    if (j < g.NB) {
+      keep = (state == 2) || (state == 1 && (key[u] >> shf) >= pre) || (state == 0);
+      if (g.sta_radius >= 0) {
+        const int kx = j % g.nX, ky = (j / g.nX) % g.nY, kt = j / (g.nX * g.nY);
+        const int dmax = max(abs(kt - qt), max(abs(ky - qy), abs(kx - qx)));
+        keep = keep || (dmax <= g.sta_radius);
+      }
+    }
+    words[u] = __ballot_sync(0xffffffffu, keep);
+    mycount += __popc(words[u]);
+  }
+  // word index of (warp, u) is 8*u + warp; store words and per-word counts
+  uint32_t* brow = bits + row * g.NW;
+  if (lane == 0) {
+#pragma unroll
+    for (int u = 0; u < NPT; ++u) {
+      const int w = 8 * u + warp;
+      if (w < g.NW) {
+        brow[w] = words[u];
+        wcount[w] = __popc(words[u]);
+      }
+    }
+  }
+  __syncthreads();
+  if (t == 0) {
+    int run = 0;
+    for (int w = 0; w < g.NW; ++w) {
+      const int c = wcount[w];
+      wcount[w] = run;
+      run += c;
+    }
+    wcount[g.NW] = run;
+    count[row] = run;
+  }
+  __syncthreads();
+  int16_t* irow = idx + row * g.NB;
+#pragma unroll
+  for (int u = 0; u < NPT; ++u) {
+    const int w = 8 * u + warp;
+    if (w < g.NW && ((words[u] >> lane) & 1u)) {
+      const int pos = wcount[w] + __popc(words[u] & ((1u << lane) - 1u));
+      irow[pos] = static_cast<int16_t>(t + 256 * u);
+    }
+  }
+  (void)mycount;
+}
+
+// ---------------------------------------------------------------------------
+// Caller-supplied bitmask -> counts + ascending index lists.  One warp per row.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) bits_to_lists_kernel(const uint32_t* __restrict__ bits, int NB, int NW,
+                                                            long long rows, int32_t* __restrict__ count,
+                                                            int16_t* __restrict__ idx) {
+  const int lane = threadIdx.x & 31;
+  const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  for (long long row = warp; row < rows; row += nwarps) {
+    const uint32_t* brow = bits + row * NW;
+    int16_t* irow = idx + row * NB;
+    int base = 0;
+    for (int w0 = 0; w0 < NW; w0 += 32) {
+      const int w = w0 + lane;
+      uint32_t word = (w < NW) ? brow[w] : 0u;
+      if (w == NW - 1 && (NB & 31)) word &= (1u << (NB & 31)) - 1u;   // ignore bits past NB
+      const int c = __popc(word);
+      int incl = c;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      int pos = base + incl - c;
+      while (word) {
+        const int b = __ffs(word) - 1;
+        word &= word - 1u;
+        irow[pos++] = static_cast<int16_t>(w * 32 + b);
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) count[row] = base;
+  }
+}
+
+}  // namespace dbst

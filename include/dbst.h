@@ -1,0 +1,141 @@
+/*
+ * dbst.h — C ABI of the block-sparse tile attention library (libdbst.so).
+ *
+ * The library implements, on one NVIDIA B200 (sm_100a), the adaptive
+ * block-sparse attention described on the page "NABLA: Neighborhood Adaptive
+ * Block-Level Attention" (section "Méthodologie : NABLA"): tokens are
+ * reordered into 3-D tiles, tiles are mean-pooled, a pooled attention map is
+ * thresholded per row by its cumulative distribution, optionally unioned with
+ * a sliding-tile neighbourhood, and exact softmax attention runs over the kept
+ * tile pairs only.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All tensors are device memory owned by the caller, contiguous, row-major.
+ *   The library never allocates, frees or retains a pointer.
+ * - q, k, v, o are bf16 tensors of shape [B, H, N, D] (N = T*Y*X tokens);
+ *   "raster" order means token n = (t*Y + y)*X + x, "tiled" order is the
+ *   output of dbst_tile_reorder.
+ * - A tile (t x y x x = tt x ty x tx tokens) must hold exactly 64 tokens; it is
+ *   both the pooling block and the attention block ("block" below).
+ *   NB = N / 64 blocks per (b, h).  D must be 64 or 128.
+ * - Every device pointer must be 16-byte aligned.
+ * - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *   enqueued asynchronously; no entry point synchronises except
+ *   dbst_get_error.
+ * - Argument errors are detected on the host before any launch and return
+ *   DBST_EINVAL; nothing is enqueued in that case.  A failed launch returns
+ *   DBST_ECUDA.  Device-side faults that the kernels detect themselves (an
+ *   expired bounded wait, an out-of-range list entry) set a device error word
+ *   that dbst_get_error reports.
+ */
+#ifndef DBST_H
+#define DBST_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DBST_OK = 0,
+  DBST_EINVAL = 1,   /* bad argument; nothing was enqueued                      */
+  DBST_ECUDA = 2,    /* a CUDA runtime call or launch failed                     */
+  DBST_ETIMEOUT = 3, /* a kernel's bounded wait expired; its outputs are invalid */
+  DBST_EBOUNDS = 4   /* a kernel met an out-of-range index list entry            */
+} dbst_status;
+
+/* Shape of one call.  Token grid T x Y x X, tile tt x ty x tx (product 64). */
+typedef struct {
+  int B, H, D;
+  int T, Y, X;
+  int tt, ty, tx;
+} dbst_geom;
+
+/* Human-readable name of a status code (static string). */
+const char* dbst_status_string(int status);
+
+/*
+ * Token reorder ("Fractal Flattening", NABLA page, section "Méthodologie").
+ * y[b,h,r,:] = x[b,h,n(r),:] where tiled position
+ *   r = ((Tt*nY + Ty)*nX + Tx)*64 + (dt*ty + dy)*tx + dx
+ * holds raster token n = (t*Y + y)*X + x with Tt, dt = divmod(t, tt), etc.;
+ * nY = Y/ty, nX = X/tx.  Tiles come in raster order of tile coordinates, tokens
+ * inside a tile in raster order.  Bit-exact copy.  x and y must not overlap.
+ */
+dbst_status dbst_tile_reorder(const void* x_bf16, void* y_bf16, const dbst_geom* g, void* stream);
+
+/* Inverse of dbst_tile_reorder: tiled [B,H,N,D] -> raster [B,H,N,D]. */
+dbst_status dbst_tile_unreorder(const void* y_bf16, void* x_bf16, const dbst_geom* g, void* stream);
+
+/* Bytes of device scratch that dbst_build_block_mask needs for geometry g. */
+size_t dbst_mask_workspace_bytes(const dbst_geom* g);
+
+/*
+ * Adaptive block mask (NABLA page, "Construction de Masque Adaptatif" and
+ * "Intégration Hybride avec STA").
+ *   1. Qp, Kp = mean of each block's 64 tiled tokens (float64, exact).
+ *   2. A[i,:] = softmax_j(<Qp_i, Kp_j> / sqrt(D)) per (b, h), float64.
+ *   3. Row i keeps the smallest set of key blocks whose mass reaches p:
+ *      blocks sorted by A descending (ties: lower index first), keep the
+ *      shortest prefix whose cumulative sum is >= p; p == 1 keeps all.
+ *   4. If sta_radius >= 0, also keep every key block whose tile lies within
+ *      Chebyshev distance sta_radius of the query block's tile (clipped at
+ *      the grid edge, no wrap).
+ * Inputs: q_tiled, k_tiled bf16 [B,H,N,D] in tiled order.  p in (0, 1].
+ * Outputs (caller-allocated):
+ *   mask_bits [B,H,NB,ceil(NB/32)] uint32 — bit (j % 32) of word j/32 of row
+ *             (b,h,i) is 1 iff key block j is kept;
+ *   kv_count  [B,H,NB] int32 — kept blocks per row (>= 1);
+ *   kv_idx    [B,H,NB,NB] int16 — row (b,h,i) lists its kept key blocks in
+ *             ascending order in its first kv_count entries; the rest of the
+ *             row is left untouched.
+ * workspace: device scratch of at least dbst_mask_workspace_bytes(g) bytes,
+ * 16-byte aligned; contents on entry are ignored.
+ */
+dbst_status dbst_build_block_mask(const void* q_tiled, const void* k_tiled, const dbst_geom* g,
+                                  float p, int sta_radius,
+                                  uint32_t* mask_bits, int32_t* kv_count, int16_t* kv_idx,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Expansion of a caller-supplied block mask into the index lists that
+ * dbst_block_sparse_attn consumes ("Expansion", NABLA page).  mask_bits has
+ * the layout written by dbst_build_block_mask; rows may be empty.
+ */
+dbst_status dbst_mask_from_bits(const uint32_t* mask_bits, const dbst_geom* g,
+                                int32_t* kv_count, int16_t* kv_idx, void* stream);
+
+/*
+ * Block-sparse attention ("Expansion", NABLA page): for each (b,h) and query
+ * block i with kept key blocks S_i = kv_idx[b,h,i,0:kv_count[b,h,i]],
+ *   o[n,:]  = sum_{m in tokens(S_i)} softmax_m(scale * <q_n, k_m>) v[m,:]
+ *   lse[n]  = log(sum_{m in tokens(S_i)} exp(scale * <q_n, k_m>))   (natural log)
+ * for every query token n of block i; float32 softmax, bf16 output.  A row
+ * with kv_count == 0 produces o = 0 and lse = -inf.  q, k, v, o are tiled
+ * [B,H,N,D] bf16; lse is [B,H,N] float32 or NULL.  scale <= 0 selects
+ * 1/sqrt(D).  List entries must be in [0, NB); an entry outside makes the
+ * kernel skip it and report DBST_EBOUNDS through dbst_get_error.
+ */
+dbst_status dbst_block_sparse_attn(const void* q, const void* k, const void* v, const dbst_geom* g,
+                                   const int32_t* kv_count, const int16_t* kv_idx, float scale,
+                                   void* o, float* lse, void* stream);
+
+/* Dense attention over all N keys with the same kernel (every list = 0..NB-1). */
+dbst_status dbst_dense_attn(const void* q, const void* k, const void* v, const dbst_geom* g,
+                            float scale, void* o, float* lse, void* stream);
+
+/*
+ * Synchronises `stream`, then reports (and clears) the first device-side
+ * error any kernel of this library recorded since the last call, or a pending
+ * CUDA error.  DBST_OK if there was none.
+ */
+dbst_status dbst_get_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DBST_H */

@@ -1,0 +1,114 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared
+symbol, and rejects bad arguments before touching the GPU (no device needed)."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+import dynamic_block_sparse_tile_b200 as dbst
+from dynamic_block_sparse_tile_b200 import build as dbst_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dbst_build.build()
+    return dbst.load()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "dbst.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dbst_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(dbst.EXPORTS) == names
+
+
+def test_status_strings(lib):
+    assert lib.dbst_status_string(0) == b"ok"
+    assert b"invalid" in lib.dbst_status_string(1)
+    assert lib.dbst_status_string(99) == b"unknown status"
+
+
+GOOD = dict(B=1, H=2, D=128, grid=(4, 8, 16), tile=(2, 4, 8))
+
+
+def geom(**kw):
+    a = dict(GOOD)
+    a.update(kw)
+    return dbst.Geom.make(a["B"], a["H"], a["D"], a["grid"], a["tile"])
+
+
+BAD_GEOMS = [
+    dict(D=96), dict(D=256), dict(B=0), dict(H=-1),
+    dict(tile=(2, 4, 4)),                    # 32 tokens per tile
+    dict(grid=(3, 8, 16)),                   # 3 frames not divisible by tt=2
+    dict(grid=(4, 8, 12)),                   # 12 not divisible by tx=8
+    dict(grid=(2, 512, 512), tile=(1, 8, 8)),  # NB = 8192 > 4096
+]
+
+
+@pytest.mark.parametrize("bad", BAD_GEOMS)
+def test_bad_geometry_is_rejected_synchronously(lib, bad):
+    g = geom(**bad)
+    p = ctypes.c_void_p(1 << 20)
+    assert lib.dbst_tile_reorder(p, ctypes.c_void_p(1 << 30), ctypes.byref(g), None) == dbst.DBST_EINVAL
+    assert lib.dbst_mask_workspace_bytes(ctypes.byref(g)) == 0
+    assert lib.dbst_dense_attn(p, p, p, ctypes.byref(g), 0.0, p, None, None) == dbst.DBST_EINVAL
+    assert lib.dbst_mask_from_bits(p, ctypes.byref(g), p, p, None) == dbst.DBST_EINVAL
+
+
+def test_null_and_misaligned_pointers(lib):
+    g = geom()
+    a, b = ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 30)
+    assert lib.dbst_tile_reorder(None, b, ctypes.byref(g), None) == dbst.DBST_EINVAL
+    assert lib.dbst_tile_reorder(ctypes.c_void_p((1 << 20) + 8), b, ctypes.byref(g), None) == dbst.DBST_EINVAL
+    assert lib.dbst_tile_reorder(a, a, ctypes.byref(g), None) == dbst.DBST_EINVAL           # in place
+    assert lib.dbst_tile_unreorder(a, ctypes.c_void_p((1 << 20) + 64), ctypes.byref(g), None) == dbst.DBST_EINVAL
+    assert lib.dbst_block_sparse_attn(a, a, a, ctypes.byref(g), None, a, 0.0, a, None, None) == dbst.DBST_EINVAL
+    assert lib.dbst_block_sparse_attn(a, a, a, ctypes.byref(g), a, a, 0.0, a,
+                                      ctypes.c_void_p((1 << 20) + 2), None) == dbst.DBST_EINVAL
+    assert lib.dbst_dense_attn(a, a, a, ctypes.byref(g), float("nan"), a, None, None) == dbst.DBST_EINVAL
+    assert lib.dbst_tile_reorder(a, b, None, None) == dbst.DBST_EINVAL
+
+
+@pytest.mark.parametrize("p", [0.0, -0.5, 1.0000001, 2.0, float("nan")])
+def test_build_mask_rejects_p_outside_unit_interval(lib, p):
+    g = geom()
+    a = ctypes.c_void_p(1 << 20)
+    ws = lib.dbst_mask_workspace_bytes(ctypes.byref(g))
+    assert lib.dbst_build_block_mask(a, a, ctypes.byref(g), p, -1, a, a, a, a, ws, None) == dbst.DBST_EINVAL
+
+
+def test_build_mask_rejects_small_workspace(lib):
+    g = geom()
+    a = ctypes.c_void_p(1 << 20)
+    ws = lib.dbst_mask_workspace_bytes(ctypes.byref(g))
+    assert lib.dbst_build_block_mask(a, a, ctypes.byref(g), 0.9, -1, a, a, a, a, ws - 1, None) == dbst.DBST_EINVAL
+
+
+def test_workspace_size_formula(lib):
+    g = geom(B=2, H=3, D=64, grid=(8, 16, 16), tile=(1, 8, 8))
+    nb, bh = 32, 6
+
+    def up(x):
+        return (x + 255) // 256 * 256
+    expect = 2 * up(bh * nb * 64 * 8) + up(bh * nb * nb * 8)
+    assert lib.dbst_mask_workspace_bytes(ctypes.byref(g)) == expect
+
+
+def test_python_binding_validates_shapes_before_calling():
+    import torch
+    g = geom()
+    x = torch.zeros((1, 2, g.N, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        dbst.tile_reorder(x, g)          # not a CUDA tensor
