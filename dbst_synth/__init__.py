@@ -87,10 +87,10 @@ WORKLOADS: List[Workload] = [
              alpha=0.5, beta=0.5, f_rms=2.54, kmax=3, p_list=(0.9,), sta_radius=-1,
              unpadded=(21, 30, 52)),
     Workload("hunyuan", 3, B=1, H=24, D=128, grid=(34, 48, 80), tile=(2, 4, 8),
-             alpha=0.4, beta=0.6, f_rms=2.0, kmax=3, p_list=(0.9,), sta_radius=1,
+             alpha=0.4, beta=0.6, f_rms=2.6, kmax=3, p_list=(0.9,), sta_radius=1,
              unpadded=(33, 45, 80)),
     Workload("sweep", 4, B=2, H=16, D=128, grid=(16, 32, 32), tile=(2, 4, 8),
-             alpha=0.7, beta=0.3, f_rms=2.0, kmax=3,
+             alpha=0.7, beta=0.3, f_rms=1.6, kmax=3,
              p_list=(0.5, 0.7, 0.8, 0.9, 0.95, 0.99, 1.0), sta_radius=-1),
 ]
 
