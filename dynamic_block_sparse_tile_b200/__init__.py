@@ -18,7 +18,7 @@ from typing import Optional, Sequence, Tuple
 import torch
 
 __all__ = ["Geom", "DbstError", "lib_path", "load", "tile_reorder", "tile_unreorder", "mask_workspace_bytes",
-           "build_block_mask", "mask_from_bits", "block_sparse_attn", "dense_attn", "get_error", "EXPORTS"]
+           "build_block_mask", "build_block_mask_noalloc", "mask_from_bits", "block_sparse_attn", "dense_attn", "get_error", "EXPORTS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libdbst.so")
@@ -26,9 +26,10 @@ _LIB_PATH = os.path.join(_HERE, "libdbst.so")
 # Every symbol declared in include/dbst.h.
 EXPORTS = ("dbst_status_string", "dbst_tile_reorder", "dbst_tile_unreorder", "dbst_mask_workspace_bytes",
            "dbst_build_block_mask", "dbst_mask_from_bits", "dbst_block_sparse_attn", "dbst_dense_attn",
-           "dbst_get_error")
+           "dbst_get_error", "dbst_build_block_mask_noalloc")
 
-DBST_OK, DBST_EINVAL, DBST_ECUDA, DBST_ETIMEOUT, DBST_EBOUNDS = 0, 1, 2, 3, 4
+DBST_OK, DBST_EINVAL, DBST_ECUDA, DBST_ETIMEOUT, DBST_EBOUNDS, DBST_ETOOLARGE = 0, 1, 2, 3, 4, 5
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class DbstError(RuntimeError):
@@ -86,6 +87,8 @@ def load() -> ctypes.CDLL:
     lib.dbst_block_sparse_attn.restype = i32
     lib.dbst_dense_attn.argtypes, lib.dbst_dense_attn.restype = [vp, vp, vp, gp, f32, vp, vp, vp], i32
     lib.dbst_get_error.argtypes, lib.dbst_get_error.restype = [vp], i32
+    lib.dbst_build_block_mask_noalloc.argtypes = [vp, vp, gp, f32, i32, vp, vp, vp, vp]
+    lib.dbst_build_block_mask_noalloc.restype = i32
     _lib = lib
     return lib
 
@@ -161,6 +164,29 @@ def build_block_mask(q_tiled: torch.Tensor, k_tiled: torch.Tensor, g: Geom, p: f
                                         _ptr(bits), _ptr(cnt), _ptr(idx), _ptr(workspace),
                                         workspace.numel() * workspace.element_size(), _stream()),
            "dbst_build_block_mask")
+    return bits, cnt, idx
+
+
+def build_block_mask_noalloc(q_tiled: torch.Tensor, k_tiled: torch.Tensor, g: Geom, p: float,
+                             sta_radius: int = -1, out=None):
+    """Adaptive block mask without a workspace argument (``dbst_build_block_mask_noalloc``).
+
+    For callers that cannot allocate device memory: the library's fixed
+    static scratch (``NOALLOC_SCRATCH_BYTES``) is used instead.  Output
+    tensors are still the caller's (pass ``out`` to avoid allocating them here).
+    """
+    _need(q_tiled, torch.bfloat16, _qkv_shape(g), "q_tiled")
+    _need(k_tiled, torch.bfloat16, _qkv_shape(g), "k_tiled")
+    dev = q_tiled.device
+    if out is None:
+        bits = torch.empty((g.B, g.H, g.NB, g.NW), dtype=torch.int32, device=dev)
+        cnt = torch.empty((g.B, g.H, g.NB), dtype=torch.int32, device=dev)
+        idx = torch.empty((g.B, g.H, g.NB, g.NB), dtype=torch.int16, device=dev)
+    else:
+        bits, cnt, idx = out
+    _check(load().dbst_build_block_mask_noalloc(_ptr(q_tiled), _ptr(k_tiled), ctypes.byref(g), float(p),
+                                                int(sta_radius), _ptr(bits), _ptr(cnt), _ptr(idx), _stream()),
+           "dbst_build_block_mask_noalloc")
     return bits, cnt, idx
 
 

@@ -189,6 +189,7 @@ const char* dbst_status_string(int status) {
     case DBST_ECUDA: return "CUDA error";
     case DBST_ETIMEOUT: return "device wait timed out";
     case DBST_EBOUNDS: return "index list entry out of range";
+    case DBST_ETOOLARGE: return "problem exceeds the static scratch of the allocation-free entry point";
     default: return "unknown status";
   }
 }
@@ -307,3 +308,42 @@ dbst_status dbst_get_error(void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free mask build: the workspace is a fixed static device array.
+// ---------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[DBST_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the static scratch on the current device, looked up once
+// per device.  In host code the array's name is only a host-side stand-in, so
+// the address must come from cudaGetSymbolAddress.
+void* scratch_for_current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_scratch_ptr[dev] = ptr;
+  }
+  return g_scratch_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" dbst_status dbst_build_block_mask_noalloc(const void* q_tiled, const void* k_tiled, const dbst_geom* g,
+                                                     float p, int sta_radius, uint32_t* mask_bits,
+                                                     int32_t* kv_count, int16_t* kv_idx, void* stream) {
+  if (!geom_ok(g)) return DBST_EINVAL;
+  if (mask_workspace(g).total > static_cast<size_t>(DBST_NOALLOC_SCRATCH_BYTES)) return DBST_ETOOLARGE;
+  void* scratch = scratch_for_current_device();
+  if (scratch == nullptr) return DBST_ECUDA;
+  return dbst_build_block_mask(q_tiled, k_tiled, g, p, sta_radius, mask_bits, kv_count, kv_idx, scratch,
+                               DBST_NOALLOC_SCRATCH_BYTES, stream);
+}

@@ -44,7 +44,8 @@ typedef enum {
   DBST_EINVAL = 1,   /* bad argument; nothing was enqueued                      */
   DBST_ECUDA = 2,    /* a CUDA runtime call or launch failed                     */
   DBST_ETIMEOUT = 3, /* a kernel's bounded wait expired; its outputs are invalid */
-  DBST_EBOUNDS = 4   /* a kernel met an out-of-range index list entry            */
+  DBST_EBOUNDS = 4,  /* a kernel met an out-of-range index list entry            */
+  DBST_ETOOLARGE = 5 /* the problem needs more scratch than the fixed static area */
 } dbst_status;
 
 /* Shape of one call.  Token grid T x Y x X, tile tt x ty x tx (product 64). */
@@ -126,6 +127,37 @@ dbst_status dbst_block_sparse_attn(const void* q, const void* k, const void* v, 
 /* Dense attention over all N keys with the same kernel (every list = 0..NB-1). */
 dbst_status dbst_dense_attn(const void* q, const void* k, const void* v, const dbst_geom* g,
                             float scale, void* o, float* lse, void* stream);
+
+/*
+ * Allocation-free variant of dbst_build_block_mask.  The paper has no
+ * counterpart: this entry point exists for callers that cannot call
+ * cudaMalloc or hand the library a workspace — for example a serving loop or
+ * plugin host that owns all device memory, forbids allocation once it is
+ * running (cudaMalloc may synchronise the device and fragments the host's own
+ * pool) and has no spare buffer to lend.
+ *
+ * It computes exactly what dbst_build_block_mask computes, with the same
+ * arguments minus the workspace.  The scratch it needs lives in a fixed
+ * static device array of DBST_NOALLOC_SCRATCH_BYTES (64 MiB) inside the
+ * library; every GPU that loads the library holds that array until the
+ * process exits.  A geometry whose dbst_mask_workspace_bytes exceeds it is
+ * rejected with DBST_ETOOLARGE before anything is enqueued (the tiny, small
+ * and B=2/H=16/N=16384 shapes fit; the Wan-like and HunyuanVideo-like shapes
+ * do not).  The call allocates nothing: no cudaMalloc, no cudaFree, no
+ * allocating library routine.
+ *
+ * Set-up: the first call on each device (with that device current) looks up
+ * the array's device address once; make that first call before any stream
+ * capture begins.  All calls share the one array and it keeps the last call's
+ * contents; nothing in it needs to start at zero.  Two calls whose kernels
+ * overlap on the GPU (different streams without ordering between them) race
+ * on the array and produce undefined masks: order them on one stream.
+ */
+#define DBST_NOALLOC_SCRATCH_BYTES (64u << 20)
+dbst_status dbst_build_block_mask_noalloc(const void* q_tiled, const void* k_tiled, const dbst_geom* g,
+                                          float p, int sta_radius,
+                                          uint32_t* mask_bits, int32_t* kv_count, int16_t* kv_idx,
+                                          void* stream);
 
 /*
  * Synchronises `stream`, then reports (and clears) the first device-side
