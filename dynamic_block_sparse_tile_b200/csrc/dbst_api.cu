@@ -157,7 +157,7 @@ dbst_status launch_attn(const void* q, const void* k, const void* v, const dbst_
   if (attr != cudaSuccess) return DBST_ECUDA;
   const long long grid = bh_count(g) * p.NB;
   if (grid >= (1ll << 31)) return DBST_EINVAL;
-  dbst::sparse_attn_kernel<D><<<static_cast<unsigned>(grid), 256, smem, s>>>(tq, tk, tv, p);
+  dbst::sparse_attn_kernel<D><<<static_cast<unsigned>(grid), dbst::kAttnThreads, smem, s>>>(tq, tk, tv, p);
   return launch_status();
 }
 
@@ -173,9 +173,14 @@ dbst_status attn_common(const void* q, const void* k, const void* v, const dbst_
 }
 
 template <int NPT>
-void launch_select(const double* S, const dbst::SelectGeo& sg, long long rows, uint32_t* bits, int32_t* cnt,
+bool launch_select(const double* S, const dbst::SelectGeo& sg, long long rows, uint32_t* bits, int32_t* cnt,
                    int16_t* idx, cudaStream_t s) {
-  dbst::select_kernel<NPT><<<static_cast<unsigned>(rows), 256, 0, s>>>(S, sg, bits, cnt, idx);
+  const int smem = 256 * NPT * 16;   // sort keys + masses
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(dbst::select_kernel<NPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return false;
+  dbst::select_kernel<NPT><<<static_cast<unsigned>(rows), 256, smem, s>>>(S, sg, bits, cnt, idx);
+  return true;
 }
 
 }  // namespace
@@ -257,11 +262,13 @@ dbst_status dbst_build_block_mask(const void* q_tiled, const void* k_tiled, cons
     sg.sta_radius = sta_radius;
     sg.p = static_cast<double>(p);
     const long long rows = nblk;
-    if (NB <= 256) launch_select<1>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
-    else if (NB <= 512) launch_select<2>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
-    else if (NB <= 1024) launch_select<4>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
-    else if (NB <= 2048) launch_select<8>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
-    else launch_select<16>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
+    bool ok;
+    if (NB <= 256) ok = launch_select<1>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
+    else if (NB <= 512) ok = launch_select<2>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
+    else if (NB <= 1024) ok = launch_select<4>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
+    else if (NB <= 2048) ok = launch_select<8>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
+    else ok = launch_select<16>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
+    if (!ok) return DBST_ECUDA;
   }
   return launch_status();
 }

@@ -121,6 +121,16 @@ __global__ void __launch_bounds__(256) pooled_logits_kernel(const double* __rest
 // ---------------------------------------------------------------------------
 // Per-row softmax + CDF selection + STA union + list expansion.
 // One CTA (256 threads) per row; thread t owns key blocks j = t + 256*u.
+//
+// Selection: every block gets a 64-bit key that orders the row by A
+// descending with ties to the lower index,
+//   key = [octave of A: 8 bits][top 40 mantissa bits of A][0xFFFF - j],
+// the keys are sorted descending with a shared-memory bitonic network, the
+// masses are prefix-summed in that order (float64), and the first position
+// whose cumulative mass reaches p fixes the threshold key.  Values below
+// 2^-255 share octave 0; they are never at the threshold for p < 1, since the
+// mass above them exceeds 1 - NB * 2^-255.  Values equal in their top 40
+// mantissa bits count as ties.
 // ---------------------------------------------------------------------------
 struct SelectGeo {
   int NB, NW;          // blocks per (b,h); 32-bit mask words per row
@@ -152,23 +162,32 @@ __device__ __forceinline__ double block_reduce_sum(double v, double* red) {
   return r;
 }
 
+__device__ __forceinline__ unsigned long long select_key(double a, int j) {
+  const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(a));
+  const int e = static_cast<int>(b >> 52) - 768;                 // A in (0,1]: biased exponent <= 1023
+  const unsigned long long oct = static_cast<unsigned long long>(e < 0 ? 0 : e);
+  const unsigned long long man = (b & ((1ull << 52) - 1)) >> 12;  // top 40 mantissa bits
+  return (oct << 56) | (man << 16) | static_cast<unsigned long long>(0xFFFF - j);
+}
+
+// dynamic shared memory: keys [256*NPT] u64, masses [256*NPT] f64
 template <int NPT>
 __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ S, SelectGeo g,
                                                      uint32_t* __restrict__ bits, int32_t* __restrict__ count,
                                                      int16_t* __restrict__ idx) {
+  constexpr int NP2 = 256 * NPT;
+  extern __shared__ __align__(16) unsigned char sel_smem[];
+  unsigned long long* s_key = reinterpret_cast<unsigned long long*>(sel_smem);
+  double* s_a = reinterpret_cast<double*>(sel_smem + NP2 * 8);
   __shared__ double red[8];
-  __shared__ double hist[256];
-  __shared__ int hcnt[256];
-  __shared__ unsigned long long s_prefix;
-  __shared__ int s_state;            // 0 searching, 1 threshold found, 2 keep all
-  __shared__ int s_shift;
-  __shared__ double s_above;
+  __shared__ double wsum[8];
+  __shared__ int s_first;
   __shared__ int wcount[128 + 1];
 
   const long long row = blockIdx.x;
   const int i = static_cast<int>(row % g.NB);
   const double* srow = S + row * g.NB;
-  const int t = threadIdx.x;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
 
   double a[NPT];
   unsigned long long key[NPT];
@@ -192,92 +211,78 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
   for (int u = 0; u < NPT; ++u) {
     const int j = t + 256 * u;
     a[u] = a[u] / sum;
-    // descending A (top 48 bits of the non-negative double), ties -> lower j first
-    key[u] = (j < g.NB) ? (((static_cast<unsigned long long>(__double_as_longlong(a[u])) >> 16) << 16) |
-                           static_cast<unsigned long long>(0xFFFF - j))
-                        : 0ull;
+    key[u] = (j < g.NB) ? select_key(a[u], j) : 0ull;
+    s_key[j] = key[u];
+    s_a[j] = a[u];
   }
 
-  // Radix select, most significant byte first: find the key of the k*-th
-  // largest element, i.e. the first element at which the cumulative mass of
-  // all larger keys plus its own reaches p.
-  if (t == 0) {
-    s_prefix = 0ull;
-    s_above = 0.0;
-    s_state = (g.p >= 1.0) ? 2 : 0;
-    s_shift = 64;
-  }
-  __syncthreads();
-  for (int shift = 56; shift >= 0 && s_state == 0; shift -= 8) {
-    hist[t] = 0.0;
-    hcnt[t] = 0;
+  unsigned long long thr = 0ull;   // keep key >= thr (0 keeps all)
+  if (g.p < 1.0) {
     __syncthreads();
-    const unsigned long long pre = s_prefix;
+    // bitonic sort, descending
+    for (int k = 2; k <= NP2; k <<= 1) {
+      for (int jj = k >> 1; jj > 0; jj >>= 1) {
+#pragma unroll
+        for (int e = 0; e < NPT / 2 + (NPT == 1); ++e) {
+          const int pi = t + 256 * e;
+          if (pi < NP2 / 2) {
+            const int lo = 2 * pi - (pi & (jj - 1));
+            const int hi = lo + jj;
+            const unsigned long long x = s_key[lo], y = s_key[hi];
+            const bool desc = (lo & k) == 0;
+            if (desc ? (x < y) : (x > y)) {
+              s_key[lo] = y;
+              s_key[hi] = x;
+            }
+          }
+        }
+        __syncthreads();
+      }
+    }
+    // masses in sorted order, prefix-summed: thread t owns sorted positions [t*NPT, (t+1)*NPT)
+    double m[NPT];
+    double local = 0.0;
 #pragma unroll
     for (int u = 0; u < NPT; ++u) {
-      const int j = t + 256 * u;
-      if (j < g.NB && (shift == 56 || (key[u] >> (shift + 8)) == pre)) {
-        const int d = static_cast<int>((key[u] >> shift) & 0xFF);
-        atomicAdd(&hist[d], a[u]);
-        atomicAdd(&hcnt[d], 1);
+      const int r = t * NPT + u;
+      m[u] = (r < g.NB) ? s_a[0xFFFF - static_cast<int>(s_key[r] & 0xFFFFull)] : 0.0;
+      local += m[u];
+    }
+    double incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const double o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    if (t == 0) s_first = 0x7FFFFFFF;
+    __syncthreads();
+    double before = incl - local;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    double c = before;
+#pragma unroll
+    for (int u = 0; u < NPT; ++u) {
+      const int r = t * NPT + u;
+      c += m[u];
+      if (r < g.NB && c >= g.p) {
+        atomicMin(&s_first, r);
+        break;
       }
     }
     __syncthreads();
-    if (t < 32) {
-      // lane l scans bins 255-8l .. 248-8l (descending); suffix mass from the top
-      double m[8];
-      double local = 0.0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        m[e] = hist[255 - 8 * t - e];
-        local += m[e];
-      }
-      double incl = local;   // inclusive scan over lanes (lane 0 = highest bins)
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const double o = __shfl_up_sync(0xffffffffu, incl, off);
-        if (t >= off) incl += o;
-      }
-      const double excl = incl - local;
-      const double need = g.p - s_above;
-      const unsigned ball = __ballot_sync(0xffffffffu, incl >= need);
-      if (ball == 0u) {
-        if (t == 0) s_state = 2;               // total mass below p (rounding): keep every block
-      } else {
-        const int L = __ffs(ball) - 1;
-        if (t == L) {
-          double cum = excl;
-          int e = 0;
-          for (; e < 8; ++e) {
-            if (cum + m[e] >= need) break;
-            cum += m[e];
-          }
-          if (e == 8) e = 7;
-          const int d = 255 - 8 * t - e;
-          s_above += cum;
-          s_prefix = (s_prefix << 8) | static_cast<unsigned long long>(d);
-          s_shift = shift;
-          if (hcnt[d] <= 1) s_state = 1;
-        }
-      }
-    }
-    __syncthreads();
+    const int first = s_first;
+    thr = (first < g.NB) ? s_key[first] : 0ull;   // no crossing (rounding): keep every block
   }
-  const int state = s_state;
-  const unsigned long long pre = s_prefix;
-  const int shf = s_shift;
 
   // tile coordinates of the query block (for the sliding-tile neighbourhood)
   const int qx = i % g.nX, qy = (i / g.nX) % g.nY, qt = i / (g.nX * g.nY);
-  const int lane = t & 31, warp = t >> 5;
   uint32_t words[NPT];
-  int mycount = 0;
 #pragma unroll
   for (int u = 0; u < NPT; ++u) {
     const int j = t + 256 * u;
     bool keep = false;
     if (j < g.NB) {
-      keep = (state == 2) || (state == 1 && (key[u] >> shf) >= pre) || (state == 0);
+      keep = key[u] >= thr;
       if (g.sta_radius >= 0) {
         const int kx = j % g.nX, ky = (j / g.nX) % g.nY, kt = j / (g.nX * g.nY);
         const int dmax = max(abs(kt - qt), max(abs(ky - qy), abs(kx - qx)));
@@ -285,7 +290,6 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
       }
     }
     words[u] = __ballot_sync(0xffffffffu, keep);
-    mycount += __popc(words[u]);
   }
   // word index of (warp, u) is 8*u + warp; store words and per-word counts
   uint32_t* brow = bits + row * g.NW;
@@ -303,9 +307,9 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
   if (t == 0) {
     int run = 0;
     for (int w = 0; w < g.NW; ++w) {
-      const int c = wcount[w];
+      const int cw = wcount[w];
       wcount[w] = run;
-      run += c;
+      run += cw;
     }
     wcount[g.NW] = run;
     count[row] = run;
@@ -320,7 +324,6 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
       irow[pos] = static_cast<int16_t>(t + 256 * u);
     }
   }
-  (void)mycount;
 }
 
 // ---------------------------------------------------------------------------
