@@ -38,6 +38,7 @@ constexpr int kSoftWG = 4;                       // softmax warpgroups
 constexpr int kCols = 64 / kSoftWG;              // query columns per softmax warpgroup
 constexpr int kAttnThreads = 128 + 128 * kSoftWG;
 constexpr float kRescaleLog2 = 16.0f;
+constexpr int kSBufs = 4;                        // S^T buffers in TMEM (tile t uses buffer t % 4)
 
 struct AttnParams {
   const int32_t* kv_count;   // [BH*NB]; null => dense (every list is 0..NB-1)
@@ -72,9 +73,9 @@ enum {
   BAR_KEMPTY = BAR_KFULL + kKSlots,
   BAR_VFULL = BAR_KEMPTY + kKSlots,
   BAR_VEMPTY = BAR_VFULL + kVSlots,
-  BAR_SFULL = BAR_VEMPTY + kVSlots,   // + 2
-  BAR_SEMPTY = BAR_SFULL + 2,         // one arrival per softmax thread
-  BAR_PFULL = BAR_SEMPTY + 2,         // one arrival per softmax thread
+  BAR_SFULL = BAR_VEMPTY + kVSlots,   // + kSBufs
+  BAR_SEMPTY = BAR_SFULL + kSBufs,    // one arrival per softmax thread
+  BAR_PFULL = BAR_SEMPTY + kSBufs,    // one arrival per softmax thread
   BAR_PEMPTY = BAR_PFULL + 2,
   BAR_OFULL = BAR_PEMPTY + 2,
   BAR_DRAIN = BAR_OFULL + 1,
@@ -136,7 +137,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (tid == 0) {
     for (int b = 0; b < BAR_COUNT; ++b) {
       uint32_t cnt = 1;
-      if (b == BAR_SEMPTY || b == BAR_SEMPTY + 1 || b == BAR_PFULL || b == BAR_PFULL + 1) cnt = 128 * kSoftWG;
+      if ((b >= BAR_SEMPTY && b < BAR_SEMPTY + kSBufs) || b == BAR_PFULL || b == BAR_PFULL + 1) cnt = 128 * kSoftWG;
       mbar_init(bar(b), cnt);
     }
     fence_mbar_init();
@@ -175,7 +176,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int T = (n + 1) >> 1;   // key tiles of two blocks
 
   if (warp == 2) {
-    tmem_alloc(sbase + AttnSmem::kMisc, 256);
+    tmem_alloc(sbase + AttnSmem::kMisc, 512);
     tmem_relinquish();
   }
   if (D == 64) {   // V^T is padded to M = 128 rows of head dim with zeros
@@ -189,8 +190,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_misc[0];
-  const uint32_t tS[2] = {tmem + 0u, tmem + 64u};
-  const uint32_t tO = tmem + 128u;
+  const uint32_t tS0 = tmem;              // S^T buffer k at TMEM columns 64k
+  const uint32_t tO = tmem + 256u;
 
   auto tile_rows = [&](int t, int32_t& y0, int32_t& y1) {
     const int j0 = s_list[2 * t];
@@ -253,16 +254,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       return __all_sync(0xffffffffu, mbar_wait(bar(slot), parity));
     };
     auto issue_s = [&](int t) -> bool {
-      const int s = t % kKSlots, b = t & 1;
+      const int s = t % kKSlots, b = t % kSBufs;
       if (!wait_all(BAR_KFULL + s, (t / kKSlots) & 1)) return false;
-      if (t >= 2 && !wait_all(BAR_SEMPTY + b, ((t >> 1) - 1) & 1)) return false;
+      if (t >= kSBufs && !wait_all(BAR_SEMPTY + b, ((t / kSBufs) - 1) & 1)) return false;
       tc_fence_after();
       const uint64_t ka = dK + static_cast<uint64_t>((s * AttnSmem::kTile) >> 4);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
         const uint32_t qoff = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
-        umma_f16_elect(tS[b], ka + off, dQ + qoff, idS, kk > 0 ? 1u : 0u);
+        umma_f16_elect(tS0 + 64u * b, ka + off, dQ + qoff, idS, kk > 0 ? 1u : 0u);
       }
       umma_commit_elect(bar(BAR_SFULL + b));
       umma_commit_elect(bar(BAR_KEMPTY + s));
@@ -315,36 +316,63 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       lpart[c] = 0.0f;
       mref[c] = 0.0f;
     }
+    uint8_t* const prow_base = sm + AttnSmem::kP + r * 128;
+    // P = 2^min(d, kRescaleLog2): per-query sums and this warpgroup's chunk of P^T row r (128-byte
+    // swizzle).  The clamp only bites on tiles that trigger a rescale; their contributions are then
+    // subtracted again, each at most 2^kRescaleLog2 and added to a sum that is rescaled by at least
+    // that factor, so the sum keeps its relative accuracy.
+    auto emit_p = [&](int b, const float (&d)[kCols], float sign) {
+      uint32_t pk[kCols / 2];
+#pragma unroll
+      for (int c = 0; c < kCols / 2; ++c) {
+        const float p0 = fast_exp2(fminf(d[2 * c], kRescaleLog2));
+        const float p1 = fast_exp2(fminf(d[2 * c + 1], kRescaleLog2));
+        lpart[2 * c] = fmaf(sign, p0, lpart[2 * c]);
+        lpart[2 * c + 1] = fmaf(sign, p1, lpart[2 * c + 1]);
+        pk[c] = pack_bf16x2(p0, p1);
+      }
+      if (sign > 0.0f) {
+        uint8_t* prow = prow_base + b * AttnSmem::kPBuf;
+#pragma unroll
+        for (int cc = 0; cc < kCols / 8; ++cc) {
+          const int phys = (kCols / 8 * wg + cc) ^ (r & 7);
+          *reinterpret_cast<uint4*>(prow + phys * 16) =
+              make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+        }
+      }
+    };
     for (int t = 0; t < T; ++t) {
       const int b = t & 1;
-      bool bad = !mbar_wait(bar(BAR_SFULL + b), (t >> 1) & 1);
+      const int sb = t % kSBufs;
+      bool bad = !mbar_wait(bar(BAR_SFULL + sb), (t / kSBufs) & 1);
+      // P^T buffer b is free once PV(t-2) has read it
+      if (t >= 2 && !mbar_wait(bar(BAR_PEMPTY + b), ((t - 2) >> 1) & 1)) bad = true;
       tc_fence_after();
       // d = scaled logit - reference max (log2 units); rows of an absent second block are -inf
       float d[kCols];
       {
         uint32_t u[kCols];
-        tmem_ld16(tS[b] + tl + c0, u);
+        tmem_ld16(tS0 + 64u * sb + tl + c0, u);
         tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < kCols; ++c) d[c] = fmaf(__uint_as_float(u[c]), sc, -mref[c]);
       }
-      tc_fence_before();
-      mbar_arrive(bar(BAR_SEMPTY + b));
       if (q >= 2 && 2 * t + 1 >= n) {
 #pragma unroll
         for (int c = 0; c < kCols; ++c) d[c] = -INFINITY;
       }
-      bool need = (t == 0);
+      // speculative pass with the current reference; the tile max decides whether it stands
+      float dmax = -INFINITY;
       if (t > 0) {
-        float dmax = d[0];
 #pragma unroll
-        for (int c = 1; c < kCols; ++c) dmax = fmaxf(dmax, d[c]);
-        need = dmax > kRescaleLog2;
+        for (int c = 0; c < kCols; ++c) dmax = fmaxf(dmax, d[c]);
+        emit_p(b, d, 1.0f);
       }
       if (bad) *wg_abort = 1;
-      need = wg_vote_or(wg, need || bad);
+      const bool need = wg_vote_or(wg, t == 0 || dmax > kRescaleLog2 || bad);
       if (*wg_abort) break;   // written before the vote by this warpgroup only: uniform
       if (need) {
+        if (t > 0) emit_p(b, d, -1.0f);   // undo the speculative sums
         // per-query max over this tile's 128 keys -> new reference, rescale factors
 #pragma unroll
         for (int c = 0; c < kCols; ++c) {
@@ -393,29 +421,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           tmem_st16(tO + tl + c0, ov);
           tmem_wait_st();
-          tc_fence_before();
         }
+        emit_p(b, d, 1.0f);
       }
-      // P = 2^d, per-query partial sums, bf16 pack
-      uint32_t pk[kCols / 2];
-#pragma unroll
-      for (int c = 0; c < kCols / 2; ++c) {
-        const float p0 = fast_exp2(d[2 * c]);
-        const float p1 = fast_exp2(d[2 * c + 1]);
-        lpart[2 * c] += p0;
-        lpart[2 * c + 1] += p1;
-        pk[c] = pack_bf16x2(p0, p1);
-      }
-      if (t >= 2 && !mbar_wait(bar(BAR_PEMPTY + b), ((t - 2) >> 1) & 1)) *wg_abort = 1;
-      // this warpgroup's kCols*2 bytes of P^T row r in the 128-byte-swizzled MN-major layout
-      uint8_t* prow = sm + AttnSmem::kP + b * AttnSmem::kPBuf + r * 128;
-#pragma unroll
-      for (int cc = 0; cc < kCols / 8; ++cc) {
-        const int phys = (kCols / 8 * wg + cc) ^ (r & 7);
-        *reinterpret_cast<uint4*>(prow + phys * 16) =
-            make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-      }
+      tc_fence_before();
       fence_async_smem();
+      mbar_arrive(bar(BAR_SEMPTY + sb));
       mbar_arrive(bar(BAR_PFULL + b));
     }
 
@@ -464,7 +475,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
