@@ -233,8 +233,8 @@ def masked_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, mask: np.ndarr
     then holds only those blocks, shape ``[len(rows), blk, D]`` /
     ``[len(rows), blk]``.  Otherwise the full ``[B, H, N, D]`` / ``[B, H, N]``.
     """
-    if q.dtype == np.uint16:
-        q, k, v = bf16_bits_to_f64(q), bf16_bits_to_f64(k), bf16_bits_to_f64(v)
+    # bf16 inputs are decoded one query block / key set at a time (bounded host memory)
+    dec = bf16_bits_to_f64 if q.dtype == np.uint16 else (lambda a: np.asarray(a, dtype=np.float64))
     B, H, N, D = q.shape
     NB = N // blk
     full = rows is None
@@ -247,9 +247,9 @@ def masked_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, mask: np.ndarr
         if kept.size == 0:
             continue
         tok = (kept[:, None] * blk + np.arange(blk)[None, :]).reshape(-1)
-        qi = np.asarray(q[b, h, i * blk:(i + 1) * blk], dtype=np.float64)
-        ks = np.asarray(k[b, h, tok], dtype=np.float64)
-        vs = np.asarray(v[b, h, tok], dtype=np.float64)
+        qi = dec(q[b, h, i * blk:(i + 1) * blk])
+        ks = dec(k[b, h, tok])
+        vs = dec(v[b, h, tok])
         s = (qi @ ks.T) * scale
         mx = s.max(axis=1, keepdims=True)
         e = np.exp(s - mx)

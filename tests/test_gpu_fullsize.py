@@ -1,0 +1,112 @@
+"""Full-size parity on the Wan-like, HunyuanVideo-like and sweep workloads.
+
+Same call sequence as bench.py (reorder -> mask -> attention -> unreorder).
+The mask is compared with the oracle on every row of every head, with the
+near-threshold exemption.  Attention is compared on a seeded sample of
+query blocks that includes the first and the last one, against the oracle
+given the oracle's mask (and, for the mask the GPU built, against the oracle
+given that mask).
+"""
+import dataclasses
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import dbst_synth as S
+import oracle as O
+import dynamic_block_sparse_tile_b200 as dbst
+from tests import parity as P
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+
+@pytest.fixture(scope="module")
+def built():
+    from dynamic_block_sparse_tile_b200 import build
+    build.build()
+    dbst.load()
+    return True
+
+
+def run_path(w, p, sta, q, k, v):
+    """The bench's call sequence on device; returns tiled/raster outputs and the GPU mask."""
+    g = dbst.Geom.make(w.B, w.H, w.D, w.grid, w.tile)
+    qd, kd, vd = (P.bits_to_torch(a) for a in (q, k, v))
+    qt, kt, vt = (dbst.tile_reorder(x, g) for x in (qd, kd, vd))
+    bits, cnt, idx = dbst.build_block_mask(qt, kt, g, p, sta)
+    ot, lse = dbst.block_sparse_attn(qt, kt, vt, g, cnt, idx)
+    o = dbst.tile_unreorder(ot, g)
+    dbst.get_error()
+    return g, (qt, kt, vt), bits, cnt, idx, ot, lse, o
+
+
+def check_full(name, p, n_rows=24):
+    w = S.workload(name)
+    og = P.geometry(w)
+    q, k, v = S.make_qkv(w)
+    g, dev_t, bits, cnt, idx, ot, lse, o = run_path(w, p, w.sta_radius, q, k, v)
+    qt, kt, vt = (O.tile_reorder(a, og) for a in (q, k, v))
+    # reorder and unreorder, bit-exact
+    np.testing.assert_array_equal(P.torch_to_bits(dev_t[0]), qt)
+    np.testing.assert_array_equal(O.tile_unreorder(P.torch_to_bits(ot), og), P.torch_to_bits(o))
+    # mask on every row, near-threshold exemption
+    ref, A = P.oracle_mask_per_head(qt, kt, og, p, w.sta_radius)
+    got = P.unpack_mask(bits.cpu().numpy().view(np.uint32), og.NB)
+    hard, excused = P.mask_mismatches(got, ref, A, p, O.sta_mask(og, w.sta_radius))
+    assert not hard, f"{len(hard)} non-excused mask disagreements, first {hard[:5]}"
+    cnt_h, idx_h = cnt.cpu().numpy(), idx.cpu().numpy()
+    assert np.array_equal(cnt_h, got.sum(-1))
+    # attention on sampled query blocks, with the GPU's own lists (== oracle mask up to exemptions)
+    scale = 1.0 / math.sqrt(w.D)
+    rows = P.sample_rows(w.B, w.H, og.NB, n_rows, seed=7 + w.index)
+    for (b, h, i) in rows:
+        js = idx_h[b, h, i, :cnt_h[b, h, i]]
+        assert np.array_equal(js, np.nonzero(got[b, h, i])[0])
+    o_ref, lse_ref = O.masked_attention(qt, kt, vt, got, 64, scale, rows=rows)
+    o_gpu = P.gpu_rows(ot, rows)
+    max_abs, rel = P.attn_errors(o_gpu, o_ref)
+    assert max_abs <= P.ATTN_MAX_ABS and rel <= P.ATTN_REL_L2, (max_abs, rel)
+    lse_gpu = np.stack([lse[b, h, i * 64:(i + 1) * 64].cpu().numpy() for (b, h, i) in rows]).astype(np.float64)
+    assert np.max(np.abs(lse_gpu - lse_ref)) <= P.LSE_MAX_ABS
+    # given the oracle's own mask, the same rows again
+    words = torch.from_numpy(P.pack_mask(ref).view(np.int32)).cuda()
+    rc, ri = dbst.mask_from_bits(words, g)
+    ot2, _ = dbst.block_sparse_attn(*dev_t, g, rc, ri)
+    dbst.get_error()
+    o_ref2, _ = O.masked_attention(qt, kt, vt, ref, 64, scale, rows=rows)
+    max_abs2, rel2 = P.attn_errors(P.gpu_rows(ot2, rows), o_ref2)
+    assert max_abs2 <= P.ATTN_MAX_ABS and rel2 <= P.ATTN_REL_L2, (max_abs2, rel2)
+    return float(ref.mean()), len(excused)
+
+
+def test_wan_like_full_size(built):
+    kept, excused = check_full("wan", 0.9)
+    assert 0.05 < kept < 0.15
+
+
+def test_hunyuan_like_full_size(built):
+    kept, excused = check_full("hunyuan", 0.9, n_rows=16)
+    assert 0.03 < kept < 0.15
+
+
+@pytest.mark.parametrize("p", [0.5, 0.9, 1.0])
+def test_sweep_full_size(built, p):
+    kept, excused = check_full("sweep", p, n_rows=16)
+    if p >= 1.0:
+        assert kept == 1.0
+
+
+def test_sweep_dense_equals_p1(built):
+    w = S.workload("sweep")
+    q, k, v = S.make_qkv(w, heads=range(2), batches=range(1))
+    w2 = dataclasses.replace(w, B=1, H=2)
+    g = dbst.Geom.make(1, 2, w.D, w.grid, w.tile)
+    qt, kt, vt = (dbst.tile_reorder(P.bits_to_torch(a), g) for a in (q, k, v))
+    bits, cnt, idx = dbst.build_block_mask(qt, kt, g, 1.0, -1)
+    o1, l1 = dbst.block_sparse_attn(qt, kt, vt, g, cnt, idx)
+    o2, l2 = dbst.dense_attn(qt, kt, vt, g)
+    dbst.get_error()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    del w2
