@@ -46,6 +46,34 @@ def peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+def attn_source_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("attn.cuh", "ptx.cuh"):
+        with open(os.path.join(ROOT, "dynamic_block_sparse_tile_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: str, p: float):
+    """DRAM bytes per attention launch from the committed ncu summary, if it matches this kernel source."""
+    path = os.path.join(ROOT, "profiles", "sparse_attn_kernel_dram_traffic.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    for line in text.splitlines():
+        if line.startswith("| ") and f"`{workload}`" in line and f"p={p}" in line:
+            cells = [c.strip() for c in line.strip("|").split("|")]
+            try:
+                digest, total = cells[1].strip("`"), float(cells[4])
+            except (IndexError, ValueError):
+                continue
+            if digest == attn_source_digest():
+                return total
+    return None
+
+
 def workload_desc(w: S.Workload, p: float) -> str:
     return (f"{w.name}-like latent: B={w.B} H={w.H} D={w.D} grid={w.grid[0]}x{w.grid[1]}x{w.grid[2]} "
             f"(N={w.N}, {w.NB} blocks of {w.tile[0]}x{w.tile[1]}x{w.tile[2]}), p={p}, "
@@ -161,8 +189,10 @@ def run_reference(args, w, p):
         return 0
     vals, secs = [], []
     desc = ""
+    # bounded: about two minutes of oracle work for the whole run, however many steps
+    budget = args.ref_budget if args.ref_budget > 0 else max(2.0, 120.0 / (args.warmup + args.steps))
     for step in range(args.warmup + args.steps):
-        v, s, desc = oracle_sample(w, p, budget_s=args.ref_budget, seed=100 + step)
+        v, s, desc = oracle_sample(w, p, budget_s=budget, seed=100 + step)
         if step >= args.warmup:
             vals.append(v)
             secs.append(s)
@@ -178,6 +208,58 @@ def run_reference(args, w, p):
     return 0
 
 
+def run_sweep(args, w):
+    """Attention time and kept-block TFLOP/s against the kept fraction; dense attention at the same shape."""
+    import torch
+    import dynamic_block_sparse_tile_b200 as dbst
+    dbst.load()
+    g = dbst.Geom.make(w.B, w.H, w.D, w.grid, w.tile)
+    q, k, v = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda() for a in S.make_qkv(w))
+    qt, kt, vt = (dbst.tile_reorder(x, g) for x in (q, k, v))
+    ot = torch.empty_like(qt)
+    lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device="cuda")
+
+    def timed(fn, reps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    dense_ms = timed(lambda: dbst.dense_attn(qt, kt, vt, g), args.steps)
+    dense_flops = 4.0 * w.D * w.N * w.N * w.B * w.H
+    _, bf16, _, src = peaks()
+    rows = []
+    for p in w.p_list:
+        bits, cnt, idx = dbst.build_block_mask(qt, kt, g, p, w.sta_radius)
+        mask_ms = timed(lambda: dbst.build_block_mask(qt, kt, g, p, w.sta_radius), args.steps)
+        ms = timed(lambda: dbst.block_sparse_attn(qt, kt, vt, g, cnt, idx, 0.0, True, ot, lse), args.steps)
+        kept = int(cnt.sum().item())
+        fl = 4.0 * w.D * 64 * 64 * kept
+        rows.append({"p": p, "kept_fraction": kept / (g.B * g.H * g.NB * g.NB), "sparse_attn_ms": ms,
+                     "kept_tflops": fl / (ms * 1e-3) / 1e12, "frac_of_bf16_peak": fl / (ms * 1e-3) / 1e12 / bf16,
+                     "mask_build_ms": mask_ms, "speedup_vs_dense": dense_ms / ms})
+    dbst.get_error()
+    crossover = None
+    for r in rows:
+        if r["sparse_attn_ms"] >= dense_ms:
+            crossover = r["kept_fraction"]
+            break
+    out = {"sweep": workload_desc(w, float("nan")), "dense_attn_ms": dense_ms,
+           "dense_tflops": dense_flops / (dense_ms * 1e-3) / 1e12, "peak_source": src, "points": rows,
+           "dense_crossover_kept_fraction": crossover}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -187,13 +269,18 @@ def main():
     ap.add_argument("--workload", default="wan")
     ap.add_argument("--p", type=float, default=None)
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
-    ap.add_argument("--ref-budget", type=float, default=10.0, help="seconds of oracle work per reference step")
+    ap.add_argument("--ref-budget", type=float, default=0.0,
+                    help="seconds of oracle work per reference step (0: about 120 s over the whole run)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="sparsity sweep: attention ms/call and kept-block TFLOP/s per p, dense crossover")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     w = S.workload(args.workload)
     p = args.p if args.p is not None else w.p_list[0]
     if args.impl == "reference":
         return run_reference(args, w, p)
+    if args.sweep:
+        return run_sweep(args, S.workload("sweep") if args.workload == "wan" else w)
 
     import torch
     import torch.distributed as dist
@@ -317,7 +404,7 @@ def main():
         "sparse_attn_ms_per_call": attn_ms, "sparse_attn_tflops": attn_tflops,
         "mask_build_ms_per_call": mask_ms, "mask_build_gbs": mask_bytes / (mask_ms * 1e-3) / 1e9,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": bf16, "unit": "TFLOP/s",
-                     "frac": attn_tflops / bf16, "traffic": None,
+                     "frac": attn_tflops / bf16, "traffic": measured_traffic(w.name, p),
                      "peak_source": f"{src} bf16 burst; frac of sustained {attn_tflops / bf16_sus:.3f}",
                      "kernel": "sparse_attn_kernel<128>"},
         "mask_roofline": {"bound": "hbm", "achieved": mask_bytes / (mask_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
