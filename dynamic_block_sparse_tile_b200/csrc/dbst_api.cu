@@ -77,16 +77,18 @@ dbst_status permute(const void* src, void* dst, const dbst_geom* g, void* stream
   const char* b = static_cast<const char*>(dst);
   if (a < b + bytes && b < a + bytes) return DBST_EINVAL;   // overlapping buffers
   auto s = static_cast<cudaStream_t>(stream);
-  const long long chunks = rows * (g->D / 8);
-  long long grid = (chunks + 255) / 256;
-  const long long cap = static_cast<long long>(sm_count()) * 16;
-  if (grid > cap) grid = cap;
+  const long long bh = bh_count(g);
+  if (bh > 65535) return DBST_EINVAL;
+  const int N = static_cast<int>(tokens(g));
+  const int cpr = g->D / 8;                                   // 16-byte chunks per token row
+  const int rows_per_cta = 256 * dbst::kPermuteUnroll / cpr;  // token rows moved by one CTA
+  dim3 grid(static_cast<unsigned>((N + rows_per_cta - 1) / rows_per_cta), static_cast<unsigned>(bh));
   const auto* in = static_cast<const uint4*>(src);
   auto* out = static_cast<uint4*>(dst);
   if (g->D == 128)
-    dbst::tile_permute_kernel<4><<<static_cast<int>(grid), 256, 0, s>>>(in, out, tile_geo(g), rows, to_tiled);
+    dbst::tile_permute_kernel<4><<<grid, 256, 0, s>>>(in, out, tile_geo(g), to_tiled);
   else
-    dbst::tile_permute_kernel<3><<<static_cast<int>(grid), 256, 0, s>>>(in, out, tile_geo(g), rows, to_tiled);
+    dbst::tile_permute_kernel<3><<<grid, 256, 0, s>>>(in, out, tile_geo(g), to_tiled);
   return launch_status();
 }
 
@@ -262,10 +264,14 @@ dbst_status dbst_build_block_mask(const void* q_tiled, const void* k_tiled, cons
     sg.sta_radius = sta_radius;
     sg.p = static_cast<double>(p);
     const long long rows = nblk;
-    bool ok;
-    if (NB <= 256) ok = launch_select<1>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
-    else if (NB <= 512) ok = launch_select<2>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
-    else if (NB <= 1024) ok = launch_select<4>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
+    bool ok = true;
+    const unsigned wgrid = static_cast<unsigned>((rows * 32 + 127) / 128);   // one warp per row
+    if (NB <= 256) dbst::select_warp_kernel<8><<<wgrid, 128, 0, s>>>(S, sg, rows, mask_bits, kv_count, kv_idx);
+    else if (NB <= 384) dbst::select_warp_kernel<12><<<wgrid, 128, 0, s>>>(S, sg, rows, mask_bits, kv_count, kv_idx);
+    else if (NB <= 512) dbst::select_warp_kernel<16><<<wgrid, 128, 0, s>>>(S, sg, rows, mask_bits, kv_count, kv_idx);
+    else if (NB <= 640) dbst::select_warp_kernel<20><<<wgrid, 128, 0, s>>>(S, sg, rows, mask_bits, kv_count, kv_idx);
+    else if (NB <= 768) dbst::select_warp_kernel<24><<<wgrid, 128, 0, s>>>(S, sg, rows, mask_bits, kv_count, kv_idx);
+    else if (NB <= 1024) dbst::select_warp_kernel<32><<<wgrid, 128, 0, s>>>(S, sg, rows, mask_bits, kv_count, kv_idx);
     else if (NB <= 2048) ok = launch_select<8>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
     else ok = launch_select<16>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
     if (!ok) return DBST_ECUDA;

@@ -162,6 +162,8 @@ __device__ __forceinline__ double block_reduce_sum(double v, double* red) {
   return r;
 }
 
+__device__ __forceinline__ double p_of(const SelectGeo& g) { return g.p; }
+
 __device__ __forceinline__ unsigned long long select_key(double a, int j) {
   const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(a));
   const int e = static_cast<int>(b >> 52) - 768;                 // A in (0,1]: biased exponent <= 1023
@@ -324,6 +326,133 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
       irow[pos] = static_cast<int16_t>(t + 256 * u);
     }
   }
+}
+
+// ---------------------------------------------------------------------------
+// Same selection with one warp per row (rows of at most 32*NPT blocks): the
+// row lives in registers (lane l owns blocks j = l + 32u), and the threshold
+// key is found by a mass quickselect instead of a sort.  Each round picks a
+// live key as pivot and sums, over the warp, the mass of the live keys above
+// it; the answer lies above the pivot, is the pivot, or lies below it, and
+// the pivot always leaves the live set.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ double warp_sum_f64(double v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+__device__ __forceinline__ double warp_max_f64(double v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, off));
+  return v;
+}
+
+// Order-preserving 64-bit key of a row entry: the float64 logit (the softmax
+// keeps its order), top 48 bits, then 0xFFFF - j so that ties go to the lower
+// index.  Logits equal in their top 48 bits (relative difference below
+// 2^-36) count as ties.
+__device__ __forceinline__ unsigned long long logit_key(double s, int j) {
+  unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(s));
+  b = (b >> 63) ? ~b : (b | (1ull << 63));
+  return ((b >> 16) << 16) | static_cast<unsigned long long>(0xFFFF - j);
+}
+
+template <int NPT>
+__global__ void __launch_bounds__(128) select_warp_kernel(const double* __restrict__ S, SelectGeo g, long long rows,
+                                                          uint32_t* __restrict__ bits, int32_t* __restrict__ count,
+                                                          int16_t* __restrict__ idx) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (row >= rows) return;                      // whole warps only
+  const int i = static_cast<int>(row % g.NB);
+  const double* srow = S + row * g.NB;
+
+  // keys from the logits; unnormalised masses e^(s - max) in float32 (summed in float64)
+  float m[NPT];
+  unsigned long long key[NPT];
+  double mx = -INFINITY;
+#pragma unroll
+  for (int u = 0; u < NPT; ++u) {
+    const int j = lane + 32 * u;
+    const double sj = (j < g.NB) ? srow[j] : -INFINITY;
+    key[u] = (j < g.NB) ? logit_key(sj, j) : 0ull;
+    mx = fmax(mx, sj);
+    m[u] = static_cast<float>(sj);   // placeholder, replaced below
+  }
+  mx = warp_max_f64(mx);
+  double total = 0.0;
+#pragma unroll
+  for (int u = 0; u < NPT; ++u) {
+    const int j = lane + 32 * u;
+    const double sj = (j < g.NB) ? srow[j] : -INFINITY;
+    m[u] = (j < g.NB) ? fast_exp2(static_cast<float>((sj - mx) * 1.4426950408889634)) : 0.0f;
+    total += static_cast<double>(m[u]);
+  }
+  total = warp_sum_f64(total);
+  const double target = g.p * total;            // cumulative mass to reach, unnormalised
+
+  unsigned long long thr = 0ull;   // keep key >= thr (0 keeps all)
+  if (g.p < 1.0) {
+    unsigned long long lo = 0ull, hi = ~0ull;   // the answer lies in (lo, hi]
+    double above = 0.0;                         // mass of keys > hi
+    for (int round = 0; round < 4 * 32 * NPT; ++round) {
+      int mycnt = 0;
+      unsigned long long mine = 0ull;
+#pragma unroll
+      for (int u = 0; u < NPT; ++u) {
+        const bool live = key[u] > lo && key[u] <= hi;
+        mycnt += live;
+        if (live) mine = key[u];
+      }
+      const unsigned holders = __ballot_sync(0xffffffffu, mycnt > 0);
+      if (holders == 0u) break;                 // total mass below p (rounding): keep every block
+      const int nh = __popc(holders);
+      const int pick = __fns(holders, 0, 1 + (round * 7) % nh);
+      const unsigned long long pivot = __shfl_sync(0xffffffffu, mine, pick);
+      double gt = 0.0, eq = 0.0;
+#pragma unroll
+      for (int u = 0; u < NPT; ++u) {
+        const bool live = key[u] > lo && key[u] <= hi;
+        if (live && key[u] > pivot) gt += static_cast<double>(m[u]);
+        if (key[u] == pivot) eq = static_cast<double>(m[u]);
+      }
+      const double g_above = above + warp_sum_f64(gt);
+      if (g_above >= target) {
+        lo = pivot;                             // the k*-th key is above the pivot
+      } else {
+        const double f = g_above + warp_sum_f64(eq);
+        if (f >= target) {
+          thr = pivot;                          // the pivot is the k*-th key
+          break;
+        }
+        hi = pivot - 1ull;                      // below the pivot; everything >= pivot counts as above
+        above = f;
+      }
+    }
+  }
+
+  const int qx = i % g.nX, qy = (i / g.nX) % g.nY, qt = i / (g.nX * g.nY);
+  uint32_t* brow = bits + row * g.NW;
+  int16_t* irow = idx + row * g.NB;
+  int base = 0;
+#pragma unroll
+  for (int u = 0; u < NPT; ++u) {
+    const int j = lane + 32 * u;
+    bool keep = false;
+    if (j < g.NB) {
+      keep = key[u] >= thr;
+      if (g.sta_radius >= 0) {
+        const int kx = j % g.nX, ky = (j / g.nX) % g.nY, kt = j / (g.nX * g.nY);
+        const int dmax = max(abs(kt - qt), max(abs(ky - qy), abs(kx - qx)));
+        keep = keep || (dmax <= g.sta_radius);
+      }
+    }
+    const unsigned w = __ballot_sync(0xffffffffu, keep);
+    if (u < g.NW && lane == 0) brow[u] = w;
+    if (keep) irow[base + __popc(w & ((1u << lane) - 1u))] = static_cast<int16_t>(j);
+    base += __popc(w);
+  }
+  if (lane == 0) count[row] = base;
 }
 
 // ---------------------------------------------------------------------------
