@@ -12,6 +12,7 @@
 
 #include "../../include/dbst.h"
 #include "attn.cuh"
+#include "attn_pair.cuh"
 #include "mask.cuh"
 #include "ptx.cuh"
 #include "reorder.cuh"
@@ -163,6 +164,46 @@ dbst_status launch_attn(const void* q, const void* k, const void* v, const dbst_
   return launch_status();
 }
 
+// Query blocks are paired with their neighbour one tile step along the slowest tile axis
+// that has more than one tile (time, else height, else width): neighbouring blocks keep
+// largely the same key blocks, so the union a pair walks stays close to each list.
+int pair_stride(const dbst_geom* g) {
+  const int nT = g->T / g->tt, nY = g->Y / g->ty, nX = g->X / g->tx;
+  if (nT > 1) return nY * nX;
+  if (nY > 1) return nX;
+  return 1;
+}
+
+template <int D>
+dbst_status launch_pair(const void* q, const void* k, const void* v, const dbst_geom* g, const int32_t* cnt,
+                        const int16_t* idx, float scale, void* o, float* lse, cudaStream_t s) {
+  const long long rows = bh_count(g) * tokens(g);
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, rows, D) || !make_tmap(&tk, k, rows, D) || !make_tmap(&tv, v, rows, D)) return DBST_ECUDA;
+  dbst::PairParams p;
+  p.kv_count = cnt;
+  p.kv_idx = idx;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.NB = nblocks(g);
+  p.N = static_cast<int>(tokens(g));
+  p.pair_stride = pair_stride(g);
+  p.pairs_per_head = ((p.NB + 2 * p.pair_stride - 1) / (2 * p.pair_stride)) * p.pair_stride;
+  const float sc = scale > 0.0f ? scale : 1.0f / std::sqrt(static_cast<float>(D));
+  p.scale_log2 = sc * 1.4426950408889634f;
+  const int smem = dbst::PairSmem::kBytes + 1024;
+  static std::once_flag once;
+  static cudaError_t attr = cudaSuccess;
+  std::call_once(once, [&] {
+    attr = cudaFuncSetAttribute(dbst::pair_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  if (attr != cudaSuccess) return DBST_ECUDA;
+  const long long grid = bh_count(g) * p.pairs_per_head;
+  if (grid >= (1ll << 31)) return DBST_EINVAL;
+  dbst::pair_attn_kernel<D><<<static_cast<unsigned>(grid), dbst::kPairThreads, smem, s>>>(tq, tk, tv, p);
+  return launch_status();
+}
+
 dbst_status attn_common(const void* q, const void* k, const void* v, const dbst_geom* g, const int32_t* cnt,
                         const int16_t* idx, float scale, void* o, float* lse, void* stream) {
   if (!geom_ok(g) || !q || !k || !v || !o) return DBST_EINVAL;
@@ -170,8 +211,8 @@ dbst_status attn_common(const void* q, const void* k, const void* v, const dbst_
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return DBST_EINVAL;
   if (!(std::isfinite(scale))) return DBST_EINVAL;
   auto s = static_cast<cudaStream_t>(stream);
-  return g->D == 128 ? launch_attn<128>(q, k, v, g, cnt, idx, scale, o, lse, s)
-                     : launch_attn<64>(q, k, v, g, cnt, idx, scale, o, lse, s);
+  return g->D == 128 ? launch_pair<128>(q, k, v, g, cnt, idx, scale, o, lse, s)
+                     : launch_pair<64>(q, k, v, g, cnt, idx, scale, o, lse, s);
 }
 
 template <int NPT>

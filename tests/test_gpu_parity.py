@@ -172,6 +172,33 @@ def test_attention_edge_masks(built, D, NBgrid):
     assert (o[0, 0, :64] == 0).all() and np.isneginf(lse[0, 0, :64]).all()
 
 
+def test_attention_repeat_launches_bit_identical(built):
+    """Repeated launches on the same inputs give bit-identical outputs.
+
+    The kernel's warps hand tiles to one another through barriers; an ordering
+    bug between them shows up as run-to-run differences long before it shows
+    up as a tolerance failure on one run.
+    """
+    w = S.Workload("rep", 7, B=1, H=4, D=128, grid=(4, 16, 32), tile=(1, 8, 8), alpha=0.7, beta=0.3, f_rms=4.0,
+                   kmax=3, p_list=(0.9,), sta_radius=-1)
+    g = P.geometry(w)
+    q, k, v = S.make_qkv(w)
+    qt, kt, vt = (O.tile_reorder(a, g) for a in (q, k, v))
+    mask = np.stack([edge_masks(g.NB, s) for s in range(w.H)])[None]
+    gg = gpu_geom(w, heads=w.H)
+    words = torch.from_numpy(P.pack_mask(mask).view(np.int32)).cuda()
+    cnt, idx = dbst.mask_from_bits(words, gg)
+    qd, kd, vd = (P.bits_to_torch(a) for a in (qt, kt, vt))
+    o0, l0 = dbst.block_sparse_attn(qd, kd, vd, gg, cnt, idx, 0.3)
+    for _ in range(30):
+        o1, l1 = dbst.block_sparse_attn(qd, kd, vd, gg, cnt, idx, 0.3)
+        assert torch.equal(o0.view(torch.int16), o1.view(torch.int16))
+        assert torch.equal(l0, l1)
+    dbst.get_error()
+    o_ref, lse_ref = O.masked_attention(qt, kt, vt, mask, 64, 0.3)
+    check_attention(o0.float().cpu().numpy().astype(np.float64), l0.cpu().numpy().astype(np.float64), o_ref, lse_ref)
+
+
 def test_constant_v_and_large_logits(built):
     """Constant V is reproduced; logits spanning > 2^16 in log2 units force rescales."""
     w = S.Workload("c", 6, B=1, H=1, D=128, grid=(2, 16, 32), tile=(2, 4, 8), alpha=0.7, beta=0.3, f_rms=6.0,
