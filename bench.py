@@ -49,7 +49,7 @@ def peaks():
 def attn_source_digest() -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in ("attn.cuh", "ptx.cuh"):
+    for f in ("attn_pair.cuh", "ptx.cuh"):
         with open(os.path.join(ROOT, "dynamic_block_sparse_tile_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -57,7 +57,7 @@ def attn_source_digest() -> str:
 
 def measured_traffic(workload: str, p: float):
     """DRAM bytes per attention launch from the committed ncu summary, if it matches this kernel source."""
-    path = os.path.join(ROOT, "profiles", "sparse_attn_kernel_dram_traffic.md")
+    path = os.path.join(ROOT, "profiles", "pair_attn_kernel_dram_traffic.md")
     try:
         text = open(path).read()
     except OSError:
@@ -406,7 +406,7 @@ def main():
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": bf16, "unit": "TFLOP/s",
                      "frac": attn_tflops / bf16, "traffic": measured_traffic(w.name, p),
                      "peak_source": f"{src} bf16 burst; frac of sustained {attn_tflops / bf16_sus:.3f}",
-                     "kernel": "sparse_attn_kernel<128>"},
+                     "kernel": "pair_attn_kernel<128>"},
         "mask_roofline": {"bound": "hbm", "achieved": mask_bytes / (mask_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
                           "frac": mask_bytes / (mask_ms * 1e-3) / 1e9 / hbm},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "ms_per_step": e2e_ms / args.steps,

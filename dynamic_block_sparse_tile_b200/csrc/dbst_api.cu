@@ -11,7 +11,6 @@
 #include <mutex>
 
 #include "../../include/dbst.h"
-#include "attn.cuh"
 #include "attn_pair.cuh"
 #include "mask.cuh"
 #include "ptx.cuh"
@@ -134,34 +133,6 @@ bool make_tmap(CUtensorMap* m, const void* base, long long rows, int D) {
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
-}
-
-template <int D>
-dbst_status launch_attn(const void* q, const void* k, const void* v, const dbst_geom* g, const int32_t* cnt,
-                        const int16_t* idx, float scale, void* o, float* lse, cudaStream_t s) {
-  const long long rows = bh_count(g) * tokens(g);
-  CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, q, rows, D) || !make_tmap(&tk, k, rows, D) || !make_tmap(&tv, v, rows, D)) return DBST_ECUDA;
-  dbst::AttnParams p;
-  p.kv_count = cnt;
-  p.kv_idx = idx;
-  p.o = static_cast<__nv_bfloat16*>(o);
-  p.lse = lse;
-  p.NB = nblocks(g);
-  p.N = static_cast<int>(tokens(g));
-  const float sc = scale > 0.0f ? scale : 1.0f / std::sqrt(static_cast<float>(D));
-  p.scale_log2 = sc * 1.4426950408889634f;
-  const int smem = dbst::AttnSmem::kBytes + 1024;
-  static std::once_flag once;
-  static cudaError_t attr = cudaSuccess;
-  std::call_once(once, [&] {
-    attr = cudaFuncSetAttribute(dbst::sparse_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  });
-  if (attr != cudaSuccess) return DBST_ECUDA;
-  const long long grid = bh_count(g) * p.NB;
-  if (grid >= (1ll << 31)) return DBST_EINVAL;
-  dbst::sparse_attn_kernel<D><<<static_cast<unsigned>(grid), dbst::kAttnThreads, smem, s>>>(tq, tk, tv, p);
-  return launch_status();
 }
 
 // Query blocks are paired with their neighbour one tile step along the slowest tile axis

@@ -2,10 +2,11 @@
 // selection, sliding-tile union and index-list expansion (NABLA page,
 // "Construction de Masque Adaptatif" and "Intégration Hybride avec STA").
 //
-// Precision: the pooled means are exact (64 bf16 values summed in float64),
-// the pooled logits, softmax and cumulative masses are float64, so the kept
-// set agrees with a float64 reference except where a cumulative mass sits
-// within rounding of p.
+// Precision: the pooled means are exact (64 bf16 values summed in float64) and
+// the pooled logits are float64.  The order of a row's blocks comes from those
+// logits; the masses are float32 exponentials summed in float64 for rows of at
+// most 1024 blocks, float64 for longer rows.  The kept set agrees with a
+// float64 reference except where a cumulative mass sits within rounding of p.
 #pragma once
 #include <cstdint>
 #include "ptx.cuh"
@@ -377,7 +378,6 @@ __global__ void __launch_bounds__(128) select_warp_kernel(const double* __restri
     const double sj = (j < g.NB) ? srow[j] : -INFINITY;
     key[u] = (j < g.NB) ? logit_key(sj, j) : 0ull;
     mx = fmax(mx, sj);
-    m[u] = static_cast<float>(sj);   // placeholder, replaced below
   }
   mx = warp_max_f64(mx);
   double total = 0.0;
