@@ -2,7 +2,12 @@
 
 One step = one pass of the whole path over one batch of the Wan-like 480p
 latent workload (B=1, H=40, D=128, token grid 21x32x56 in 1x8x8 tiles,
-N=37632, 588 blocks; CDF threshold p=0.9; seeded synthetic q/k/v):
+N=37632, 588 blocks; CDF threshold p=0.9; seeded synthetic q/k/v).  Default
+(`--path fused`): raster q, k, v in, raster o out, the tile reorder done by the
+kernels' own loads and stores:
+    build_block_mask_raster(q, k) -> block_sparse_attn_raster(q, k, v) -> o
+(4 launches: pool, pooled logits, select, attention).  `--path explicit` runs
+the same steps as separate passes (8 launches):
     tile_reorder(q, k, v) -> build_block_mask -> block_sparse_attn -> tile_unreorder(o)
 
 `value` = kept-block TFLOP/s of the whole step (4*D*64*64 FLOP per kept
@@ -55,7 +60,7 @@ def attn_source_digest() -> str:
     return h.hexdigest()[:16]
 
 
-def measured_traffic(workload: str, p: float):
+def measured_traffic(workload: str, p: float, layout: str):
     """DRAM bytes per attention launch from the committed ncu summary, if it matches this kernel source."""
     path = os.path.join(ROOT, "profiles", "pair_attn_kernel_dram_traffic.md")
     try:
@@ -63,7 +68,7 @@ def measured_traffic(workload: str, p: float):
     except OSError:
         return None
     for line in text.splitlines():
-        if line.startswith("| ") and f"`{workload}`" in line and f"p={p}" in line:
+        if line.startswith("| ") and f"`{workload}`" in line and f"p={p}" in line and layout in line:
             cells = [c.strip() for c in line.strip("|").split("|")]
             try:
                 digest, total = cells[1].strip("`"), float(cells[4])
@@ -274,6 +279,8 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="sparsity sweep: attention ms/call and kept-block TFLOP/s per p, dense crossover")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", default="fused", choices=["fused", "explicit"],
+                    help="fused: tile reorder folded into the kernels (raster entry points); explicit: separate passes")
     args = ap.parse_args()
     w = S.workload(args.workload)
     p = args.p if args.p is not None else w.p_list[0]
@@ -305,7 +312,10 @@ def main():
     host = [to_t(a).pin_memory() for a in (q_h, k_h, v_h)]
     del q_h, k_h, v_h
     q, k, v = (t.cuda() for t in host)
-    qt, kt, vt, ot, o = (torch.empty_like(q) for _ in range(5))
+    o = torch.empty_like(q)
+    qt = kt = vt = ot = None
+    if args.path == "explicit":
+        qt, kt, vt, ot = (torch.empty_like(q) for _ in range(4))
     bits = torch.empty((g.B, g.H, g.NB, g.NW), dtype=torch.int32, device="cuda")
     cnt = torch.empty((g.B, g.H, g.NB), dtype=torch.int32, device="cuda")
     idx = torch.empty((g.B, g.H, g.NB, g.NB), dtype=torch.int16, device="cuda")
@@ -313,27 +323,37 @@ def main():
     lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device="cuda")
     o_host = torch.empty_like(host[0]).pin_memory()
     stream = torch.cuda.current_stream()
-    launches_per_step = 8   # 3 reorder + pool + logits + select + attention + unreorder
+    fused = args.path == "fused"
+    # fused: pool + logits + select + attention; explicit: 3 reorders + those 4 + unreorder
+    launches_per_step = 4 if fused else 8
 
     ev = {}
 
     def step(timed_parts: bool):
-        dbst.tile_reorder(q, g, out=qt)
-        dbst.tile_reorder(k, g, out=kt)
-        dbst.tile_reorder(v, g, out=vt)
+        if not fused:
+            dbst.tile_reorder(q, g, out=qt)
+            dbst.tile_reorder(k, g, out=kt)
+            dbst.tile_reorder(v, g, out=vt)
         if timed_parts:
             e0 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-        dbst.build_block_mask(qt, kt, g, p, w.sta_radius, workspace=ws, out=(bits, cnt, idx))
+        if fused:
+            dbst.build_block_mask_raster(q, k, g, p, w.sta_radius, workspace=ws, out=(bits, cnt, idx))
+        else:
+            dbst.build_block_mask(qt, kt, g, p, w.sta_radius, workspace=ws, out=(bits, cnt, idx))
         if timed_parts:
             e1 = torch.cuda.Event(enable_timing=True)
             e1.record(stream)
-        dbst.block_sparse_attn(qt, kt, vt, g, cnt, idx, 0.0, want_lse=True, out=ot, lse=lse)
+        if fused:
+            dbst.block_sparse_attn_raster(q, k, v, g, cnt, idx, 0.0, want_lse=True, out=o, lse=lse)
+        else:
+            dbst.block_sparse_attn(qt, kt, vt, g, cnt, idx, 0.0, want_lse=True, out=ot, lse=lse)
         if timed_parts:
             e2 = torch.cuda.Event(enable_timing=True)
             e2.record(stream)
             ev.setdefault("parts", []).append((e0, e1, e2))
-        dbst.tile_unreorder(ot, g, out=o)
+        if not fused:
+            dbst.tile_unreorder(ot, g, out=o)
 
     for _ in range(args.warmup):
         step(False)
@@ -400,13 +420,15 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": workload_desc(w, p), "kept_fraction": kept_frac, "kept_block_pairs": kept_pairs,
-                   "l2": "inputs (385 MB per tensor) larger than L2; no flush", "parallelism": f"dp{world} (independent problems)"},
+                   "l2": "inputs (385 MB per tensor) larger than L2; no flush", "parallelism": f"dp{world} (independent problems)",
+                   "path": "raster in/out, tile reorder inside the kernels" if fused else
+                           "explicit tile_reorder / tile_unreorder passes"},
         "sparse_attn_ms_per_call": attn_ms, "sparse_attn_tflops": attn_tflops,
         "mask_build_ms_per_call": mask_ms, "mask_build_gbs": mask_bytes / (mask_ms * 1e-3) / 1e9,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": bf16, "unit": "TFLOP/s",
-                     "frac": attn_tflops / bf16, "traffic": measured_traffic(w.name, p),
+                     "frac": attn_tflops / bf16, "traffic": measured_traffic(w.name, p, "raster" if fused else "tiled"),
                      "peak_source": f"{src} bf16 burst; frac of sustained {attn_tflops / bf16_sus:.3f}",
-                     "kernel": "pair_attn_kernel<128>"},
+                     "kernel": "pair_attn_kernel<128, raster>" if fused else "pair_attn_kernel<128, tiled>"},
         "mask_roofline": {"bound": "hbm", "achieved": mask_bytes / (mask_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
                           "frac": mask_bytes / (mask_ms * 1e-3) / 1e9 / hbm},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "ms_per_step": e2e_ms / args.steps,

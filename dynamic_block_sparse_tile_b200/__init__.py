@@ -18,7 +18,8 @@ from typing import Optional, Sequence, Tuple
 import torch
 
 __all__ = ["Geom", "DbstError", "lib_path", "load", "tile_reorder", "tile_unreorder", "mask_workspace_bytes",
-           "build_block_mask", "build_block_mask_noalloc", "mask_from_bits", "block_sparse_attn", "dense_attn", "get_error", "EXPORTS"]
+           "build_block_mask", "build_block_mask_noalloc", "mask_from_bits", "block_sparse_attn", "dense_attn",
+           "build_block_mask_raster", "block_sparse_attn_raster", "dense_attn_raster", "get_error", "EXPORTS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libdbst.so")
@@ -26,7 +27,8 @@ _LIB_PATH = os.path.join(_HERE, "libdbst.so")
 # Every symbol declared in include/dbst.h.
 EXPORTS = ("dbst_status_string", "dbst_tile_reorder", "dbst_tile_unreorder", "dbst_mask_workspace_bytes",
            "dbst_build_block_mask", "dbst_mask_from_bits", "dbst_block_sparse_attn", "dbst_dense_attn",
-           "dbst_get_error", "dbst_build_block_mask_noalloc")
+           "dbst_get_error", "dbst_build_block_mask_noalloc", "dbst_build_block_mask_raster",
+           "dbst_block_sparse_attn_raster", "dbst_dense_attn_raster")
 
 DBST_OK, DBST_EINVAL, DBST_ECUDA, DBST_ETIMEOUT, DBST_EBOUNDS, DBST_ETOOLARGE = 0, 1, 2, 3, 4, 5
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -80,12 +82,15 @@ def load() -> ctypes.CDLL:
         getattr(lib, name).argtypes = [vp, vp, gp, vp]
         getattr(lib, name).restype = i32
     lib.dbst_mask_workspace_bytes.argtypes, lib.dbst_mask_workspace_bytes.restype = [gp], ctypes.c_size_t
-    lib.dbst_build_block_mask.argtypes = [vp, vp, gp, f32, i32, vp, vp, vp, vp, ctypes.c_size_t, vp]
-    lib.dbst_build_block_mask.restype = i32
+    for name in ("dbst_build_block_mask", "dbst_build_block_mask_raster"):
+        getattr(lib, name).argtypes = [vp, vp, gp, f32, i32, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        getattr(lib, name).restype = i32
     lib.dbst_mask_from_bits.argtypes, lib.dbst_mask_from_bits.restype = [vp, gp, vp, vp, vp], i32
-    lib.dbst_block_sparse_attn.argtypes = [vp, vp, vp, gp, vp, vp, f32, vp, vp, vp]
-    lib.dbst_block_sparse_attn.restype = i32
-    lib.dbst_dense_attn.argtypes, lib.dbst_dense_attn.restype = [vp, vp, vp, gp, f32, vp, vp, vp], i32
+    for name in ("dbst_block_sparse_attn", "dbst_block_sparse_attn_raster"):
+        getattr(lib, name).argtypes = [vp, vp, vp, gp, vp, vp, f32, vp, vp, vp]
+        getattr(lib, name).restype = i32
+    for name in ("dbst_dense_attn", "dbst_dense_attn_raster"):
+        getattr(lib, name).argtypes, getattr(lib, name).restype = [vp, vp, vp, gp, f32, vp, vp, vp], i32
     lib.dbst_get_error.argtypes, lib.dbst_get_error.restype = [vp], i32
     lib.dbst_build_block_mask_noalloc.argtypes = [vp, vp, gp, f32, i32, vp, vp, vp, vp]
     lib.dbst_build_block_mask_noalloc.restype = i32
@@ -148,6 +153,16 @@ def mask_workspace_bytes(g: Geom) -> int:
 def build_block_mask(q_tiled: torch.Tensor, k_tiled: torch.Tensor, g: Geom, p: float, sta_radius: int = -1,
                      workspace: Optional[torch.Tensor] = None, out=None):
     """Adaptive block mask (``dbst_build_block_mask``) -> (mask_bits, kv_count, kv_idx)."""
+    return _build_block_mask("dbst_build_block_mask", q_tiled, k_tiled, g, p, sta_radius, workspace, out)
+
+
+def build_block_mask_raster(q: torch.Tensor, k: torch.Tensor, g: Geom, p: float, sta_radius: int = -1,
+                            workspace: Optional[torch.Tensor] = None, out=None):
+    """Adaptive block mask from raster-order q, k (``dbst_build_block_mask_raster``)."""
+    return _build_block_mask("dbst_build_block_mask_raster", q, k, g, p, sta_radius, workspace, out)
+
+
+def _build_block_mask(fn: str, q_tiled, k_tiled, g: Geom, p: float, sta_radius: int, workspace, out):
     _need(q_tiled, torch.bfloat16, _qkv_shape(g), "q_tiled")
     _need(k_tiled, torch.bfloat16, _qkv_shape(g), "k_tiled")
     dev = q_tiled.device
@@ -160,10 +175,9 @@ def build_block_mask(q_tiled: torch.Tensor, k_tiled: torch.Tensor, g: Geom, p: f
     nbytes = mask_workspace_bytes(g)
     if workspace is None:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
-    _check(load().dbst_build_block_mask(_ptr(q_tiled), _ptr(k_tiled), ctypes.byref(g), float(p), int(sta_radius),
-                                        _ptr(bits), _ptr(cnt), _ptr(idx), _ptr(workspace),
-                                        workspace.numel() * workspace.element_size(), _stream()),
-           "dbst_build_block_mask")
+    _check(getattr(load(), fn)(_ptr(q_tiled), _ptr(k_tiled), ctypes.byref(g), float(p), int(sta_radius),
+                               _ptr(bits), _ptr(cnt), _ptr(idx), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream()), fn)
     return bits, cnt, idx
 
 
@@ -203,6 +217,17 @@ def mask_from_bits(bits: torch.Tensor, g: Geom):
 def block_sparse_attn(q, k, v, g: Geom, kv_count, kv_idx, scale: float = 0.0, want_lse: bool = True,
                       out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None):
     """Attention over kept blocks (``dbst_block_sparse_attn``) -> (o, lse or None)."""
+    return _block_sparse_attn("dbst_block_sparse_attn", q, k, v, g, kv_count, kv_idx, scale, want_lse, out, lse)
+
+
+def block_sparse_attn_raster(q, k, v, g: Geom, kv_count, kv_idx, scale: float = 0.0, want_lse: bool = True,
+                             out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None):
+    """Attention over kept blocks on raster-order tensors (``dbst_block_sparse_attn_raster``)."""
+    return _block_sparse_attn("dbst_block_sparse_attn_raster", q, k, v, g, kv_count, kv_idx, scale, want_lse, out,
+                              lse)
+
+
+def _block_sparse_attn(fn: str, q, k, v, g: Geom, kv_count, kv_idx, scale, want_lse, out, lse):
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, torch.bfloat16, _qkv_shape(g), n)
     _need(kv_count, torch.int32, (g.B, g.H, g.NB), "kv_count")
@@ -210,20 +235,28 @@ def block_sparse_attn(q, k, v, g: Geom, kv_count, kv_idx, scale: float = 0.0, wa
     o = torch.empty_like(q) if out is None else out
     if want_lse and lse is None:
         lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device=q.device)
-    _check(load().dbst_block_sparse_attn(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(g), _ptr(kv_count),
-                                         _ptr(kv_idx), float(scale), _ptr(o), _ptr(lse if want_lse else None),
-                                         _stream()), "dbst_block_sparse_attn")
+    _check(getattr(load(), fn)(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(g), _ptr(kv_count), _ptr(kv_idx),
+                               float(scale), _ptr(o), _ptr(lse if want_lse else None), _stream()), fn)
     return o, (lse if want_lse else None)
 
 
 def dense_attn(q, k, v, g: Geom, scale: float = 0.0, want_lse: bool = True):
     """Dense attention over all tokens (``dbst_dense_attn``) -> (o, lse or None)."""
+    return _dense_attn("dbst_dense_attn", q, k, v, g, scale, want_lse)
+
+
+def dense_attn_raster(q, k, v, g: Geom, scale: float = 0.0, want_lse: bool = True):
+    """Dense attention on raster-order tensors (``dbst_dense_attn_raster``) -> (o, lse or None)."""
+    return _dense_attn("dbst_dense_attn_raster", q, k, v, g, scale, want_lse)
+
+
+def _dense_attn(fn: str, q, k, v, g: Geom, scale, want_lse):
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, torch.bfloat16, _qkv_shape(g), n)
     o = torch.empty_like(q)
     lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device=q.device) if want_lse else None
-    _check(load().dbst_dense_attn(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(g), float(scale), _ptr(o), _ptr(lse),
-                                  _stream()), "dbst_dense_attn")
+    _check(getattr(load(), fn)(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(g), float(scale), _ptr(o), _ptr(lse),
+                               _stream()), fn)
     return o, lse
 
 

@@ -31,6 +31,7 @@
 #include <cstdint>
 #include <cuda_bf16.h>
 #include "ptx.cuh"
+#include "reorder.cuh"
 
 namespace dbst {
 
@@ -51,6 +52,7 @@ struct PairParams {
   int pair_stride;           // qb = qa + pair_stride
   int pairs_per_head;
   float scale_log2;          // softmax scale * log2(e)
+  TileGeo tg;                // token grid and tile shape (raster layout only)
 };
 
 struct PairSmem {
@@ -97,7 +99,12 @@ __device__ __forceinline__ void umma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, 
       : "memory");
 }
 
-template <int D>
+// RASTER = false: q, k, v, o are in tile order (block j = rows 64j .. 64j+63 of a head), loaded
+// with 2-D boxes.  RASTER = true: they are in the caller's raster order; the tile reorder is done
+// by the loads themselves (5-D boxes tx x ty x tt tokens x 64 channels land in shared memory in
+// exactly the tile-ordered layout) and by the epilogue, which writes o and lse rows in raster
+// order.  Both produce bit-identical results.
+template <int D, bool RASTER>
 __global__ void __launch_bounds__(kPairThreads, 1)
     pair_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const PairParams prm) {
@@ -123,8 +130,20 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   const int qa = (pi / ps) * 2 * ps + (pi % ps);
   const int qb = qa + ps;
   const bool has_b = qb < NB;
-  const long long rowa = bh * prm.N + static_cast<long long>(qa) * 64;
-  const long long rowb = bh * prm.N + static_cast<long long>(has_b ? qb : qa) * 64;
+  // global row of row rr (0..63) of query block blk of this head
+  auto out_row = [&](int blk, int rr) -> long long {
+    if constexpr (RASTER) return bh * prm.N + tiled_to_raster(blk * 64 + rr, prm.tg);
+    else return bh * prm.N + static_cast<long long>(blk) * 64 + rr;
+  };
+  // TMA load of block blk's channels 64h .. 64h+63 (8 KB) into shared memory
+  auto load_block = [&](uint32_t dst, const CUtensorMap* map, uint32_t mbar, int blk, int h) {
+    if constexpr (RASTER) {
+      const int Tx = blk % prm.tg.nX, Ty = (blk / prm.tg.nX) % prm.tg.nY, Tt = blk / (prm.tg.nX * prm.tg.nY);
+      tma_load_5d(dst, map, mbar, 64 * h, Tx * prm.tg.tx, Ty * prm.tg.ty, Tt * prm.tg.tt, static_cast<int32_t>(bh));
+    } else {
+      tma_load_2d(dst, map, mbar, 64 * h, static_cast<int32_t>(bh * prm.N + static_cast<long long>(blk) * 64));
+    }
+  };
 
   // ---- union of the two lists as bitmasks -> ascending entries with membership flags
   for (int w = tid; w < 2 * 128; w += kPairThreads) s_words[w] = 0u;
@@ -199,12 +218,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   const int nu = static_cast<int>(s_misc[1]);
   if (nu == 0) {   // neither block keeps anything: o = 0, lse = -inf
     for (int e = tid; e < 64 * D / 8; e += kPairThreads) {
-      reinterpret_cast<uint4*>(prm.o + rowa * D)[e] = make_uint4(0, 0, 0, 0);
-      if (has_b) reinterpret_cast<uint4*>(prm.o + rowb * D)[e] = make_uint4(0, 0, 0, 0);
+      const int rr = e / (D / 8), c = e % (D / 8);
+      reinterpret_cast<uint4*>(prm.o + out_row(qa, rr) * D)[c] = make_uint4(0, 0, 0, 0);
+      if (has_b) reinterpret_cast<uint4*>(prm.o + out_row(qb, rr) * D)[c] = make_uint4(0, 0, 0, 0);
     }
     if (prm.lse && tid < 64) {
-      prm.lse[rowa + tid] = -INFINITY;
-      if (has_b) prm.lse[rowb + tid] = -INFINITY;
+      prm.lse[out_row(qa, tid)] = -INFINITY;
+      if (has_b) prm.lse[out_row(qb, tid)] = -INFINITY;
     }
     return;
   }
@@ -218,12 +238,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_misc[0];
-  auto tile_rows = [&](int t, int32_t& y0, int32_t& y1) {
-    const int j0 = s_union[2 * t] & 0xFFFF;
-    const int j1 = (2 * t + 1 < nu) ? (s_union[2 * t + 1] & 0xFFFF) : j0;   // odd tail: duplicate, masked
-    y0 = static_cast<int32_t>(bh * prm.N + static_cast<long long>(j0) * 64);
-    y1 = static_cast<int32_t>(bh * prm.N + static_cast<long long>(j1) * 64);
-  };
 
   if (warp == 13 || warp == 14) {
     // ------------------------------------------------------------ TMA producers
@@ -239,8 +253,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         tma_prefetch_desc(&tmQ);
         mbar_expect_tx(bar(PB_Q), 128 * D * 2);
         for (int h = 0; h < DH; ++h) {
-          tma_load_2d(sbase + PairSmem::kQ + h * 16384, &tmQ, bar(PB_Q), 64 * h, static_cast<int32_t>(rowa));
-          tma_load_2d(sbase + PairSmem::kQ + h * 16384 + 8192, &tmQ, bar(PB_Q), 64 * h, static_cast<int32_t>(rowb));
+          load_block(sbase + PairSmem::kQ + h * 16384, &tmQ, bar(PB_Q), qa, h);
+          load_block(sbase + PairSmem::kQ + h * 16384 + 8192, &tmQ, bar(PB_Q), has_b ? qb : qa, h);
         }
       }
       int armed[kPairKSlots] = {0, 0, 0};
@@ -251,13 +265,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           *s_abort = 1;
           break;
         }
-        int32_t y0, y1;
-        tile_rows(t, y0, y1);
+        const int j0 = s_union[2 * t] & 0xFFFF;
+        const int j1 = (2 * t + 1 < nu) ? (s_union[2 * t + 1] & 0xFFFF) : j0;   // odd tail: duplicate, masked
         const uint32_t dst = ring + s * PairSmem::kTile;
         mbar_expect_tx(bar(full0 + s), 128 * D * 2);
         for (int h = 0; h < DH; ++h) {
-          tma_load_2d(dst + h * 16384, map, bar(full0 + s), 64 * h, y0);
-          tma_load_2d(dst + h * 16384 + 8192, map, bar(full0 + s), 64 * h, y1);
+          load_block(dst + h * 16384, map, bar(full0 + s), j0, h);
+          load_block(dst + h * 16384 + 8192, map, bar(full0 + s), j1, h);
         }
         armed[s] = t / slots + 1;
       }
@@ -457,7 +471,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const float lt = lpart + s_lsum[(hc ^ 1) * 128 + r];
     if (side == 0 || has_b) {
       const float inv = (lt > 0.0f) ? 1.0f / lt : 0.0f;
-      const long long orow = (side ? rowb : rowa) + (r & 63);
+      const long long orow = out_row(side ? qb : qa, r & 63);
       uint4* dst = reinterpret_cast<uint4*>(prm.o + orow * D + (D / 2) * hc);
 #pragma unroll
       for (int c0 = 0; c0 < D / 2; c0 += 32) {

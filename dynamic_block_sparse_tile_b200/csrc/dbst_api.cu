@@ -145,13 +145,36 @@ int pair_stride(const dbst_geom* g) {
   return 1;
 }
 
-template <int D>
+// Raster layout [B*H, T, Y, X, D] bf16 as a 5-D tensor (innermost first); one box is one tile's
+// tokens x 64 channels, 8 KB, arriving in shared memory in tile order.
+bool make_tmap_raster(CUtensorMap* m, const void* base, const dbst_geom* g) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t D = static_cast<cuuint64_t>(g->D);
+  cuuint64_t dims[5] = {D, static_cast<cuuint64_t>(g->X), static_cast<cuuint64_t>(g->Y), static_cast<cuuint64_t>(g->T),
+                        static_cast<cuuint64_t>(bh_count(g))};
+  cuuint64_t strides[4] = {D * 2, D * 2 * dims[1], D * 2 * dims[1] * dims[2], D * 2 * dims[1] * dims[2] * dims[3]};
+  cuuint32_t box[5] = {64, static_cast<cuuint32_t>(g->tx), static_cast<cuuint32_t>(g->ty),
+                       static_cast<cuuint32_t>(g->tt), 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, bool RASTER>
 dbst_status launch_pair(const void* q, const void* k, const void* v, const dbst_geom* g, const int32_t* cnt,
                         const int16_t* idx, float scale, void* o, float* lse, cudaStream_t s) {
   const long long rows = bh_count(g) * tokens(g);
   CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, q, rows, D) || !make_tmap(&tk, k, rows, D) || !make_tmap(&tv, v, rows, D)) return DBST_ECUDA;
+  if (RASTER) {
+    if (!make_tmap_raster(&tq, q, g) || !make_tmap_raster(&tk, k, g) || !make_tmap_raster(&tv, v, g)) return DBST_ECUDA;
+  } else {
+    if (!make_tmap(&tq, q, rows, D) || !make_tmap(&tk, k, rows, D) || !make_tmap(&tv, v, rows, D)) return DBST_ECUDA;
+  }
   dbst::PairParams p;
+  p.tg = tile_geo(g);
   p.kv_count = cnt;
   p.kv_idx = idx;
   p.o = static_cast<__nv_bfloat16*>(o);
@@ -166,24 +189,27 @@ dbst_status launch_pair(const void* q, const void* k, const void* v, const dbst_
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [&] {
-    attr = cudaFuncSetAttribute(dbst::pair_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    attr = cudaFuncSetAttribute(dbst::pair_attn_kernel<D, RASTER>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   });
   if (attr != cudaSuccess) return DBST_ECUDA;
   const long long grid = bh_count(g) * p.pairs_per_head;
   if (grid >= (1ll << 31)) return DBST_EINVAL;
-  dbst::pair_attn_kernel<D><<<static_cast<unsigned>(grid), dbst::kPairThreads, smem, s>>>(tq, tk, tv, p);
+  dbst::pair_attn_kernel<D, RASTER><<<static_cast<unsigned>(grid), dbst::kPairThreads, smem, s>>>(tq, tk, tv, p);
   return launch_status();
 }
 
 dbst_status attn_common(const void* q, const void* k, const void* v, const dbst_geom* g, const int32_t* cnt,
-                        const int16_t* idx, float scale, void* o, float* lse, void* stream) {
+                        const int16_t* idx, float scale, void* o, float* lse, void* stream, bool raster) {
   if (!geom_ok(g) || !q || !k || !v || !o) return DBST_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return DBST_EINVAL;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return DBST_EINVAL;
   if (!(std::isfinite(scale))) return DBST_EINVAL;
   auto s = static_cast<cudaStream_t>(stream);
-  return g->D == 128 ? launch_pair<128>(q, k, v, g, cnt, idx, scale, o, lse, s)
-                     : launch_pair<64>(q, k, v, g, cnt, idx, scale, o, lse, s);
+  if (raster)
+    return g->D == 128 ? launch_pair<128, true>(q, k, v, g, cnt, idx, scale, o, lse, s)
+                       : launch_pair<64, true>(q, k, v, g, cnt, idx, scale, o, lse, s);
+  return g->D == 128 ? launch_pair<128, false>(q, k, v, g, cnt, idx, scale, o, lse, s)
+                     : launch_pair<64, false>(q, k, v, g, cnt, idx, scale, o, lse, s);
 }
 
 template <int NPT>
@@ -197,38 +223,10 @@ bool launch_select(const double* S, const dbst::SelectGeo& sg, long long rows, u
   return true;
 }
 
-}  // namespace
-
-extern "C" {
-
-const char* dbst_status_string(int status) {
-  switch (status) {
-    case DBST_OK: return "ok";
-    case DBST_EINVAL: return "invalid argument";
-    case DBST_ECUDA: return "CUDA error";
-    case DBST_ETIMEOUT: return "device wait timed out";
-    case DBST_EBOUNDS: return "index list entry out of range";
-    case DBST_ETOOLARGE: return "problem exceeds the static scratch of the allocation-free entry point";
-    default: return "unknown status";
-  }
-}
-
-dbst_status dbst_tile_reorder(const void* x, void* y, const dbst_geom* g, void* stream) {
-  return permute(x, y, g, stream, 1);
-}
-
-dbst_status dbst_tile_unreorder(const void* y, void* x, const dbst_geom* g, void* stream) {
-  return permute(y, x, g, stream, 0);
-}
-
-size_t dbst_mask_workspace_bytes(const dbst_geom* g) {
-  if (!geom_ok(g)) return 0;
-  return mask_workspace(g).total;
-}
-
-dbst_status dbst_build_block_mask(const void* q_tiled, const void* k_tiled, const dbst_geom* g, float p,
-                                  int sta_radius, uint32_t* mask_bits, int32_t* kv_count, int16_t* kv_idx,
-                                  void* workspace, size_t workspace_bytes, void* stream) {
+// Mask build over tile-ordered (raster = false) or raster-ordered (raster = true) q and k.
+dbst_status build_mask(const void* q_tiled, const void* k_tiled, const dbst_geom* g, float p, int sta_radius,
+                       uint32_t* mask_bits, int32_t* kv_count, int16_t* kv_idx, void* workspace,
+                       size_t workspace_bytes, void* stream, bool raster) {
   if (!geom_ok(g) || !q_tiled || !k_tiled || !mask_bits || !kv_count || !kv_idx || !workspace) return DBST_EINVAL;
   if (!aligned16(q_tiled) || !aligned16(k_tiled) || !aligned16(mask_bits) || !aligned16(kv_count) ||
       !aligned16(kv_idx) || !aligned16(workspace))
@@ -251,10 +249,15 @@ dbst_status dbst_build_block_mask(const void* q_tiled, const void* k_tiled, cons
     if (grid > cap) grid = cap;
     const auto* qa = static_cast<const uint4*>(q_tiled);
     const auto* ka = static_cast<const uint4*>(k_tiled);
-    if (g->D == 128)
-      dbst::pool_kernel<128><<<static_cast<unsigned>(grid), 256, 0, s>>>(qa, ka, qp, kp, nblk);
-    else
-      dbst::pool_kernel<64><<<static_cast<unsigned>(grid), 256, 0, s>>>(qa, ka, qp, kp, nblk);
+    const unsigned gr = static_cast<unsigned>(grid);
+    const dbst::TileGeo tg = tile_geo(g);
+    if (g->D == 128) {
+      if (raster) dbst::pool_kernel<128, true><<<gr, 256, 0, s>>>(qa, ka, qp, kp, nblk, NB, tg);
+      else dbst::pool_kernel<128, false><<<gr, 256, 0, s>>>(qa, ka, qp, kp, nblk, NB, tg);
+    } else {
+      if (raster) dbst::pool_kernel<64, true><<<gr, 256, 0, s>>>(qa, ka, qp, kp, nblk, NB, tg);
+      else dbst::pool_kernel<64, false><<<gr, 256, 0, s>>>(qa, ka, qp, kp, nblk, NB, tg);
+    }
     if (cudaGetLastError() != cudaSuccess) return DBST_ECUDA;
   }
   {  // 2. pooled logits (float64)
@@ -291,6 +294,48 @@ dbst_status dbst_build_block_mask(const void* q_tiled, const void* k_tiled, cons
   return launch_status();
 }
 
+}  // namespace
+
+extern "C" {
+
+const char* dbst_status_string(int status) {
+  switch (status) {
+    case DBST_OK: return "ok";
+    case DBST_EINVAL: return "invalid argument";
+    case DBST_ECUDA: return "CUDA error";
+    case DBST_ETIMEOUT: return "device wait timed out";
+    case DBST_EBOUNDS: return "index list entry out of range";
+    case DBST_ETOOLARGE: return "problem exceeds the static scratch of the allocation-free entry point";
+    default: return "unknown status";
+  }
+}
+
+dbst_status dbst_tile_reorder(const void* x, void* y, const dbst_geom* g, void* stream) {
+  return permute(x, y, g, stream, 1);
+}
+
+dbst_status dbst_tile_unreorder(const void* y, void* x, const dbst_geom* g, void* stream) {
+  return permute(y, x, g, stream, 0);
+}
+
+size_t dbst_mask_workspace_bytes(const dbst_geom* g) {
+  if (!geom_ok(g)) return 0;
+  return mask_workspace(g).total;
+}
+
+dbst_status dbst_build_block_mask(const void* q_tiled, const void* k_tiled, const dbst_geom* g, float p,
+                                  int sta_radius, uint32_t* mask_bits, int32_t* kv_count, int16_t* kv_idx,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  return build_mask(q_tiled, k_tiled, g, p, sta_radius, mask_bits, kv_count, kv_idx, workspace, workspace_bytes,
+                    stream, false);
+}
+
+dbst_status dbst_build_block_mask_raster(const void* q, const void* k, const dbst_geom* g, float p, int sta_radius,
+                                         uint32_t* mask_bits, int32_t* kv_count, int16_t* kv_idx, void* workspace,
+                                         size_t workspace_bytes, void* stream) {
+  return build_mask(q, k, g, p, sta_radius, mask_bits, kv_count, kv_idx, workspace, workspace_bytes, stream, true);
+}
+
 dbst_status dbst_mask_from_bits(const uint32_t* bits, const dbst_geom* g, int32_t* kv_count, int16_t* kv_idx,
                                 void* stream) {
   if (!geom_ok(g) || !bits || !kv_count || !kv_idx) return DBST_EINVAL;
@@ -310,12 +355,25 @@ dbst_status dbst_block_sparse_attn(const void* q, const void* k, const void* v, 
                                    void* stream) {
   if (!kv_count || !kv_idx) return DBST_EINVAL;
   if (!aligned16(kv_count) || !aligned16(kv_idx)) return DBST_EINVAL;
-  return attn_common(q, k, v, g, kv_count, kv_idx, scale, o, lse, stream);
+  return attn_common(q, k, v, g, kv_count, kv_idx, scale, o, lse, stream, false);
 }
 
 dbst_status dbst_dense_attn(const void* q, const void* k, const void* v, const dbst_geom* g, float scale, void* o,
                             float* lse, void* stream) {
-  return attn_common(q, k, v, g, nullptr, nullptr, scale, o, lse, stream);
+  return attn_common(q, k, v, g, nullptr, nullptr, scale, o, lse, stream, false);
+}
+
+dbst_status dbst_block_sparse_attn_raster(const void* q, const void* k, const void* v, const dbst_geom* g,
+                                          const int32_t* kv_count, const int16_t* kv_idx, float scale, void* o,
+                                          float* lse, void* stream) {
+  if (!kv_count || !kv_idx) return DBST_EINVAL;
+  if (!aligned16(kv_count) || !aligned16(kv_idx)) return DBST_EINVAL;
+  return attn_common(q, k, v, g, kv_count, kv_idx, scale, o, lse, stream, true);
+}
+
+dbst_status dbst_dense_attn_raster(const void* q, const void* k, const void* v, const dbst_geom* g, float scale,
+                                   void* o, float* lse, void* stream) {
+  return attn_common(q, k, v, g, nullptr, nullptr, scale, o, lse, stream, true);
 }
 
 dbst_status dbst_get_error(void* stream) {

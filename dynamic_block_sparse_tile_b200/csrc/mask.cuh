@@ -10,16 +10,19 @@
 #pragma once
 #include <cstdint>
 #include "ptx.cuh"
+#include "reorder.cuh"
 
 namespace dbst {
 
 // ---------------------------------------------------------------------------
 // Block mean-pool: one warp per 64-token block; out[blk][c] = mean (float64).
+// RASTER: q and k are in raster token order and the block's rows are gathered
+// through the tile permutation (the same rows, summed in the same order).
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool RASTER>
 __global__ void __launch_bounds__(256) pool_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
                                                    double* __restrict__ qp, double* __restrict__ kp,
-                                                   long long nblocks) {
+                                                   long long nblocks, int NB, TileGeo tg) {
   constexpr int CPR = D / 8;            // 16-byte chunks per token row
   constexpr int RPW = 32 / CPR;         // token rows covered by one warp pass
   const int lane = threadIdx.x & 31;
@@ -31,12 +34,15 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint4* __restrict__ q, 
     const bool isk = w >= nblocks;
     const long long b = isk ? w - nblocks : w;
     const uint4* src = (isk ? k : q) + b * 64 * CPR;
+    const uint4* head = (isk ? k : q) + (b / NB) * static_cast<long long>(tg.N) * CPR;
+    const int blk = static_cast<int>(b % NB);
     double acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.0;
 #pragma unroll 8
     for (int r = r0; r < 64; r += RPW) {
-      const uint4 v = ld_stream(src + r * CPR + ch);
+      const uint4 v = RASTER ? ld_stream(head + static_cast<long long>(tiled_to_raster(blk * 64 + r, tg)) * CPR + ch)
+                             : ld_stream(src + r * CPR + ch);
       const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {

@@ -129,6 +129,31 @@ dbst_status dbst_dense_attn(const void* q, const void* k, const void* v, const d
                             float scale, void* o, float* lse, void* stream);
 
 /*
+ * The same three operations on tensors in the caller's raster token order,
+ * with the tile reorder ("Fractal Flattening", NABLA page, section
+ * "Méthodologie : NABLA") folded into the kernels' own loads and stores
+ * instead of separate dbst_tile_reorder / dbst_tile_unreorder passes.
+ *   q, k, v, o : raster [B,H,N,D] bf16, token n = (t*Y + y)*X + x
+ *   lse        : raster [B,H,N] float32 or NULL
+ * The mask outputs (mask_bits, kv_count, kv_idx) are indexed by tile-ordered
+ * block as in the tiled entry points, and the workspace is the same
+ * (dbst_mask_workspace_bytes).  Results are bit-identical to the tiled entry
+ * points applied to dbst_tile_reorder'ed inputs, followed by
+ * dbst_tile_unreorder of o (and the same permutation of lse).  Arguments,
+ * ownership and errors as for the tiled entry points; in addition q, k, v
+ * and o must each be 16-byte aligned (their row stride D*2 bytes always is).
+ */
+dbst_status dbst_build_block_mask_raster(const void* q, const void* k, const dbst_geom* g,
+                                         float p, int sta_radius,
+                                         uint32_t* mask_bits, int32_t* kv_count, int16_t* kv_idx,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+dbst_status dbst_block_sparse_attn_raster(const void* q, const void* k, const void* v, const dbst_geom* g,
+                                          const int32_t* kv_count, const int16_t* kv_idx, float scale,
+                                          void* o, float* lse, void* stream);
+dbst_status dbst_dense_attn_raster(const void* q, const void* k, const void* v, const dbst_geom* g,
+                                   float scale, void* o, float* lse, void* stream);
+
+/*
  * Allocation-free variant of dbst_build_block_mask.  The paper has no
  * counterpart: this entry point exists for callers that cannot call
  * cudaMalloc or hand the library a workspace — for example a serving loop or

@@ -79,6 +79,16 @@ def test_null_and_misaligned_pointers(lib):
                                       ctypes.c_void_p((1 << 20) + 2), None) == dbst.DBST_EINVAL
     assert lib.dbst_dense_attn(a, a, a, ctypes.byref(g), float("nan"), a, None, None) == dbst.DBST_EINVAL
     assert lib.dbst_tile_reorder(a, b, None, None) == dbst.DBST_EINVAL
+    # the raster entry points validate exactly like the tiled ones
+    assert lib.dbst_block_sparse_attn_raster(a, a, a, ctypes.byref(g), None, a, 0.0, a, None, None) == dbst.DBST_EINVAL
+    assert lib.dbst_block_sparse_attn_raster(a, ctypes.c_void_p((1 << 20) + 8), a, ctypes.byref(g), a, a, 0.0, a,
+                                             None, None) == dbst.DBST_EINVAL
+    assert lib.dbst_dense_attn_raster(a, a, a, ctypes.byref(g), float("inf"), a, None, None) == dbst.DBST_EINVAL
+    assert lib.dbst_dense_attn_raster(None, a, a, ctypes.byref(g), 0.0, a, None, None) == dbst.DBST_EINVAL
+    ws = lib.dbst_mask_workspace_bytes(ctypes.byref(g))
+    assert lib.dbst_build_block_mask_raster(None, a, ctypes.byref(g), 0.9, -1, a, a, a, a, ws, None) == dbst.DBST_EINVAL
+    assert lib.dbst_build_block_mask_raster(a, a, ctypes.byref(g), 0.9, -1, a, a, a, a, ws - 1, None) == dbst.DBST_EINVAL
+    assert lib.dbst_build_block_mask_raster(a, a, ctypes.byref(g), 1.5, -1, a, a, a, a, ws, None) == dbst.DBST_EINVAL
 
 
 @pytest.mark.parametrize("p", [0.0, -0.5, 1.0000001, 2.0, float("nan")])
