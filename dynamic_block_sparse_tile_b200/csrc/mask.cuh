@@ -343,6 +343,11 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
 // it; the answer lies above the pivot, is the pivot, or lies below it, and
 // the pivot always leaves the live set.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_sum_f32(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
 __device__ __forceinline__ double warp_sum_f64(double v) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
@@ -374,7 +379,10 @@ __global__ void __launch_bounds__(128) select_warp_kernel(const double* __restri
   const int i = static_cast<int>(row % g.NB);
   const double* srow = S + row * g.NB;
 
-  // keys from the logits; unnormalised masses e^(s - max) in float32 (summed in float64)
+  // keys from the float64 logits; unnormalised masses e^(s - max) and their sums in float32.  A
+  // row of at most 1024 masses, each <= 1, sums with a relative error below 1024 * 2^-24 = 6e-5,
+  // so a kept set can differ from a float64 reference only where the cumulative mass lies that
+  // close to p; the order itself comes from the exact logits.
   float m[NPT];
   unsigned long long key[NPT];
   double mx = -INFINITY;
@@ -386,21 +394,21 @@ __global__ void __launch_bounds__(128) select_warp_kernel(const double* __restri
     mx = fmax(mx, sj);
   }
   mx = warp_max_f64(mx);
-  double total = 0.0;
+  float total = 0.0f;
 #pragma unroll
   for (int u = 0; u < NPT; ++u) {
     const int j = lane + 32 * u;
     const double sj = (j < g.NB) ? srow[j] : -INFINITY;
     m[u] = (j < g.NB) ? fast_exp2(static_cast<float>((sj - mx) * 1.4426950408889634)) : 0.0f;
-    total += static_cast<double>(m[u]);
+    total += m[u];
   }
-  total = warp_sum_f64(total);
-  const double target = g.p * total;            // cumulative mass to reach, unnormalised
+  total = warp_sum_f32(total);
+  const float target = static_cast<float>(g.p * static_cast<double>(total));   // cumulative mass to reach
 
   unsigned long long thr = 0ull;   // keep key >= thr (0 keeps all)
   if (g.p < 1.0) {
     unsigned long long lo = 0ull, hi = ~0ull;   // the answer lies in (lo, hi]
-    double above = 0.0;                         // mass of keys > hi
+    float above = 0.0f;                         // mass of keys > hi
     for (int round = 0; round < 4 * 32 * NPT; ++round) {
       int mycnt = 0;
       unsigned long long mine = 0ull;
@@ -415,18 +423,18 @@ __global__ void __launch_bounds__(128) select_warp_kernel(const double* __restri
       const int nh = __popc(holders);
       const int pick = __fns(holders, 0, 1 + (round * 7) % nh);
       const unsigned long long pivot = __shfl_sync(0xffffffffu, mine, pick);
-      double gt = 0.0, eq = 0.0;
+      float gt = 0.0f, eq = 0.0f;
 #pragma unroll
       for (int u = 0; u < NPT; ++u) {
         const bool live = key[u] > lo && key[u] <= hi;
-        if (live && key[u] > pivot) gt += static_cast<double>(m[u]);
-        if (key[u] == pivot) eq = static_cast<double>(m[u]);
+        if (live && key[u] > pivot) gt += m[u];
+        if (key[u] == pivot) eq = m[u];
       }
-      const double g_above = above + warp_sum_f64(gt);
+      const float g_above = above + warp_sum_f32(gt);
       if (g_above >= target) {
         lo = pivot;                             // the k*-th key is above the pivot
       } else {
-        const double f = g_above + warp_sum_f64(eq);
+        const float f = g_above + warp_sum_f32(eq);
         if (f >= target) {
           thr = pivot;                          // the pivot is the k*-th key
           break;
