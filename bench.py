@@ -188,6 +188,21 @@ def oracle_sample(w: S.Workload, p: float, budget_s: float, seed: int = 7):
     return flops / elapsed / 1e12, elapsed, desc
 
 
+def max_over_ranks(vals, world: int, device: str):
+    """Element-wise max over ranks of per-rank timings: the slowest rank sets the job's time."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(vals), dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_tflops(world: int, flops_per_rank: float, ms_per_step: float) -> float:
+    """Whole-job throughput under weak scaling: every rank runs its own problem of flops_per_rank per step."""
+    return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 def run_reference(args, w, p):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -404,13 +419,10 @@ def main():
     e2e_ms = s2.elapsed_time(e2)
     dbst.get_error()
 
-    t = torch.tensor([ms_total, e2e_ms, attn_ms, mask_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total, e2e_ms, attn_ms, mask_ms = (float(x) for x in t.tolist())
+    ms_total, e2e_ms, attn_ms, mask_ms = max_over_ranks([ms_total, e2e_ms, attn_ms, mask_ms], world, "cuda")
     ms_step = ms_total / args.steps
-    value = world * flops / (ms_step * 1e-3) / 1e12
-    e2e_value = world * flops / (e2e_ms / args.steps * 1e-3) / 1e12
+    value = job_tflops(world, flops, ms_step)
+    e2e_value = job_tflops(world, flops, e2e_ms / args.steps)
 
     hbm, bf16, bf16_sus, src = peaks()
     attn_tflops = flops / (attn_ms * 1e-3) / 1e12
