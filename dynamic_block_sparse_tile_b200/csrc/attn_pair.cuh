@@ -121,6 +121,23 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   uint32_t* s_misc = reinterpret_cast<uint32_t*>(sm + PairSmem::kMisc);
   volatile uint32_t* s_abort = s_misc + 2;
   auto bar = [&](int slot) -> uint32_t { return sbase + PairSmem::kBars + 8u * slot; };
+  // Bounded wait used inside the softmax loops.  The abort flag is read only when the phase is
+  // not already complete, so a wait that succeeds at once costs one barrier test; `live` turns
+  // false for good once this warp times out or sees another role's abort, and later waits are
+  // then skipped so the warp runs its remaining iterations without blocking.
+  auto wait_live = [&](uint32_t mb, uint32_t parity, bool& live) {
+    if (!live || mbar_try(mb, parity)) return;
+    const long long t0 = clock64();
+    while (!mbar_try(mb, parity)) {
+      if (*s_abort) { live = false; return; }
+      if (clock64() - t0 > kWaitLimitCycles) {
+        record_error(kErrTimeout);
+        *s_abort = 1;
+        live = false;
+        return;
+      }
+    }
+  };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int NB = prm.NB, NW = (NB + 31) >> 5;
@@ -339,13 +356,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const uint32_t lrow = static_cast<uint32_t>(32 * q) << 16;
     const float sc = prm.scale_log2;
     float m = -INFINITY;                      // running reference max (log2 units) of this row
+    bool live = true;
     for (int t = 0; t < T; ++t) {
       const int b = t & 1;
-      bool live = (*s_abort == 0);
-      if (live && !mbar_wait(bar(PB_SFULL + b), (t >> 1) & 1)) {
-        *s_abort = 1;
-        live = false;
-      }
+      wait_live(bar(PB_SFULL + b), (t >> 1) & 1, live);
       tc_fence_after();
       const bool v0 = (s_union[2 * t] >> (16 + side)) & 1;
       const bool v1 = (2 * t + 1 < nu) && ((s_union[2 * t + 1] >> (16 + side)) & 1);
@@ -372,14 +386,16 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         if (m != -INFINITY) a = fast_exp2(m - tmax);
         m = tmax;
       }
+      // P buffer b is rewritten for tile t only after PV(t-2), its last reader, has completed.  The
+      // exponential warps learn that from the reference-ready barrier, published after this wait.
+      // The same wait keeps this warp (which runs ahead) from arriving on P full for tile t while
+      // that barrier's phase still waits for the exponential warps' tile t-2.
+      if (t >= 2) wait_live(bar(PB_PVDONE + b), ((t - 2) >> 1) & 1, live);
       s_ring[b * 128 + r] = make_float2(m, a);
       mbar_arrive(bar(PB_MREADY + 4 * b + q));
       if (__any_sync(0xffffffffu, a != 1.0f)) {
         // rescale these rows of O; PV(t-1), the last product into O, must be done
-        if (live && !mbar_wait(bar(PB_PVDONE + ((t - 1) & 1)), ((t - 1) >> 1) & 1)) {
-          *s_abort = 1;
-          live = false;
-        }
+        wait_live(bar(PB_PVDONE + ((t - 1) & 1)), ((t - 1) >> 1) & 1, live);
         tc_fence_after();
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
@@ -391,13 +407,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           tmem_st32(tmem + kTmemO + c0 + lrow, ov);
         }
         tmem_wait_st();
-      }
-      // This warp runs ahead of the exponential warps: its arrival for tile t must not land in the
-      // phase of PFULL[b] that still waits for their tile t-2.  PV(t-2) completing shows that phase
-      // is over (and the exponential warps wait for the same event before writing P(t)).
-      if (live && t >= 2 && !mbar_wait(bar(PB_PVDONE + b), ((t - 2) >> 1) & 1)) {
-        *s_abort = 1;
-        live = false;
       }
       tc_fence_before();
       mbar_arrive(bar(PB_PFULL + b));
@@ -413,20 +422,18 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const float2 sc2 = make_float2(sc, sc);
     float m = -INFINITY;                      // this row's reference for the current tile
     float2 l2 = make_float2(0.0f, 0.0f);      // partial row sum of 2^(x - m) over this warp's columns
+    bool live = true;
+    int ent = (hc < nu) ? s_union[hc] : 0;    // union entry of this warp's key block, one tile ahead
     for (int t = 0; t < T; ++t) {
       const int b = t & 1;
-      bool live = (*s_abort == 0);
-      if (live && !mbar_wait(bar(PB_MREADY + 4 * b + q), (t >> 1) & 1)) {
-        *s_abort = 1;
-        live = false;
-      }
+      wait_live(bar(PB_MREADY + 4 * b + q), (t >> 1) & 1, live);
       const float2 ma = s_ring[b * 128 + r];
+      const bool vh = (2 * t + hc < nu) && ((ent >> (16 + side)) & 1);   // uniform per warp
+      ent = (2 * t + 2 + hc < nu) ? s_union[2 * t + 2 + hc] : 0;
       m = ma.x;
       l2.x *= ma.y;
       l2.y *= ma.y;
       tc_fence_after();
-      const int ei = (2 * t + hc < nu) ? 2 * t + hc : 2 * t;
-      const bool vh = (2 * t + hc < nu) && ((s_union[ei] >> (16 + side)) & 1);   // uniform per warp
       uint32_t u[64];
       if (vh) {
         tmem_ld32(tmem + kTmemS + 128u * b + 64u * hc + lrow, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
@@ -450,12 +457,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 #pragma unroll
         for (int c = 0; c < 32; ++c) pk[c] = 0u;
       }
-      // the P buffer was last read by PV(t-2)
-      if (live && t >= 2 && !mbar_wait(bar(PB_PVDONE + b), ((t - 2) >> 1) & 1)) {
-        *s_abort = 1;
-        live = false;
-      }
-      tc_fence_after();
+      // PV(t-2), the P buffer's last reader, completed before the reference for tile t was published
       tmem_st32(tmem + kTmemP + 64u * b + 32u * hc + lrow, pk);
       tmem_wait_st();
       tc_fence_before();
