@@ -5,8 +5,8 @@ latent workload (B=1, H=40, D=128, token grid 21x32x56 in 1x8x8 tiles,
 N=37632, 588 blocks; CDF threshold p=0.9; seeded synthetic q/k/v).  Default
 (`--path fused`): raster q, k, v in, raster o out, the tile reorder done by the
 kernels' own loads and stores:
-    build_block_mask_raster(q, k) -> block_sparse_attn_raster(q, k, v) -> o
-(4 launches: pool, pooled logits, select, attention).  `--path explicit` runs
+    build_block_mask_raster(q, k) -> pair_query_blocks -> block_sparse_attn_raster(q, k, v, pairs) -> o
+(5 launches: pool, pooled logits, select, query-block pairing, attention).  `--path explicit` runs
 the same steps as separate passes (8 launches):
     tile_reorder(q, k, v) -> build_block_mask -> block_sparse_attn -> tile_unreorder(o)
 
@@ -339,8 +339,9 @@ def main():
     o_host = torch.empty_like(host[0]).pin_memory()
     stream = torch.cuda.current_stream()
     fused = args.path == "fused"
-    # fused: pool + logits + select + attention; explicit: 3 reorders + those 4 + unreorder
-    launches_per_step = 4 if fused else 8
+    # fused: pool + logits + select + pairing + attention; explicit: 3 reorders + 4 + unreorder
+    launches_per_step = 5 if fused else 8
+    pairs = torch.empty((g.B, g.H, (g.NB + 1) // 2), dtype=torch.int32, device="cuda")
 
     ev = {}
 
@@ -354,13 +355,14 @@ def main():
             e0.record(stream)
         if fused:
             dbst.build_block_mask_raster(q, k, g, p, w.sta_radius, workspace=ws, out=(bits, cnt, idx))
+            dbst.pair_query_blocks(bits, g, out=pairs)
         else:
             dbst.build_block_mask(qt, kt, g, p, w.sta_radius, workspace=ws, out=(bits, cnt, idx))
         if timed_parts:
             e1 = torch.cuda.Event(enable_timing=True)
             e1.record(stream)
         if fused:
-            dbst.block_sparse_attn_raster(q, k, v, g, cnt, idx, 0.0, want_lse=True, out=o, lse=lse)
+            dbst.block_sparse_attn_raster(q, k, v, g, cnt, idx, 0.0, want_lse=True, out=o, lse=lse, pairs=pairs)
         else:
             dbst.block_sparse_attn(qt, kt, vt, g, cnt, idx, 0.0, want_lse=True, out=ot, lse=lse)
         if timed_parts:

@@ -19,7 +19,8 @@ import torch
 
 __all__ = ["Geom", "DbstError", "lib_path", "load", "tile_reorder", "tile_unreorder", "mask_workspace_bytes",
            "build_block_mask", "build_block_mask_noalloc", "mask_from_bits", "block_sparse_attn", "dense_attn",
-           "build_block_mask_raster", "block_sparse_attn_raster", "dense_attn_raster", "get_error", "EXPORTS"]
+           "build_block_mask_raster", "block_sparse_attn_raster", "dense_attn_raster", "pair_query_blocks",
+           "get_error", "EXPORTS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libdbst.so")
@@ -28,7 +29,7 @@ _LIB_PATH = os.path.join(_HERE, "libdbst.so")
 EXPORTS = ("dbst_status_string", "dbst_tile_reorder", "dbst_tile_unreorder", "dbst_mask_workspace_bytes",
            "dbst_build_block_mask", "dbst_mask_from_bits", "dbst_block_sparse_attn", "dbst_dense_attn",
            "dbst_get_error", "dbst_build_block_mask_noalloc", "dbst_build_block_mask_raster",
-           "dbst_block_sparse_attn_raster", "dbst_dense_attn_raster")
+           "dbst_block_sparse_attn_raster", "dbst_dense_attn_raster", "dbst_pair_query_blocks")
 
 DBST_OK, DBST_EINVAL, DBST_ECUDA, DBST_ETIMEOUT, DBST_EBOUNDS, DBST_ETOOLARGE = 0, 1, 2, 3, 4, 5
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -86,9 +87,11 @@ def load() -> ctypes.CDLL:
         getattr(lib, name).argtypes = [vp, vp, gp, f32, i32, vp, vp, vp, vp, ctypes.c_size_t, vp]
         getattr(lib, name).restype = i32
     lib.dbst_mask_from_bits.argtypes, lib.dbst_mask_from_bits.restype = [vp, gp, vp, vp, vp], i32
-    for name in ("dbst_block_sparse_attn", "dbst_block_sparse_attn_raster"):
-        getattr(lib, name).argtypes = [vp, vp, vp, gp, vp, vp, f32, vp, vp, vp]
-        getattr(lib, name).restype = i32
+    lib.dbst_block_sparse_attn.argtypes = [vp, vp, vp, gp, vp, vp, f32, vp, vp, vp]
+    lib.dbst_block_sparse_attn.restype = i32
+    lib.dbst_block_sparse_attn_raster.argtypes = [vp, vp, vp, gp, vp, vp, vp, f32, vp, vp, vp]
+    lib.dbst_block_sparse_attn_raster.restype = i32
+    lib.dbst_pair_query_blocks.argtypes, lib.dbst_pair_query_blocks.restype = [vp, gp, vp, vp], i32
     for name in ("dbst_dense_attn", "dbst_dense_attn_raster"):
         getattr(lib, name).argtypes, getattr(lib, name).restype = [vp, vp, vp, gp, f32, vp, vp, vp], i32
     lib.dbst_get_error.argtypes, lib.dbst_get_error.restype = [vp], i32
@@ -221,13 +224,30 @@ def block_sparse_attn(q, k, v, g: Geom, kv_count, kv_idx, scale: float = 0.0, wa
 
 
 def block_sparse_attn_raster(q, k, v, g: Geom, kv_count, kv_idx, scale: float = 0.0, want_lse: bool = True,
-                             out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None):
-    """Attention over kept blocks on raster-order tensors (``dbst_block_sparse_attn_raster``)."""
+                             out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                             pairs: Optional[torch.Tensor] = None):
+    """Attention over kept blocks on raster-order tensors (``dbst_block_sparse_attn_raster``).
+
+    ``pairs`` is an optional schedule from :func:`pair_query_blocks`.
+    """
+    if pairs is not None:
+        _need(pairs, torch.int32, (g.B, g.H, (g.NB + 1) // 2), "pairs")
     return _block_sparse_attn("dbst_block_sparse_attn_raster", q, k, v, g, kv_count, kv_idx, scale, want_lse, out,
-                              lse)
+                              lse, pairs=pairs, with_pairs=True)
 
 
-def _block_sparse_attn(fn: str, q, k, v, g: Geom, kv_count, kv_idx, scale, want_lse, out, lse):
+def pair_query_blocks(mask_bits: torch.Tensor, g: Geom, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Query-block pairs for the attention kernel (``dbst_pair_query_blocks``) -> int32 [B, H, ceil(NB/2)]."""
+    _need(mask_bits, torch.int32, (g.B, g.H, g.NB, g.NW), "mask_bits")
+    pairs = torch.empty((g.B, g.H, (g.NB + 1) // 2), dtype=torch.int32, device=mask_bits.device) if out is None else out
+    _need(pairs, torch.int32, (g.B, g.H, (g.NB + 1) // 2), "pairs")
+    _check(load().dbst_pair_query_blocks(_ptr(mask_bits), ctypes.byref(g), _ptr(pairs), _stream()),
+           "dbst_pair_query_blocks")
+    return pairs
+
+
+def _block_sparse_attn(fn: str, q, k, v, g: Geom, kv_count, kv_idx, scale, want_lse, out, lse, pairs=None,
+                       with_pairs=False):
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, torch.bfloat16, _qkv_shape(g), n)
     _need(kv_count, torch.int32, (g.B, g.H, g.NB), "kv_count")
@@ -235,8 +255,13 @@ def _block_sparse_attn(fn: str, q, k, v, g: Geom, kv_count, kv_idx, scale, want_
     o = torch.empty_like(q) if out is None else out
     if want_lse and lse is None:
         lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device=q.device)
-    _check(getattr(load(), fn)(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(g), _ptr(kv_count), _ptr(kv_idx),
-                               float(scale), _ptr(o), _ptr(lse if want_lse else None), _stream()), fn)
+    lib = load()
+    if with_pairs:
+        _check(getattr(lib, fn)(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(g), _ptr(kv_count), _ptr(kv_idx), _ptr(pairs),
+                                float(scale), _ptr(o), _ptr(lse if want_lse else None), _stream()), fn)
+    else:
+        _check(getattr(lib, fn)(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(g), _ptr(kv_count), _ptr(kv_idx),
+                                float(scale), _ptr(o), _ptr(lse if want_lse else None), _stream()), fn)
     return o, (lse if want_lse else None)
 
 

@@ -49,7 +49,8 @@ struct PairParams {
   __nv_bfloat16* o;          // tiled [BH, N, D]
   float* lse;                // [BH, N] or null
   int NB, N;
-  int pair_stride;           // qb = qa + pair_stride
+  const int32_t* pairs;      // [BH][pairs_per_head] qa | qb << 16 (qb 0xFFFF: none), or null
+  int pair_stride;           // without a pair list: qb = qa + pair_stride
   int pairs_per_head;
   float scale_log2;          // softmax scale * log2(e)
   TileGeo tg;                // token grid and tile shape (raster layout only)
@@ -143,9 +144,20 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   const int NB = prm.NB, NW = (NB + 31) >> 5;
   const long long bh = blockIdx.x / prm.pairs_per_head;
   const int pi = blockIdx.x - static_cast<int>(bh * prm.pairs_per_head);
-  const int ps = prm.pair_stride;
-  const int qa = (pi / ps) * 2 * ps + (pi % ps);
-  const int qb = qa + ps;
+  int qa, qb;
+  if (prm.pairs != nullptr) {
+    const int32_t ent = prm.pairs[bh * prm.pairs_per_head + pi];
+    qa = ent & 0xFFFF;
+    qb = (ent >> 16) & 0xFFFF;
+    if (qa >= NB || (qb >= NB && qb != 0xFFFF)) {   // not a block of this head: report, compute nothing
+      if (threadIdx.x == 0) record_error(kErrBounds);
+      return;
+    }
+  } else {
+    const int ps = prm.pair_stride;
+    qa = (pi / ps) * 2 * ps + (pi % ps);
+    qb = qa + ps;
+  }
   const bool has_b = qb < NB;
   // global row of row rr (0..63) of query block blk of this head
   auto out_row = [&](int blk, int rr) -> long long {

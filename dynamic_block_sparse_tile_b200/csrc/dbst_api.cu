@@ -12,6 +12,7 @@
 
 #include "../../include/dbst.h"
 #include "attn_pair.cuh"
+#include "pairing.cuh"
 #include "mask.cuh"
 #include "ptx.cuh"
 #include "reorder.cuh"
@@ -165,7 +166,7 @@ bool make_tmap_raster(CUtensorMap* m, const void* base, const dbst_geom* g) {
 
 template <int D, bool RASTER>
 dbst_status launch_pair(const void* q, const void* k, const void* v, const dbst_geom* g, const int32_t* cnt,
-                        const int16_t* idx, float scale, void* o, float* lse, cudaStream_t s) {
+                        const int16_t* idx, const int32_t* pairs, float scale, void* o, float* lse, cudaStream_t s) {
   const long long rows = bh_count(g) * tokens(g);
   CUtensorMap tq, tk, tv;
   if (RASTER) {
@@ -181,8 +182,9 @@ dbst_status launch_pair(const void* q, const void* k, const void* v, const dbst_
   p.lse = lse;
   p.NB = nblocks(g);
   p.N = static_cast<int>(tokens(g));
+  p.pairs = pairs;
   p.pair_stride = pair_stride(g);
-  p.pairs_per_head = ((p.NB + 2 * p.pair_stride - 1) / (2 * p.pair_stride)) * p.pair_stride;
+  p.pairs_per_head = pairs ? (p.NB + 1) / 2 : ((p.NB + 2 * p.pair_stride - 1) / (2 * p.pair_stride)) * p.pair_stride;
   const float sc = scale > 0.0f ? scale : 1.0f / std::sqrt(static_cast<float>(D));
   p.scale_log2 = sc * 1.4426950408889634f;
   const int smem = dbst::PairSmem::kBytes + 1024;
@@ -199,17 +201,19 @@ dbst_status launch_pair(const void* q, const void* k, const void* v, const dbst_
 }
 
 dbst_status attn_common(const void* q, const void* k, const void* v, const dbst_geom* g, const int32_t* cnt,
-                        const int16_t* idx, float scale, void* o, float* lse, void* stream, bool raster) {
+                        const int16_t* idx, const int32_t* pairs, float scale, void* o, float* lse, void* stream,
+                        bool raster) {
   if (!geom_ok(g) || !q || !k || !v || !o) return DBST_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return DBST_EINVAL;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return DBST_EINVAL;
   if (!(std::isfinite(scale))) return DBST_EINVAL;
   auto s = static_cast<cudaStream_t>(stream);
+  if (pairs && (reinterpret_cast<uintptr_t>(pairs) & 3u)) return DBST_EINVAL;
   if (raster)
-    return g->D == 128 ? launch_pair<128, true>(q, k, v, g, cnt, idx, scale, o, lse, s)
-                       : launch_pair<64, true>(q, k, v, g, cnt, idx, scale, o, lse, s);
-  return g->D == 128 ? launch_pair<128, false>(q, k, v, g, cnt, idx, scale, o, lse, s)
-                     : launch_pair<64, false>(q, k, v, g, cnt, idx, scale, o, lse, s);
+    return g->D == 128 ? launch_pair<128, true>(q, k, v, g, cnt, idx, pairs, scale, o, lse, s)
+                       : launch_pair<64, true>(q, k, v, g, cnt, idx, pairs, scale, o, lse, s);
+  return g->D == 128 ? launch_pair<128, false>(q, k, v, g, cnt, idx, pairs, scale, o, lse, s)
+                     : launch_pair<64, false>(q, k, v, g, cnt, idx, pairs, scale, o, lse, s);
 }
 
 template <int NPT>
@@ -355,25 +359,46 @@ dbst_status dbst_block_sparse_attn(const void* q, const void* k, const void* v, 
                                    void* stream) {
   if (!kv_count || !kv_idx) return DBST_EINVAL;
   if (!aligned16(kv_count) || !aligned16(kv_idx)) return DBST_EINVAL;
-  return attn_common(q, k, v, g, kv_count, kv_idx, scale, o, lse, stream, false);
+  return attn_common(q, k, v, g, kv_count, kv_idx, nullptr, scale, o, lse, stream, false);
 }
 
 dbst_status dbst_dense_attn(const void* q, const void* k, const void* v, const dbst_geom* g, float scale, void* o,
                             float* lse, void* stream) {
-  return attn_common(q, k, v, g, nullptr, nullptr, scale, o, lse, stream, false);
+  return attn_common(q, k, v, g, nullptr, nullptr, nullptr, scale, o, lse, stream, false);
 }
 
 dbst_status dbst_block_sparse_attn_raster(const void* q, const void* k, const void* v, const dbst_geom* g,
-                                          const int32_t* kv_count, const int16_t* kv_idx, float scale, void* o,
-                                          float* lse, void* stream) {
+                                          const int32_t* kv_count, const int16_t* kv_idx, const int32_t* pairs,
+                                          float scale, void* o, float* lse, void* stream) {
   if (!kv_count || !kv_idx) return DBST_EINVAL;
   if (!aligned16(kv_count) || !aligned16(kv_idx)) return DBST_EINVAL;
-  return attn_common(q, k, v, g, kv_count, kv_idx, scale, o, lse, stream, true);
+  return attn_common(q, k, v, g, kv_count, kv_idx, pairs, scale, o, lse, stream, true);
 }
 
 dbst_status dbst_dense_attn_raster(const void* q, const void* k, const void* v, const dbst_geom* g, float scale,
                                    void* o, float* lse, void* stream) {
-  return attn_common(q, k, v, g, nullptr, nullptr, scale, o, lse, stream, true);
+  return attn_common(q, k, v, g, nullptr, nullptr, nullptr, scale, o, lse, stream, true);
+}
+
+dbst_status dbst_pair_query_blocks(const uint32_t* mask_bits, const dbst_geom* g, int32_t* pairs, void* stream) {
+  if (!geom_ok(g) || !mask_bits || !pairs) return DBST_EINVAL;
+  if (!aligned16(mask_bits) || (reinterpret_cast<uintptr_t>(pairs) & 3u)) return DBST_EINVAL;
+  const long long bh = bh_count(g);
+  if (bh >= (1ll << 31)) return DBST_EINVAL;
+  dbst::PairingGeo pg;
+  pg.NB = nblocks(g);
+  pg.NW = (pg.NB + 31) / 32;
+  pg.nX = g->X / g->tx;
+  pg.nY = g->Y / g->ty;
+  pg.nT = g->T / g->tt;
+  const size_t smem = dbst::pairing_smem_bytes(pg.NB);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(dbst::pair_blocks_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return DBST_ECUDA;
+  dbst::pair_blocks_kernel<<<static_cast<unsigned>(bh), dbst::kPairingThreads, smem,
+                             static_cast<cudaStream_t>(stream)>>>(mask_bits, pg, pairs);
+  return launch_status();
 }
 
 dbst_status dbst_get_error(void* stream) {

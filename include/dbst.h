@@ -148,10 +148,28 @@ dbst_status dbst_build_block_mask_raster(const void* q, const void* k, const dbs
                                          uint32_t* mask_bits, int32_t* kv_count, int16_t* kv_idx,
                                          void* workspace, size_t workspace_bytes, void* stream);
 dbst_status dbst_block_sparse_attn_raster(const void* q, const void* k, const void* v, const dbst_geom* g,
-                                          const int32_t* kv_count, const int16_t* kv_idx, float scale,
+                                          const int32_t* kv_count, const int16_t* kv_idx,
+                                          const int32_t* pairs, float scale,
                                           void* o, float* lse, void* stream);
 dbst_status dbst_dense_attn_raster(const void* q, const void* k, const void* v, const dbst_geom* g,
                                    float scale, void* o, float* lse, void* stream);
+
+/*
+ * Schedule for the attention kernel (no counterpart on the pages: it changes
+ * which query blocks share a thread block, never which keys a query sees).
+ * The kernel runs two 64-token query blocks at a time over the union of their
+ * lists; this pairs each block with one of its six face neighbours on the tile
+ * grid so that the unions stay small (greedy on the tiles saved, from the mask
+ * rows' overlaps), and pairs the rest in ascending order.
+ *   mask_bits : [B,H,NB,ceil(NB/32)] uint32 as written by the mask builders
+ *   pairs     : out, [B,H,ceil(NB/2)] int32, entry = qa | qb << 16 with
+ *               qb = 0xFFFF for a single block; every block of a head appears
+ *               exactly once.  4-byte aligned.
+ * Pass `pairs` to dbst_block_sparse_attn_raster (NULL there selects fixed
+ * pairs of neighbours one tile step apart).  An entry naming a block outside
+ * [0, NB) makes the attention skip that entry and report DBST_EBOUNDS.
+ */
+dbst_status dbst_pair_query_blocks(const uint32_t* mask_bits, const dbst_geom* g, int32_t* pairs, void* stream);
 
 /*
  * Allocation-free variant of dbst_build_block_mask.  The paper has no

@@ -80,9 +80,15 @@ def test_null_and_misaligned_pointers(lib):
     assert lib.dbst_dense_attn(a, a, a, ctypes.byref(g), float("nan"), a, None, None) == dbst.DBST_EINVAL
     assert lib.dbst_tile_reorder(a, b, None, None) == dbst.DBST_EINVAL
     # the raster entry points validate exactly like the tiled ones
-    assert lib.dbst_block_sparse_attn_raster(a, a, a, ctypes.byref(g), None, a, 0.0, a, None, None) == dbst.DBST_EINVAL
-    assert lib.dbst_block_sparse_attn_raster(a, ctypes.c_void_p((1 << 20) + 8), a, ctypes.byref(g), a, a, 0.0, a,
+    assert lib.dbst_block_sparse_attn_raster(a, a, a, ctypes.byref(g), None, a, None, 0.0, a, None,
+                                             None) == dbst.DBST_EINVAL
+    assert lib.dbst_block_sparse_attn_raster(a, ctypes.c_void_p((1 << 20) + 8), a, ctypes.byref(g), a, a, None, 0.0, a,
                                              None, None) == dbst.DBST_EINVAL
+    assert lib.dbst_block_sparse_attn_raster(a, a, a, ctypes.byref(g), a, a, ctypes.c_void_p((1 << 20) + 2), 0.0, a,
+                                             None, None) == dbst.DBST_EINVAL   # misaligned pair list
+    assert lib.dbst_pair_query_blocks(None, ctypes.byref(g), a, None) == dbst.DBST_EINVAL
+    assert lib.dbst_pair_query_blocks(a, ctypes.byref(g), ctypes.c_void_p((1 << 20) + 1), None) == dbst.DBST_EINVAL
+    assert lib.dbst_pair_query_blocks(a, None, a, None) == dbst.DBST_EINVAL
     assert lib.dbst_dense_attn_raster(a, a, a, ctypes.byref(g), float("inf"), a, None, None) == dbst.DBST_EINVAL
     assert lib.dbst_dense_attn_raster(None, a, a, ctypes.byref(g), 0.0, a, None, None) == dbst.DBST_EINVAL
     ws = lib.dbst_mask_workspace_bytes(ctypes.byref(g))
