@@ -391,13 +391,14 @@ dbst_status dbst_pair_query_blocks(const uint32_t* mask_bits, const dbst_geom* g
   pg.nX = g->X / g->tx;
   pg.nY = g->Y / g->ty;
   pg.nT = g->T / g->tt;
-  const size_t smem = dbst::pairing_smem_bytes(pg.NB);
+  const bool stage = dbst::pairing_rows_bytes(pg.NB, pg.NW) <= static_cast<size_t>(dbst::kPairingStageBytes);
+  const size_t smem = dbst::pairing_smem_bytes(pg.NB, pg.NW, stage);
+  auto kern = stage ? dbst::pair_blocks_kernel<true> : dbst::pair_blocks_kernel<false>;
   if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(dbst::pair_blocks_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
     return DBST_ECUDA;
-  dbst::pair_blocks_kernel<<<static_cast<unsigned>(bh), dbst::kPairingThreads, smem,
-                             static_cast<cudaStream_t>(stream)>>>(mask_bits, pg, pairs);
+  kern<<<static_cast<unsigned>(bh), dbst::kPairingThreads, smem, static_cast<cudaStream_t>(stream)>>>(mask_bits, pg,
+                                                                                                     pairs);
   return launch_status();
 }
 

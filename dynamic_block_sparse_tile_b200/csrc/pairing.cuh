@@ -26,7 +26,9 @@
 
 namespace dbst {
 
-constexpr int kPairingThreads = 256;
+constexpr int kPairingThreads = 512;
+// A head's mask rows are staged in shared memory when they fit in this many bytes.
+constexpr int kPairingStageBytes = 96 * 1024;
 constexpr int kPairingMaxRounds = 64;
 
 struct PairingGeo {
@@ -46,7 +48,8 @@ __device__ __forceinline__ int pairing_neighbour(int v, int k, const PairingGeo&
   }
 }
 
-// Block-wide exclusive scan of one int per thread; returns the total in *total.
+// Block-wide exclusive scan of one int per thread (kPairingThreads / 32 <= 32 warps); the total
+// goes to *total.
 __device__ __forceinline__ int pairing_scan(int x, int* warp_sums, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int incl = x;
@@ -74,7 +77,9 @@ __device__ __forceinline__ int pairing_scan(int x, int* warp_sums, int* total) {
   return r;
 }
 
-// Dynamic shared memory: count[NB], weight[NB][6], partner[NB], best[NB] (ints) + scan scratch.
+// Dynamic shared memory: count[NB], weight[NB][6], partner[NB], best[NB] (ints), scan scratch,
+// then (STAGE) the head's mask rows.
+template <bool STAGE>
 __global__ void __launch_bounds__(kPairingThreads) pair_blocks_kernel(const uint32_t* __restrict__ bits, PairingGeo g,
                                                                       int32_t* __restrict__ pairs) {
   extern __shared__ int pairing_smem[];
@@ -83,11 +88,18 @@ __global__ void __launch_bounds__(kPairingThreads) pair_blocks_kernel(const uint
   int* weight = count + NB;
   int* partner = weight + 6 * NB;
   int* best = partner + NB;
-  int* scratch = best + NB;              // 8 warp sums + 2 totals + change flag
-  volatile int* changed = scratch + 10;
+  int* scratch = best + NB;              // 16 warp sums + 2 totals + change flag
+  volatile int* changed = scratch + 18;
   const long long bh = blockIdx.x;
-  const uint32_t* head = bits + bh * static_cast<long long>(NB) * g.NW;
+  const uint32_t* gh = bits + bh * static_cast<long long>(NB) * g.NW;
   const int tid = threadIdx.x;
+  const uint32_t* head = gh;
+  if constexpr (STAGE) {
+    uint32_t* st = reinterpret_cast<uint32_t*>(scratch + 32);
+    for (int i = tid; i < NB * g.NW; i += kPairingThreads) st[i] = gh[i];
+    head = st;
+    __syncthreads();
+  }
 
   for (int v = tid; v < NB; v += kPairingThreads) {
     int c = 0;
@@ -146,7 +158,7 @@ __global__ void __launch_bounds__(kPairingThreads) pair_blocks_kernel(const uint
   }
 
   // output: matched pairs (by lower index), then the leftovers paired in ascending order
-  constexpr int PER = 16;                // blocks per thread in the scans (NB <= 4096)
+  constexpr int PER = 4096 / kPairingThreads;   // blocks per thread in the scans (NB <= 4096)
   const int v0 = tid * PER;
   int leads = 0, lefts = 0;
   for (int i = 0; i < PER; ++i) {
@@ -155,10 +167,10 @@ __global__ void __launch_bounds__(kPairingThreads) pair_blocks_kernel(const uint
     leads += (partner[v] > v);
     lefts += (partner[v] < 0);
   }
-  const int lead_base = pairing_scan(leads, scratch, scratch + 8);
-  const int n_lead = scratch[8];
-  const int left_base = pairing_scan(lefts, scratch, scratch + 9);
-  const int n_left = scratch[9];
+  const int lead_base = pairing_scan(leads, scratch, scratch + 16);
+  const int n_lead = scratch[16];
+  const int left_base = pairing_scan(lefts, scratch, scratch + 17);
+  const int n_left = scratch[17];
   int32_t* out = pairs + bh * ((NB + 1) / 2);
   int li = lead_base, fi = left_base;
   for (int i = 0; i < PER; ++i) {
@@ -183,6 +195,9 @@ __global__ void __launch_bounds__(kPairingThreads) pair_blocks_kernel(const uint
   }
 }
 
-inline size_t pairing_smem_bytes(int NB) { return static_cast<size_t>(NB) * 9 * sizeof(int) + 16 * sizeof(int); }
+inline size_t pairing_rows_bytes(int NB, int NW) { return static_cast<size_t>(NB) * NW * sizeof(uint32_t); }
+inline size_t pairing_smem_bytes(int NB, int NW, bool stage) {
+  return static_cast<size_t>(NB) * 9 * sizeof(int) + 32 * sizeof(int) + (stage ? pairing_rows_bytes(NB, NW) : 0);
+}
 
 }  // namespace dbst
