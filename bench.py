@@ -267,13 +267,15 @@ def run_sweep(args, w):
         rows.append({"p": p, "kept_fraction": kept / (g.B * g.H * g.NB * g.NB), "sparse_attn_ms": ms,
                      "kept_tflops": fl / (ms * 1e-3) / 1e12, "frac_of_bf16_peak": fl / (ms * 1e-3) / 1e12 / bf16,
                      "mask_build_ms": mask_ms, "speedup_vs_dense": dense_ms / ms})
+    # dense again at the end: the GPU runs under its power cap, so the first and last points
+    # of a sweep can see different clocks; the crossover uses the slower of the two dense times
+    dense_end_ms = timed(lambda: dbst.dense_attn(qt, kt, vt, g), args.steps)
     dbst.get_error()
-    crossover = None
+    dense_ref = max(dense_ms, dense_end_ms)
     for r in rows:
-        if r["sparse_attn_ms"] >= dense_ms:
-            crossover = r["kept_fraction"]
-            break
-    out = {"sweep": workload_desc(w, float("nan")), "dense_attn_ms": dense_ms,
+        r["speedup_vs_dense"] = dense_ref / r["sparse_attn_ms"]
+    crossover = next((r["kept_fraction"] for r in rows if r["sparse_attn_ms"] >= dense_ref), None)
+    out = {"sweep": workload_desc(w, float("nan")), "dense_attn_ms": dense_ms, "dense_attn_ms_end": dense_end_ms,
            "dense_tflops": dense_flops / (dense_ms * 1e-3) / 1e12, "peak_source": src, "points": rows,
            "dense_crossover_kept_fraction": crossover}
     print(json.dumps(out), flush=True)
