@@ -17,7 +17,9 @@ namespace dbst {
 // ---------------------------------------------------------------------------
 // Block mean-pool: one warp per 64-token block; out[blk][c] = mean (float64).
 // RASTER: q and k are in raster token order and the block's rows are gathered
-// through the tile permutation (the same rows, summed in the same order).
+// through the tile permutation (the same rows, summed in the same order).  A
+// row's raster offset from its tile's first token depends only on the row's
+// place in the tile, so the 64 offsets are tabulated once per CTA.
 // ---------------------------------------------------------------------------
 template <int D, bool RASTER>
 __global__ void __launch_bounds__(256) pool_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
@@ -30,19 +32,24 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint4* __restrict__ q, 
   const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
   const int ch = lane % CPR;
   const int r0 = lane / CPR;
+  __shared__ int row_off[64];             // raster offset of tile row r from the tile's first token
+  if (RASTER) {
+    if (threadIdx.x < 64) row_off[threadIdx.x] = tiled_to_raster(threadIdx.x, tg);   // tile 0 starts at token 0
+    __syncthreads();
+  }
   for (long long w = warp; w < 2 * nblocks; w += nwarps) {
     const bool isk = w >= nblocks;
     const long long b = isk ? w - nblocks : w;
     const uint4* src = (isk ? k : q) + b * 64 * CPR;
-    const uint4* head = (isk ? k : q) + (b / NB) * static_cast<long long>(tg.N) * CPR;
     const int blk = static_cast<int>(b % NB);
+    const uint4* head = (isk ? k : q) +
+                        ((b / NB) * static_cast<long long>(tg.N) + (RASTER ? tiled_to_raster(blk * 64, tg) : 0)) * CPR;
     double acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.0;
 #pragma unroll 8
     for (int r = r0; r < 64; r += RPW) {
-      const uint4 v = RASTER ? ld_stream(head + static_cast<long long>(tiled_to_raster(blk * 64 + r, tg)) * CPR + ch)
-                             : ld_stream(src + r * CPR + ch);
+      const uint4 v = RASTER ? ld_stream(head + row_off[r] * CPR + ch) : ld_stream(src + r * CPR + ch);
       const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
