@@ -187,27 +187,46 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     for (int i = 1; i < 16; ++i) s_misc[i] = 0;
   }
   __syncthreads();
-  for (int side = 0; side < 2; ++side) {
-    if (side == 1 && !has_b) break;
-    const int qblk = side ? qb : qa;
-    int n = NB;
-    const int16_t* gl = nullptr;
-    if (prm.kv_count != nullptr) {
-      n = prm.kv_count[bh * NB + qblk];
-      gl = prm.kv_idx + (bh * NB + qblk) * static_cast<long long>(NB);
-      if (n < 0 || n > NB) {
-        if (tid == 0) record_error(kErrBounds);
-        n = n < 0 ? 0 : NB;
-      }
+  // Work that does not depend on the lists starts at once: the Q tiles' loads and the TMEM
+  // allocation overlap the list reads below.
+  if (warp == 13 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    mbar_expect_tx(bar(PB_Q), 128 * D * 2);
+    for (int h = 0; h < DH; ++h) {
+      load_block(sbase + PairSmem::kQ + h * 16384, &tmQ, bar(PB_Q), qa, h);
+      load_block(sbase + PairSmem::kQ + h * 16384 + 8192, &tmQ, bar(PB_Q), has_b ? qb : qa, h);
     }
-    for (int e = tid; e < n; e += kPairThreads) {
-      const int j = gl ? static_cast<int>(gl[e]) : e;
-      if (j < 0 || j >= NB) {
-        record_error(kErrBounds);
-        continue;
-      }
-      atomicOr(&s_words[side * 128 + (j >> 5)], 1u << (j & 31));
+  }
+  if (warp == 12) {
+    tmem_alloc(sbase + PairSmem::kMisc, 512);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  // Both lists: both counts first, then all entries in one pass (two independent chains of loads).
+  int n0 = NB, n1 = has_b ? NB : 0;
+  const int16_t* g0 = nullptr;
+  const int16_t* g1 = nullptr;
+  if (prm.kv_count != nullptr) {
+    n0 = prm.kv_count[bh * NB + qa];
+    n1 = has_b ? prm.kv_count[bh * NB + qb] : 0;
+    g0 = prm.kv_idx + (bh * NB + qa) * static_cast<long long>(NB);
+    g1 = prm.kv_idx + (bh * NB + (has_b ? qb : qa)) * static_cast<long long>(NB);
+    if (n0 < 0 || n0 > NB || n1 < 0 || n1 > NB) {
+      if (tid == 0) record_error(kErrBounds);
+      n0 = min(max(n0, 0), NB);
+      n1 = min(max(n1, 0), NB);
     }
+  }
+  for (int e = tid; e < n0 + n1; e += kPairThreads) {
+    const int side = e >= n0;
+    const int ei = side ? e - n0 : e;
+    const int16_t* gl = side ? g1 : g0;
+    const int j = gl ? static_cast<int>(gl[ei]) : ei;
+    if (j < 0 || j >= NB) {
+      record_error(kErrBounds);
+      continue;
+    }
+    atomicOr(&s_words[side * 128 + (j >> 5)], 1u << (j & 31));
   }
   __syncthreads();
   if (warp == 0) {   // exclusive scan of the union's popcounts over NW <= 128 words
@@ -244,8 +263,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     }
   }
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_misc[0];
   const int nu = static_cast<int>(s_misc[1]);
   if (nu == 0) {   // neither block keeps anything: o = 0, lse = -inf
+    // the Q loads are in flight and TMEM is held: let the one land and free the other
+    if (warp == 13 && lane == 0) mbar_wait(bar(PB_Q), 0);
+    if (warp == 12) tmem_dealloc(tmem, 512);
     for (int e = tid; e < 64 * D / 8; e += kPairThreads) {
       const int rr = e / (D / 8), c = e % (D / 8);
       reinterpret_cast<uint4*>(prm.o + out_row(qa, rr) * D)[c] = make_uint4(0, 0, 0, 0);
@@ -259,15 +283,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   }
   const int T = (nu + 1) >> 1;
 
-  if (warp == 12) {
-    tmem_alloc(sbase + PairSmem::kMisc, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = s_misc[0];
-
   if (warp == 13 || warp == 14) {
     // ------------------------------------------------------------ TMA producers
     if (lane == 0) {
@@ -278,14 +293,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const int empty0 = isK ? PB_KEMPTY : PB_VEMPTY;
       const uint32_t ring = sbase + (isK ? PairSmem::kK : PairSmem::kV);
       tma_prefetch_desc(map);
-      if (isK) {
-        tma_prefetch_desc(&tmQ);
-        mbar_expect_tx(bar(PB_Q), 128 * D * 2);
-        for (int h = 0; h < DH; ++h) {
-          load_block(sbase + PairSmem::kQ + h * 16384, &tmQ, bar(PB_Q), qa, h);
-          load_block(sbase + PairSmem::kQ + h * 16384 + 8192, &tmQ, bar(PB_Q), has_b ? qb : qa, h);
-        }
-      }
       int armed[kPairKSlots] = {0, 0, 0};
       for (int t = 0; t < T; ++t) {
         if (*s_abort) break;

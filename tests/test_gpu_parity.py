@@ -199,6 +199,34 @@ def test_attention_repeat_launches_bit_identical(built):
     check_attention(o0.float().cpu().numpy().astype(np.float64), l0.cpu().numpy().astype(np.float64), o_ref, lse_ref)
 
 
+@pytest.mark.parametrize("raster", [False, True])
+def test_heads_with_no_kept_blocks(built, raster):
+    """Every pair of query blocks empty in one head (the kernel's early exit), full lists in the other."""
+    w = S.Workload("empty", 9, B=1, H=2, D=128, grid=(4, 16, 32), tile=(1, 8, 8), alpha=0.7, beta=0.3, f_rms=2.0,
+                   kmax=3, p_list=(0.9,), sta_radius=-1)
+    g = P.geometry(w)
+    q, k, v = S.make_qkv(w)
+    mask = np.zeros((1, 2, g.NB, g.NB), bool)
+    mask[0, 1] = True
+    gg = gpu_geom(w)
+    words = torch.from_numpy(P.pack_mask(mask).view(np.int32)).cuda()
+    cnt, idx = dbst.mask_from_bits(words, gg)
+    if raster:
+        o, lse = dbst.block_sparse_attn_raster(*(P.bits_to_torch(a) for a in (q, k, v)), gg, cnt, idx)
+        o = dbst.tile_reorder(o, gg)
+        lse = torch.from_numpy(O.tile_reorder(lse.cpu().numpy()[..., None], g)[..., 0])
+    else:
+        qt, kt, vt = (O.tile_reorder(a, g) for a in (q, k, v))
+        o, lse = dbst.block_sparse_attn(*(P.bits_to_torch(a) for a in (qt, kt, vt)), gg, cnt, idx)
+    dbst.get_error()
+    o = o.float().cpu().numpy()
+    lse = lse.cpu().numpy()
+    assert (o[0, 0] == 0).all() and np.isneginf(lse[0, 0]).all()
+    qt, kt, vt = (O.tile_reorder(a, g) for a in (q, k, v))
+    o_ref, lse_ref = O.masked_attention(qt, kt, vt, mask, 64, 1.0 / math.sqrt(w.D))
+    check_attention(o.astype(np.float64), lse.astype(np.float64), o_ref, lse_ref)
+
+
 def test_constant_v_and_large_logits(built):
     """Constant V is reproduced; logits spanning > 2^16 in log2 units force rescales."""
     w = S.Workload("c", 6, B=1, H=1, D=128, grid=(2, 16, 32), tile=(2, 4, 8), alpha=0.7, beta=0.3, f_rms=6.0,
