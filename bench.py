@@ -347,16 +347,18 @@ def main():
 
     ev = {}
 
-    def step(timed_parts: bool):
+    def step(timed_parts: bool, io=None):
+        """One pass of the path on `stream`; io = (q, k, v, o) device buffers (default: the resident ones)."""
+        q_, k_, v_, o_ = (q, k, v, o) if io is None else io
         if not fused:
-            dbst.tile_reorder(q, g, out=qt)
-            dbst.tile_reorder(k, g, out=kt)
-            dbst.tile_reorder(v, g, out=vt)
+            dbst.tile_reorder(q_, g, out=qt)
+            dbst.tile_reorder(k_, g, out=kt)
+            dbst.tile_reorder(v_, g, out=vt)
         if timed_parts:
             e0 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
         if fused:
-            dbst.build_block_mask_raster(q, k, g, p, w.sta_radius, workspace=ws, out=(bits, cnt, idx))
+            dbst.build_block_mask_raster(q_, k_, g, p, w.sta_radius, workspace=ws, out=(bits, cnt, idx))
             dbst.pair_query_blocks(bits, g, out=pairs)
         else:
             dbst.build_block_mask(qt, kt, g, p, w.sta_radius, workspace=ws, out=(bits, cnt, idx))
@@ -364,7 +366,7 @@ def main():
             e1 = torch.cuda.Event(enable_timing=True)
             e1.record(stream)
         if fused:
-            dbst.block_sparse_attn_raster(q, k, v, g, cnt, idx, 0.0, want_lse=True, out=o, lse=lse, pairs=pairs)
+            dbst.block_sparse_attn_raster(q_, k_, v_, g, cnt, idx, 0.0, want_lse=True, out=o_, lse=lse, pairs=pairs)
         else:
             dbst.block_sparse_attn(qt, kt, vt, g, cnt, idx, 0.0, want_lse=True, out=ot, lse=lse)
         if timed_parts:
@@ -372,7 +374,7 @@ def main():
             e2.record(stream)
             ev.setdefault("parts", []).append((e0, e1, e2))
         if not fused:
-            dbst.tile_unreorder(ot, g, out=o)
+            dbst.tile_unreorder(ot, g, out=o_)
 
     for _ in range(args.warmup):
         step(False)
@@ -401,23 +403,50 @@ def main():
     mask_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev["parts"])
     attn_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev["parts"])
 
-    # end to end: pinned host inputs -> device -> path -> output back to pinned host
-    def e2e_step():
-        for src, dst in zip(host, (q, k, v)):
-            dst.copy_(src, non_blocking=True)
-        step(False)
-        o_host.copy_(o, non_blocking=True)
+    # End to end, as a serving loop runs it: every step copies its inputs in from pinned host
+    # memory and its output back out, and the copies of neighbouring steps overlap this step's
+    # compute (host->device on one stream, device->host on another; PCIe runs both directions at
+    # once).  Inputs and outputs are double-buffered; events order each buffer's reuse.
+    dev_io = [(q, k, v, o), tuple(torch.empty_like(q) for _ in range(4))]
+    host_out = [o_host, torch.empty_like(o_host).pin_memory()]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
 
-    for _ in range(2):
-        e2e_step()
+    def e2e_run(n, start=None, end=None):
+        ev_in, ev_done, ev_out = [None, None], [None, None], [None, None]
+        if start is not None:
+            start.record(s_in)
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(s_in):
+                if ev_done[b] is not None:
+                    s_in.wait_event(ev_done[b])          # step i-2 has finished reading buffer b
+                for src, dst in zip(host, dev_io[b][:3]):
+                    dst.copy_(src, non_blocking=True)
+                ev_in[b] = torch.cuda.Event()
+                ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            if ev_out[b] is not None:
+                stream.wait_event(ev_out[b])             # step i-2's output has left buffer b
+            step(False, dev_io[b])
+            ev_done[b] = torch.cuda.Event()
+            ev_done[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[b])
+                host_out[b].copy_(dev_io[b][3], non_blocking=True)
+                ev_out[b] = torch.cuda.Event()
+                ev_out[b].record(s_out)
+        if end is not None:
+            for e in ev_out:
+                if e is not None:
+                    s_out.wait_event(e)
+            end.record(s_out)
+
+    e2e_run(2)
     torch.cuda.synchronize()
     barrier()
     s2 = torch.cuda.Event(enable_timing=True)
     e2 = torch.cuda.Event(enable_timing=True)
-    s2.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e2.record(stream)
+    e2e_run(args.steps, s2, e2)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = s2.elapsed_time(e2)
@@ -448,6 +477,7 @@ def main():
         "mask_roofline": {"bound": "hbm", "achieved": mask_bytes / (mask_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
                           "frac": mask_bytes / (mask_ms * 1e-3) / 1e9 / hbm},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "ms_per_step": e2e_ms / args.steps,
+                "pipelined": "host->device of step i+1 and device->host of step i-1 overlap step i",
                 "h2d_bytes_per_step": 3 * host[0].numel() * 2, "d2h_bytes_per_step": o_host.numel() * 2},
         "clocks": clk, "gpu_launches": launches_per_step * args.steps,
     }
