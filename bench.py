@@ -409,22 +409,26 @@ def main():
     # once).  Inputs and outputs are double-buffered; events order each buffer's reuse.
     dev_io = [(q, k, v, o), tuple(torch.empty_like(q) for _ in range(4))]
     host_out = [o_host, torch.empty_like(o_host).pin_memory()]
-    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    s_ins = [torch.cuda.Stream() for _ in range(3)]   # q, k, v copied in side by side
+    s_out = torch.cuda.Stream()
 
     def e2e_run(n, start=None, end=None):
-        ev_in, ev_done, ev_out = [None, None], [None, None], [None, None]
+        ev_in, ev_done, ev_out = [[None] * 3, [None] * 3], [None, None], [None, None]
         if start is not None:
-            start.record(s_in)
+            start.record(s_ins[0])
+            for s_ in s_ins[1:]:
+                s_.wait_event(start)
         for i in range(n):
             b = i % 2
-            with torch.cuda.stream(s_in):
-                if ev_done[b] is not None:
-                    s_in.wait_event(ev_done[b])          # step i-2 has finished reading buffer b
-                for src, dst in zip(host, dev_io[b][:3]):
+            for t_, (s_, src, dst) in enumerate(zip(s_ins, host, dev_io[b][:3])):
+                with torch.cuda.stream(s_):
+                    if ev_done[b] is not None:
+                        s_.wait_event(ev_done[b])        # step i-2 has finished reading buffer b
                     dst.copy_(src, non_blocking=True)
-                ev_in[b] = torch.cuda.Event()
-                ev_in[b].record(s_in)
-            stream.wait_event(ev_in[b])
+                    ev_in[b][t_] = torch.cuda.Event()
+                    ev_in[b][t_].record(s_)
+            for e in ev_in[b]:
+                stream.wait_event(e)
             if ev_out[b] is not None:
                 stream.wait_event(ev_out[b])             # step i-2's output has left buffer b
             step(False, dev_io[b])
@@ -477,7 +481,7 @@ def main():
         "mask_roofline": {"bound": "hbm", "achieved": mask_bytes / (mask_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
                           "frac": mask_bytes / (mask_ms * 1e-3) / 1e9 / hbm},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "ms_per_step": e2e_ms / args.steps,
-                "pipelined": "host->device of step i+1 and device->host of step i-1 overlap step i",
+                "pipelined": "host->device of step i+1 (q, k, v on three streams) and device->host of step i-1 overlap step i",
                 "h2d_bytes_per_step": 3 * host[0].numel() * 2, "d2h_bytes_per_step": o_host.numel() * 2},
         "clocks": clk, "gpu_launches": launches_per_step * args.steps,
     }
