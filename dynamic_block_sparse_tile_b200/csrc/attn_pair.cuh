@@ -3,8 +3,9 @@
 // pairs only).
 //
 // Formulation ("query pairs").  One CTA owns two 64-token query blocks qa, qb
-// (neighbours one tile step apart) as one 128-row query tile, and walks the
-// union of their kept key blocks two at a time:
+// (the pair the caller's pair list names, else neighbours one tile step apart)
+// as one 128-row query tile, and walks the union of their kept key blocks two
+// at a time:
 //     S[128 queries x 128 keys] = Q[128 x D] . K_tile[128 x D]^T      (tcgen05 SS, M=128, N=128)
 //     O[128 queries x D]       += P[128 x 128 keys] . V_tile[128 x D]  (tcgen05 TS: P read from TMEM)
 // A key block kept by only one of the two query blocks is masked (P = 0) in
@@ -46,8 +47,8 @@ constexpr float kPairRescale = 16.0f;
 struct PairParams {
   const int32_t* kv_count;   // [BH*NB]; null => dense (every list is 0..NB-1)
   const int16_t* kv_idx;     // [BH*NB*NB]
-  __nv_bfloat16* o;          // tiled [BH, N, D]
-  float* lse;                // [BH, N] or null
+  __nv_bfloat16* o;          // [BH, N, D], tile or raster order (RASTER)
+  float* lse;                // [BH, N] in the same order, or null
   int NB, N;
   const int32_t* pairs;      // [BH][pairs_per_head] qa | qb << 16 (qb 0xFFFF: none), or null
   int pair_stride;           // without a pair list: qb = qa + pair_stride
