@@ -51,13 +51,24 @@ def peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def attn_source_digest() -> str:
+def source_digest(texts) -> str:
+    """sha256 (first 16 hex digits) of C++ sources with // comments and blank space removed, so a
+    measurement stays attached to its code across edits that touch only comments."""
     import hashlib
+    import re
     h = hashlib.sha256()
-    for f in ("attn_pair.cuh", "ptx.cuh"):
-        with open(os.path.join(ROOT, "dynamic_block_sparse_tile_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+    for text in texts:
+        code = "\n".join(" ".join(re.sub(r"//.*", "", line).split()) for line in text.splitlines())
+        h.update(re.sub(r"\n+", "\n", code).strip().encode())
     return h.hexdigest()[:16]
+
+
+def attn_source_digest() -> str:
+    texts = []
+    for f in ("attn_pair.cuh", "ptx.cuh"):
+        with open(os.path.join(ROOT, "dynamic_block_sparse_tile_b200", "csrc", f)) as fh:
+            texts.append(fh.read())
+    return source_digest(texts)
 
 
 def measured_traffic(workload: str, p: float, layout: str):

@@ -86,6 +86,40 @@ def test_wan_like_full_size(built):
     assert 0.05 < kept < 0.15
 
 
+def test_wan_like_full_size_bench_path(built):
+    """The benchmarked configuration: raster q, k, v in, the pair list, raster o and lse out."""
+    w = S.workload("wan")
+    og = P.geometry(w)
+    q, k, v = S.make_qkv(w)
+    g = dbst.Geom.make(w.B, w.H, w.D, w.grid, w.tile)
+    qd, kd, vd = (P.bits_to_torch(a) for a in (q, k, v))
+    bits, cnt, idx = dbst.build_block_mask_raster(qd, kd, g, 0.9, w.sta_radius)
+    pairs = dbst.pair_query_blocks(bits, g)
+    o, lse = dbst.block_sparse_attn_raster(qd, kd, vd, g, cnt, idx, pairs=pairs)
+    dbst.get_error()
+    qt, kt, vt = (O.tile_reorder(a, og) for a in (q, k, v))
+    ref, A = P.oracle_mask_per_head(qt, kt, og, 0.9, w.sta_radius)
+    got = P.unpack_mask(bits.cpu().numpy().view(np.uint32), og.NB)
+    hard, _ = P.mask_mismatches(got, ref, A, 0.9, O.sta_mask(og, w.sta_radius))
+    assert not hard, f"{len(hard)} non-excused mask disagreements, first {hard[:5]}"
+    assert P.lists_match_bits(cnt.cpu().numpy(), idx.cpu().numpy(), got)
+    e = pairs.cpu().numpy().astype(np.int64)
+    qa, qb = e & 0xFFFF, (e >> 16) & 0xFFFF
+    for h in range(og.H):
+        seen = np.bincount(np.concatenate([qa[0, h], qb[0, h][qb[0, h] != 0xFFFF]]), minlength=og.NB)
+        assert (seen == 1).all()
+    # sampled query blocks, compared in raster order
+    scale = 1.0 / math.sqrt(w.D)
+    rows = P.sample_rows(w.B, w.H, og.NB, 24, seed=17)
+    o_ref_t, lse_ref_t = O.masked_attention(qt, kt, vt, got, 64, scale, rows=rows)
+    o_t = dbst.tile_reorder(o, g)                       # back to tile order to pick the sampled blocks
+    lse_t = O.tile_reorder(lse.cpu().numpy()[..., None], og)[..., 0]
+    max_abs, rel = P.attn_errors(P.gpu_rows(o_t, rows), o_ref_t)
+    assert max_abs <= P.ATTN_MAX_ABS and rel <= P.ATTN_REL_L2, (max_abs, rel)
+    lse_gpu = np.stack([lse_t[b, h, i * 64:(i + 1) * 64] for (b, h, i) in rows]).astype(np.float64)
+    assert np.max(np.abs(lse_gpu - lse_ref_t)) <= P.LSE_MAX_ABS
+
+
 def test_hunyuan_like_full_size(built):
     kept, excused = check_full("hunyuan", 0.9, n_rows=16)
     assert 0.03 < kept < 0.15
