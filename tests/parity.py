@@ -113,6 +113,17 @@ def sample_rows(B: int, H: int, NB: int, count: int, seed: int) -> List[Tuple[in
     return sorted(rows)
 
 
+def sample_rows_per_head(B: int, H: int, NB: int, per_head: int, seed: int) -> List[Tuple[int, int, int]]:
+    """`per_head` distinct seeded query blocks in every (b, h), plus the first and the last block."""
+    rng = np.random.default_rng(seed)
+    rows = {(0, 0, 0), (B - 1, H - 1, NB - 1)}
+    for b in range(B):
+        for h in range(H):
+            for i in rng.choice(NB, size=min(per_head, NB), replace=False):
+                rows.add((b, h, int(i)))
+    return sorted(rows)
+
+
 def gpu_rows(t: torch.Tensor, rows: Sequence[Tuple[int, int, int]], blk: int = 64) -> np.ndarray:
     """Gather [len(rows), blk, ...] query blocks of a [B, H, N, ...] GPU tensor as float64."""
     out = [t[b, h, i * blk:(i + 1) * blk].float().cpu().numpy() for (b, h, i) in rows]

@@ -1,11 +1,11 @@
 """Full-size parity on the Wan-like, HunyuanVideo-like and sweep workloads.
 
-Same call sequence as bench.py (reorder -> mask -> attention -> unreorder).
-The mask is compared with the oracle on every row of every head, with the
-near-threshold exemption.  Attention is compared on a seeded sample of
-query blocks that includes the first and the last one, against the oracle
-given the oracle's mask (and, for the mask the GPU built, against the oracle
-given that mask).
+Same call sequence as bench.py's explicit path (reorder -> mask -> attention
+-> unreorder), and the bench's default path in its own test.  The mask is
+compared with the oracle on every row of every head, with the near-threshold
+exemption.  Attention is compared on seeded query blocks in every head (plus
+the first and the last block), against the oracle given the mask the GPU built
+and given the oracle's own mask.
 """
 import dataclasses
 import math
@@ -42,7 +42,7 @@ def run_path(w, p, sta, q, k, v):
     return g, (qt, kt, vt), bits, cnt, idx, ot, lse, o
 
 
-def check_full(name, p, n_rows=24):
+def check_full(name, p, per_head=8):
     w = S.workload(name)
     og = P.geometry(w)
     q, k, v = S.make_qkv(w)
@@ -60,7 +60,7 @@ def check_full(name, p, n_rows=24):
     assert np.array_equal(cnt_h, got.sum(-1))
     # attention on sampled query blocks, with the GPU's own lists (== oracle mask up to exemptions)
     scale = 1.0 / math.sqrt(w.D)
-    rows = P.sample_rows(w.B, w.H, og.NB, n_rows, seed=7 + w.index)
+    rows = P.sample_rows_per_head(w.B, w.H, og.NB, per_head, seed=7 + w.index)
     for (b, h, i) in rows:
         js = idx_h[b, h, i, :cnt_h[b, h, i]]
         assert np.array_equal(js, np.nonzero(got[b, h, i])[0])
@@ -82,7 +82,7 @@ def check_full(name, p, n_rows=24):
 
 
 def test_wan_like_full_size(built):
-    kept, excused = check_full("wan", 0.9)
+    kept, excused = check_full("wan", 0.9, per_head=16)
     assert 0.05 < kept < 0.15
 
 
@@ -110,7 +110,7 @@ def test_wan_like_full_size_bench_path(built):
         assert (seen == 1).all()
     # sampled query blocks, compared in raster order
     scale = 1.0 / math.sqrt(w.D)
-    rows = P.sample_rows(w.B, w.H, og.NB, 24, seed=17)
+    rows = P.sample_rows_per_head(w.B, w.H, og.NB, 16, seed=17)
     o_ref_t, lse_ref_t = O.masked_attention(qt, kt, vt, got, 64, scale, rows=rows)
     o_t = dbst.tile_reorder(o, g)                       # back to tile order to pick the sampled blocks
     lse_t = O.tile_reorder(lse.cpu().numpy()[..., None], og)[..., 0]
@@ -121,13 +121,13 @@ def test_wan_like_full_size_bench_path(built):
 
 
 def test_hunyuan_like_full_size(built):
-    kept, excused = check_full("hunyuan", 0.9, n_rows=16)
+    kept, excused = check_full("hunyuan", 0.9, per_head=64)
     assert 0.03 < kept < 0.15
 
 
 @pytest.mark.parametrize("p", [0.5, 0.9, 1.0])
 def test_sweep_full_size(built, p):
-    kept, excused = check_full("sweep", p, n_rows=16)
+    kept, excused = check_full("sweep", p, per_head=8)
     if p >= 1.0:
         assert kept == 1.0
 
