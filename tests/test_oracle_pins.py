@@ -323,3 +323,31 @@ def test_end_to_end_p1_is_dense_attention():
     ref = torch.nn.functional.scaled_dot_product_attention(
         *(torch.from_numpy(a) for a in (q, k, v)), scale=0.25).numpy()
     np.testing.assert_allclose(O.tile_unreorder(o, g), ref, rtol=1e-11, atol=1e-12)
+
+
+def test_cdf_select_batched_rows():
+    """The batched selection keeps, per row, what the row selection keeps; p = 1 keeps every
+    block; a one-hot row keeps exactly its hot block at any p."""
+    A = RNG.random((2, 3, 5, 5))
+    A /= A.sum(-1, keepdims=True)
+    for p in (0.3, 0.9):
+        got = O.cdf_select(A, p)
+        assert got.shape == A.shape
+        for idx in itertools.product(range(2), range(3), range(5)):
+            np.testing.assert_array_equal(got[idx], O.cdf_select_row(A[idx], p))
+    assert O.cdf_select(A, 1.0).all()
+    hot = np.zeros((4, 4))
+    hot[np.arange(4), [2, 0, 3, 1]] = 1.0
+    for p in (0.01, 0.5, 0.999):
+        sel = O.cdf_select(hot, p)
+        np.testing.assert_array_equal(sel, hot > 0)
+
+
+def test_kept_pair_flops_full_lists_equal_dense_flops():
+    """Every list full: 4 * D * N^2 * B * H, the dense attention FLOP count."""
+    B, H, D, NB = 2, 3, 128, 7
+    kv_count = np.full((B, H, NB), NB, dtype=np.int32)
+    N = NB * 64
+    assert O.kept_pair_flops(kv_count, D) == 4.0 * D * N * N * B * H
+    kv_count[0, 0, 0] = 0
+    assert O.kept_pair_flops(kv_count, D) == 4.0 * D * N * N * B * H - 4.0 * D * NB * 64 * 64
