@@ -35,6 +35,7 @@ from .nabla import (  # noqa: F401
     build_block_mask,
     mask_to_lists,
     masked_attention,
+    masked_attention_backward,
     dense_attention,
     kept_pair_flops,
 )

@@ -33,6 +33,11 @@ R7  Token reorder ("Fractal Flattening") generalised from P x P spatial
     tokens inside a tile in raster order.  The time order of tiles is kept.
 R8  Blocks are the 64-token tiles: the pooling block of N tokens is one
     tile, so query block i and key block j both mean tile i / tile j.
+R9  Backward (the page claims faster training but prints no backward): the
+    exact gradient of the forward definition of :func:`masked_attention`
+    with respect to q, k and v, for an upstream gradient do of o.  A key
+    token receives gradient only from the query blocks that keep its block;
+    a query block with no kept key block receives none.
 """
 from __future__ import annotations
 
@@ -259,6 +264,46 @@ def masked_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, mask: np.ndarr
     if full:
         return o_out.reshape(B, H, N, D), lse_out.reshape(B, H, N)
     return o_out, lse_out
+
+
+def masked_attention_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, mask: np.ndarray, blk: int,
+                              scale: float, do: np.ndarray):
+    """Gradients (dq, dk, dv) of :func:`masked_attention` for upstream gradient ``do`` (reading R9).
+
+    Per query block i with kept key tokens S_i, with P the row softmax of
+    s = scale * q_i k_S^T and o_i = P v_S (the softmax calculus, step by step):
+        dv_S += P^T do_i,  dP = do_i v_S^T,  delta = rowsum(do_i * o_i),
+        ds = P * (dP - delta),  dq_i = scale * ds k_S,  dk_S += scale * ds^T q_i.
+    All inputs ``[B, H, N, D]`` tile-ordered (bf16 bits or floats); float64 out.
+    """
+    dec = bf16_bits_to_f64 if q.dtype == np.uint16 else (lambda a: np.asarray(a, dtype=np.float64))
+    B, H, N, D = q.shape
+    NB = N // blk
+    do = np.asarray(do, dtype=np.float64)
+    dq = np.zeros((B, H, N, D))
+    dk = np.zeros((B, H, N, D))
+    dv = np.zeros((B, H, N, D))
+    for b in range(B):
+        for h in range(H):
+            kh, vh = dec(k[b, h]), dec(v[b, h])
+            for i in range(NB):
+                kept = np.nonzero(mask[b, h, i])[0]
+                if kept.size == 0:
+                    continue
+                tok = (kept[:, None] * blk + np.arange(blk)[None, :]).reshape(-1)
+                rows = slice(i * blk, (i + 1) * blk)
+                qi, ks, vs, doi = dec(q[b, h, rows]), kh[tok], vh[tok], do[b, h, rows]
+                s = (qi @ ks.T) * scale
+                e = np.exp(s - s.max(axis=1, keepdims=True))
+                P = e / e.sum(axis=1, keepdims=True)
+                oi = P @ vs
+                dv[b, h, tok] += P.T @ doi
+                dP = doi @ vs.T
+                delta = np.sum(doi * oi, axis=1, keepdims=True)
+                ds = P * (dP - delta)
+                dq[b, h, rows] = scale * (ds @ ks)
+                dk[b, h, tok] += scale * (ds.T @ qi)
+    return dq, dk, dv
 
 
 def dense_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float):

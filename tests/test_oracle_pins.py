@@ -351,3 +351,107 @@ def test_kept_pair_flops_full_lists_equal_dense_flops():
     assert O.kept_pair_flops(kv_count, D) == 4.0 * D * N * N * B * H
     kv_count[0, 0, 0] = 0
     assert O.kept_pair_flops(kv_count, D) == 4.0 * D * N * N * B * H - 4.0 * D * NB * 64 * 64
+
+
+# --------------------------------------------------------------------------
+# Backward of the block-sparse attention (gradient of the forward definition)
+# --------------------------------------------------------------------------
+
+def _loss(q, k, v, mask, blk, scale, do):
+    o, _ = O.masked_attention(q, k, v, mask, blk, scale)
+    return float(np.sum(o * do))
+
+
+def test_backward_matches_central_finite_differences():
+    """d/dx of sum(o * do) by central differences, every element of q, k and v."""
+    B, H, NB, blk, D, scale = 1, 2, 3, 2, 3, 0.7
+    q, k, v, do = (RNG.standard_normal((B, H, NB * blk, D)) for _ in range(4))
+    mask = np.array([[[[1, 0, 1], [0, 0, 0], [1, 1, 1]],
+                      [[0, 1, 0], [1, 1, 0], [0, 0, 1]]]], dtype=bool)
+    grads = O.masked_attention_backward(q, k, v, mask, blk, scale, do)
+    h = 1e-6
+    for which, g in enumerate(grads):
+        args = [q, k, v]
+        for idx in np.ndindex(q.shape):
+            plus = [a.copy() for a in args]
+            minus = [a.copy() for a in args]
+            plus[which][idx] += h
+            minus[which][idx] -= h
+            fd = (_loss(*plus, mask, blk, scale, do) - _loss(*minus, mask, blk, scale, do)) / (2 * h)
+            assert abs(fd - g[idx]) < 1e-7 * (1 + abs(fd)), (which, idx, fd, g[idx])
+
+
+def _torch_grads(q, k, v, tok, scale, do):
+    t = [torch.from_numpy(a.copy()).requires_grad_(True) for a in (q, k, v)]
+    o = torch.nn.functional.scaled_dot_product_attention(
+        *t, attn_mask=None if tok is None else torch.from_numpy(tok), scale=scale)
+    o.backward(torch.from_numpy(do))
+    return [x.grad.numpy() for x in t]
+
+
+def test_backward_full_mask_equals_dense_autograd():
+    B, H, NB, blk, D = 1, 2, 3, 64, 16
+    q, k, v, do = (RNG.standard_normal((B, H, NB * blk, D)) for _ in range(4))
+    got = O.masked_attention_backward(q, k, v, np.ones((B, H, NB, NB), bool), blk, 0.25, do)
+    for g, r in zip(got, _torch_grads(q, k, v, None, 0.25, do)):
+        np.testing.assert_allclose(g, r, rtol=1e-10, atol=1e-12)
+
+
+def test_backward_sparse_mask_equals_autograd_with_expanded_mask():
+    B, H, NB, blk, D = 1, 2, 4, 64, 8
+    q, k, v, do = (RNG.standard_normal((B, H, NB * blk, D)) for _ in range(4))
+    mask = RNG.random((B, H, NB, NB)) < 0.4
+    mask[..., np.arange(NB), np.arange(NB)] = True            # no empty row (sdpa would give NaN)
+    tok = np.repeat(np.repeat(mask, blk, axis=2), blk, axis=3)
+    got = O.masked_attention_backward(q, k, v, mask, blk, 0.3, do)
+    for g, r in zip(got, _torch_grads(q, k, v, tok, 0.3, do)):
+        np.testing.assert_allclose(g, r, rtol=1e-10, atol=1e-12)
+
+
+def test_backward_empty_row_has_no_gradient_and_gives_none():
+    """A query block with no kept key block: zero dq, and its do moves no dk / dv."""
+    B, H, NB, blk, D = 1, 1, 3, 4, 5
+    q, k, v, do = (RNG.standard_normal((B, H, NB * blk, D)) for _ in range(4))
+    mask = np.ones((B, H, NB, NB), bool)
+    mask[0, 0, 1] = False
+    dq, dk, dv = O.masked_attention_backward(q, k, v, mask, blk, 0.5, do)
+    assert (dq[0, 0, blk:2 * blk] == 0).all()
+    do2 = do.copy()
+    do2[0, 0, blk:2 * blk] = RNG.standard_normal((blk, D)) * 10
+    dq2, dk2, dv2 = O.masked_attention_backward(q, k, v, mask, blk, 0.5, do2)
+    np.testing.assert_array_equal(dk, dk2)
+    np.testing.assert_array_equal(dv, dv2)
+    np.testing.assert_array_equal(dq, dq2)
+
+
+def test_backward_single_kept_key_closed_form():
+    """One key per block and one kept block per row: softmax is 1, so dq = 0, dk = 0 and
+    the kept key's dv is the sum of do over the rows that keep it."""
+    B, H, NB, blk, D = 1, 1, 5, 1, 4
+    q, k, v, do = (RNG.standard_normal((B, H, NB, D)) for _ in range(4))
+    pick = np.array([3, 0, 3, 4, 3])
+    mask = np.zeros((B, H, NB, NB), bool)
+    mask[0, 0, np.arange(NB), pick] = True
+    dq, dk, dv = O.masked_attention_backward(q, k, v, mask, blk, 0.9, do)
+    assert np.abs(dq).max() < 1e-15 and np.abs(dk).max() < 1e-15
+    ref = np.zeros((NB, D))
+    np.add.at(ref, pick, do[0, 0])
+    np.testing.assert_allclose(dv[0, 0], ref, rtol=1e-15, atol=1e-15)
+
+
+def test_backward_is_linear_in_do_and_reads_bf16_bits():
+    B, H, NB, blk, D = 1, 1, 3, 8, 4
+    q, k, v = (torch.randn(B, H, NB * blk, D, dtype=torch.bfloat16,
+                           generator=torch.Generator().manual_seed(s)) for s in (1, 2, 3))
+    bits = [a.view(torch.int16).numpy().view(np.uint16) for a in (q, k, v)]
+    f = [a.double().numpy() for a in (q, k, v)]
+    mask = RNG.random((B, H, NB, NB)) < 0.6
+    mask[..., 0] = True
+    d1, d2 = RNG.standard_normal((2, B, H, NB * blk, D))
+    g1 = O.masked_attention_backward(*bits, mask, blk, 0.5, d1)
+    g2 = O.masked_attention_backward(*bits, mask, blk, 0.5, d2)
+    g12 = O.masked_attention_backward(*bits, mask, blk, 0.5, 2 * d1 - 3 * d2)
+    gf = O.masked_attention_backward(*f, mask, blk, 0.5, d1)
+    for a, b, c, e in zip(g1, g2, g12, gf):
+        np.testing.assert_allclose(c, 2 * a - 3 * b, rtol=1e-12, atol=1e-12)
+        np.testing.assert_array_equal(a, e)
