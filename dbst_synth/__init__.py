@@ -16,6 +16,8 @@ Recipe (per workload, per (batch, head) pair):
 * ``q = alpha * f + beta * eps_q``, ``k = alpha * f + beta * eps_k`` (the same
   ``f`` for both: the "Q=K basis"), ``v = eps_v``, with ``eps ~ N(0, 1)``.
 * Values are rounded to bf16 with round-to-nearest-even on the host.
+* The upstream gradient of the backward (``make_grad``) is ``N(0, 1)`` from
+  ``default_rng([seed, b, h, 1])``, rounded the same way.
 
 Tokens are laid out in raster order ``n = (t*Y + y)*X + x``, tensors are
 ``[B, H, N, D]`` contiguous.  The mixing weights ``alpha``/``beta`` follow the
@@ -179,3 +181,16 @@ def make_qkv(w: Workload, heads: Optional[range] = None, batches: Optional[range
             k[bi, hi] = bf16_bits_from_f32(a * f + be * ek)
             v[bi, hi] = bf16_bits_from_f32(ev)
     return q, k, v
+
+
+def make_grad(w: Workload, heads: Optional[range] = None, batches: Optional[range] = None) -> np.ndarray:
+    """Seeded upstream gradient dO as bf16 bit patterns, raster order ``[B', H', N, D]``;
+    per (b, h) it depends only on (seed, b, h), like :func:`make_qkv`."""
+    heads = range(w.H) if heads is None else heads
+    batches = range(w.B) if batches is None else batches
+    out = np.empty((len(batches), len(heads), w.N, w.D), np.uint16)
+    for bi, b in enumerate(batches):
+        for hi, h in enumerate(heads):
+            rng = np.random.default_rng([w.seed, b, h, 1])
+            out[bi, hi] = bf16_bits_from_f32(rng.standard_normal((w.N, w.D), dtype=np.float32))
+    return out

@@ -20,6 +20,7 @@ import torch
 __all__ = ["Geom", "DbstError", "lib_path", "load", "tile_reorder", "tile_unreorder", "mask_workspace_bytes",
            "build_block_mask", "build_block_mask_noalloc", "mask_from_bits", "block_sparse_attn", "dense_attn",
            "build_block_mask_raster", "block_sparse_attn_raster", "dense_attn_raster", "pair_query_blocks",
+           "transpose_block_mask", "attn_backward_workspace_bytes", "block_sparse_attn_backward",
            "get_error", "EXPORTS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -29,7 +30,9 @@ _LIB_PATH = os.path.join(_HERE, "libdbst.so")
 EXPORTS = ("dbst_status_string", "dbst_tile_reorder", "dbst_tile_unreorder", "dbst_mask_workspace_bytes",
            "dbst_build_block_mask", "dbst_mask_from_bits", "dbst_block_sparse_attn", "dbst_dense_attn",
            "dbst_get_error", "dbst_build_block_mask_noalloc", "dbst_build_block_mask_raster",
-           "dbst_block_sparse_attn_raster", "dbst_dense_attn_raster", "dbst_pair_query_blocks")
+           "dbst_block_sparse_attn_raster", "dbst_dense_attn_raster", "dbst_pair_query_blocks",
+           "dbst_transpose_block_mask", "dbst_attn_backward_workspace_bytes", "dbst_block_sparse_attn_backward",
+           "dbst_block_sparse_attn_backward_raster")
 
 DBST_OK, DBST_EINVAL, DBST_ECUDA, DBST_ETIMEOUT, DBST_EBOUNDS, DBST_ETOOLARGE = 0, 1, 2, 3, 4, 5
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -97,6 +100,12 @@ def load() -> ctypes.CDLL:
     lib.dbst_get_error.argtypes, lib.dbst_get_error.restype = [vp], i32
     lib.dbst_build_block_mask_noalloc.argtypes = [vp, vp, gp, f32, i32, vp, vp, vp, vp]
     lib.dbst_build_block_mask_noalloc.restype = i32
+    lib.dbst_transpose_block_mask.argtypes, lib.dbst_transpose_block_mask.restype = [vp, gp, vp, vp, vp, vp], i32
+    lib.dbst_attn_backward_workspace_bytes.argtypes = [gp]
+    lib.dbst_attn_backward_workspace_bytes.restype = ctypes.c_size_t
+    for name in ("dbst_block_sparse_attn_backward", "dbst_block_sparse_attn_backward_raster"):
+        getattr(lib, name).argtypes = [vp, vp, vp, vp, vp, gp, vp, vp, vp, vp, f32, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        getattr(lib, name).restype = i32
     _lib = lib
     return lib
 
@@ -283,6 +292,54 @@ def _dense_attn(fn: str, q, k, v, g: Geom, scale, want_lse):
     _check(getattr(load(), fn)(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(g), float(scale), _ptr(o), _ptr(lse),
                                _stream()), fn)
     return o, lse
+
+
+def transpose_block_mask(mask_bits: torch.Tensor, g: Geom, out=None):
+    """Transposed block mask and its lists (``dbst_transpose_block_mask``) -> (mask_bits_t, q_count, q_idx).
+
+    Row j of the result lists the query blocks whose kept set contains key block j.
+    """
+    _need(mask_bits, torch.int32, (g.B, g.H, g.NB, g.NW), "mask_bits")
+    dev = mask_bits.device
+    if out is None:
+        bits_t = torch.empty_like(mask_bits)
+        cnt = torch.empty((g.B, g.H, g.NB), dtype=torch.int32, device=dev)
+        idx = torch.empty((g.B, g.H, g.NB, g.NB), dtype=torch.int16, device=dev)
+    else:
+        bits_t, cnt, idx = out
+    _check(load().dbst_transpose_block_mask(_ptr(mask_bits), ctypes.byref(g), _ptr(bits_t), _ptr(cnt), _ptr(idx),
+                                            _stream()), "dbst_transpose_block_mask")
+    return bits_t, cnt, idx
+
+
+def attn_backward_workspace_bytes(g: Geom) -> int:
+    return int(load().dbst_attn_backward_workspace_bytes(ctypes.byref(g)))
+
+
+def block_sparse_attn_backward(q, k, v, lse, d_o, g: Geom, kv_count, kv_idx, q_count, q_idx, scale: float = 0.0,
+                               raster: bool = False, workspace: Optional[torch.Tensor] = None, out=None):
+    """Gradients of the block-sparse attention (``dbst_block_sparse_attn_backward[_raster]``) -> (dq, dk, dv).
+
+    ``lse`` is the forward's log-sum-exp for the same lists; (q_count, q_idx)
+    come from :func:`transpose_block_mask` of the forward's mask.
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (d_o, "d_o")):
+        _need(t, torch.bfloat16, _qkv_shape(g), n)
+    _need(lse, torch.float32, (g.B, g.H, g.N), "lse")
+    for c, i, n in ((kv_count, kv_idx, "kv"), (q_count, q_idx, "q")):
+        _need(c, torch.int32, (g.B, g.H, g.NB), f"{n}_count")
+        _need(i, torch.int16, (g.B, g.H, g.NB, g.NB), f"{n}_idx")
+    if out is None:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    else:
+        dq, dk, dv = out
+    if workspace is None:
+        workspace = torch.empty(attn_backward_workspace_bytes(g), dtype=torch.uint8, device=q.device)
+    fn = "dbst_block_sparse_attn_backward_raster" if raster else "dbst_block_sparse_attn_backward"
+    _check(getattr(load(), fn)(_ptr(q), _ptr(k), _ptr(v), _ptr(lse), _ptr(d_o), ctypes.byref(g), _ptr(kv_count),
+                               _ptr(kv_idx), _ptr(q_count), _ptr(q_idx), float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
+                               _ptr(workspace), workspace.numel() * workspace.element_size(), _stream()), fn)
+    return dq, dk, dv
 
 
 def get_error() -> None:

@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "../../include/dbst.h"
+#include "attn_bwd.cuh"
 #include "attn_pair.cuh"
 #include "pairing.cuh"
 #include "mask.cuh"
@@ -216,6 +217,86 @@ dbst_status attn_common(const void* q, const void* k, const void* v, const dbst_
                      : launch_pair<64, false>(q, k, v, g, cnt, idx, pairs, scale, o, lse, s);
 }
 
+size_t bwd_workspace(const dbst_geom* g) { return align_up(static_cast<size_t>(bh_count(g) * tokens(g)) * 8u); }
+
+// Backward: the dq pass over the forward's lists (it also writes each query row's (lse * log2 e,
+// delta) to `stats`), then the dk/dv pass over the transposed lists.  Own blocks are paired like
+// the forward's query blocks.
+template <int D, bool RASTER>
+dbst_status launch_bwd(const void* q, const void* k, const void* v, const float* lse, const void* dout,
+                       const dbst_geom* g, const int32_t* kv_count, const int16_t* kv_idx, const int32_t* q_count,
+                       const int16_t* q_idx, float scale, void* dq, void* dk, void* dv, float2* stats,
+                       cudaStream_t s) {
+  const long long rows = bh_count(g) * tokens(g);
+  CUtensorMap tq, tk, tv, tdo;
+  if (RASTER) {
+    if (!make_tmap_raster(&tq, q, g) || !make_tmap_raster(&tk, k, g) || !make_tmap_raster(&tv, v, g) ||
+        !make_tmap_raster(&tdo, dout, g))
+      return DBST_ECUDA;
+  } else {
+    if (!make_tmap(&tq, q, rows, D) || !make_tmap(&tk, k, rows, D) || !make_tmap(&tv, v, rows, D) ||
+        !make_tmap(&tdo, dout, rows, D))
+      return DBST_ECUDA;
+  }
+  dbst::BwdParams p;
+  p.tg = tile_geo(g);
+  p.lse = lse;
+  p.stats = stats;
+  p.NB = nblocks(g);
+  p.N = static_cast<int>(tokens(g));
+  p.pair_stride = pair_stride(g);
+  p.pairs_per_head = ((p.NB + 2 * p.pair_stride - 1) / (2 * p.pair_stride)) * p.pair_stride;
+  const float sc = scale > 0.0f ? scale : 1.0f / std::sqrt(static_cast<float>(D));
+  p.scale = sc;
+  p.scale_log2 = sc * 1.4426950408889634f;
+  const int smem = dbst::BwdSmem::kBytes + 1024;
+  static std::once_flag once;
+  static cudaError_t attr = cudaSuccess;
+  std::call_once(once, [&] {
+    attr = cudaFuncSetAttribute(dbst::bwd_kernel<D, RASTER, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (attr == cudaSuccess)
+      attr = cudaFuncSetAttribute(dbst::bwd_kernel<D, RASTER, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  if (attr != cudaSuccess) return DBST_ECUDA;
+  const long long grid = bh_count(g) * p.pairs_per_head;
+  if (grid >= (1ll << 31)) return DBST_EINVAL;
+  p.count = kv_count;
+  p.idx = kv_idx;
+  p.out0 = static_cast<__nv_bfloat16*>(dq);
+  p.out1 = nullptr;
+  dbst::bwd_kernel<D, RASTER, false><<<static_cast<unsigned>(grid), dbst::kBwdThreads, smem, s>>>(tq, tdo, tk, tv, p);
+  if (cudaGetLastError() != cudaSuccess) return DBST_ECUDA;
+  p.count = q_count;
+  p.idx = q_idx;
+  p.out0 = static_cast<__nv_bfloat16*>(dv);
+  p.out1 = static_cast<__nv_bfloat16*>(dk);
+  dbst::bwd_kernel<D, RASTER, true><<<static_cast<unsigned>(grid), dbst::kBwdThreads, smem, s>>>(tk, tv, tq, tdo, p);
+  return launch_status();
+}
+
+dbst_status bwd_common(const void* q, const void* k, const void* v, const float* lse, const void* dout,
+                       const dbst_geom* g, const int32_t* kv_count, const int16_t* kv_idx, const int32_t* q_count,
+                       const int16_t* q_idx, float scale, void* dq, void* dk, void* dv, void* workspace,
+                       size_t workspace_bytes, void* stream, bool raster) {
+  if (!geom_ok(g) || !q || !k || !v || !lse || !dout || !dq || !dk || !dv || !workspace) return DBST_EINVAL;
+  if (!kv_count || !kv_idx || !q_count || !q_idx) return DBST_EINVAL;
+  for (const void* ptr : {q, k, v, dout, static_cast<const void*>(dq), static_cast<const void*>(dk),
+                          static_cast<const void*>(dv), static_cast<const void*>(workspace),
+                          static_cast<const void*>(kv_count), static_cast<const void*>(kv_idx),
+                          static_cast<const void*>(q_count), static_cast<const void*>(q_idx)})
+    if (!aligned16(ptr)) return DBST_EINVAL;
+  if (reinterpret_cast<uintptr_t>(lse) & 3u) return DBST_EINVAL;
+  if (!std::isfinite(scale)) return DBST_EINVAL;
+  if (workspace_bytes < bwd_workspace(g)) return DBST_EINVAL;
+  auto s = static_cast<cudaStream_t>(stream);
+  auto* stats = static_cast<float2*>(workspace);
+  if (raster)
+    return g->D == 128 ? launch_bwd<128, true>(q, k, v, lse, dout, g, kv_count, kv_idx, q_count, q_idx, scale, dq, dk, dv, stats, s)
+                       : launch_bwd<64, true>(q, k, v, lse, dout, g, kv_count, kv_idx, q_count, q_idx, scale, dq, dk, dv, stats, s);
+  return g->D == 128 ? launch_bwd<128, false>(q, k, v, lse, dout, g, kv_count, kv_idx, q_count, q_idx, scale, dq, dk, dv, stats, s)
+                     : launch_bwd<64, false>(q, k, v, lse, dout, g, kv_count, kv_idx, q_count, q_idx, scale, dq, dk, dv, stats, s);
+}
+
 template <int NPT>
 bool launch_select(const double* S, const dbst::SelectGeo& sg, long long rows, uint32_t* bits, int32_t* cnt,
                    int16_t* idx, cudaStream_t s) {
@@ -400,6 +481,47 @@ dbst_status dbst_pair_query_blocks(const uint32_t* mask_bits, const dbst_geom* g
   kern<<<static_cast<unsigned>(bh), dbst::kPairingThreads, smem, static_cast<cudaStream_t>(stream)>>>(mask_bits, pg,
                                                                                                      pairs);
   return launch_status();
+}
+
+dbst_status dbst_transpose_block_mask(const uint32_t* mask_bits, const dbst_geom* g, uint32_t* mask_bits_t,
+                                      int32_t* q_count, int16_t* q_idx, void* stream) {
+  if (!geom_ok(g) || !mask_bits || !mask_bits_t || !q_count || !q_idx) return DBST_EINVAL;
+  if (!aligned16(mask_bits) || !aligned16(mask_bits_t) || !aligned16(q_count) || !aligned16(q_idx))
+    return DBST_EINVAL;
+  if (mask_bits == mask_bits_t) return DBST_EINVAL;
+  const int NB = nblocks(g), NW = (NB + 31) / 32;
+  const long long words = bh_count(g) * NB * NW;
+  long long grid = (words + 255) / 256;
+  const long long cap = static_cast<long long>(sm_count()) * 8;
+  if (grid > cap) grid = cap;
+  auto s = static_cast<cudaStream_t>(stream);
+  dbst::transpose_bits_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(mask_bits, mask_bits_t, NB, NW, words);
+  if (cudaGetLastError() != cudaSuccess) return DBST_ECUDA;
+  return dbst_mask_from_bits(mask_bits_t, g, q_count, q_idx, stream);
+}
+
+size_t dbst_attn_backward_workspace_bytes(const dbst_geom* g) {
+  if (!geom_ok(g)) return 0;
+  return bwd_workspace(g);
+}
+
+dbst_status dbst_block_sparse_attn_backward(const void* q, const void* k, const void* v, const float* lse,
+                                            const void* d_o, const dbst_geom* g,
+                                            const int32_t* kv_count, const int16_t* kv_idx, const int32_t* q_count,
+                                            const int16_t* q_idx, float scale, void* dq, void* dk, void* dv,
+                                            void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_common(q, k, v, lse, d_o, g, kv_count, kv_idx, q_count, q_idx, scale, dq, dk, dv, workspace,
+                    workspace_bytes, stream, false);
+}
+
+dbst_status dbst_block_sparse_attn_backward_raster(const void* q, const void* k, const void* v, const float* lse,
+                                                   const void* d_o, const dbst_geom* g,
+                                                   const int32_t* kv_count, const int16_t* kv_idx,
+                                                   const int32_t* q_count, const int16_t* q_idx, float scale,
+                                                   void* dq, void* dk, void* dv, void* workspace,
+                                                   size_t workspace_bytes, void* stream) {
+  return bwd_common(q, k, v, lse, d_o, g, kv_count, kv_idx, q_count, q_idx, scale, dq, dk, dv, workspace,
+                    workspace_bytes, stream, true);
 }
 
 dbst_status dbst_get_error(void* stream) {

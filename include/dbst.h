@@ -203,6 +203,63 @@ dbst_status dbst_build_block_mask_noalloc(const void* q_tiled, const void* k_til
                                           void* stream);
 
 /*
+ * Transposed block mask for the backward pass.  Row j of mask_bits_t lists
+ * the query blocks whose kept set contains key block j:
+ *   bit i of mask_bits_t[b,h,j,:]  ==  bit j of mask_bits[b,h,i,:]
+ * and (q_count, q_idx) are its index lists, ascending, in the layout of
+ * (kv_count, kv_idx).
+ *   mask_bits   : [B,H,NB,ceil(NB/32)] uint32, as written by the mask builders
+ *   mask_bits_t : out, same shape; must not be mask_bits
+ *   q_count     : out, [B,H,NB] int32
+ *   q_idx       : out, [B,H,NB,NB] int16 (entries past q_count unspecified)
+ */
+dbst_status dbst_transpose_block_mask(const uint32_t* mask_bits, const dbst_geom* g, uint32_t* mask_bits_t,
+                                      int32_t* q_count, int16_t* q_idx, void* stream);
+
+/* Bytes of device workspace dbst_block_sparse_attn_backward needs (8 per token row). */
+size_t dbst_attn_backward_workspace_bytes(const dbst_geom* g);
+
+/*
+ * Backward of dbst_block_sparse_attn over the same kept blocks.  The NABLA
+ * page trains and fine-tunes with the same adaptive mask; this is the exact
+ * gradient of the forward definition for an upstream gradient d_o of o.  For
+ * query block i with kept key tokens S_i, P = softmax(scale * q_i k_S^T):
+ *   dP      = d_o_i v_S^T
+ *   delta_n = sum_m P[n,m] * dP[n,m]       (per query token n; = d_o[n] . o[n])
+ *   dS      = P * (dP - delta)
+ *   dq_i    = scale * dS k_S
+ *   dk_S   += scale * dS^T q_i,   dv_S += P^T d_o_i        (over all i keeping S)
+ * P is recomputed from lse in float32 and delta is summed from that P, so the
+ * forward's o is not an input.  dS and P are rounded to bf16 before the
+ * products, accumulation is float32, outputs are bf16.  A query block with an
+ * empty list gets dq = 0 and contributes nothing; a key block no query keeps
+ * gets dk = dv = 0.
+ *   q, k, v     : tiled [B,H,N,D] bf16, the forward's inputs
+ *   lse         : the forward's [B,H,N] float32 log-sum-exp for the same lists
+ *   d_o         : tiled [B,H,N,D] bf16
+ *   kv_count, kv_idx : the forward's lists
+ *   q_count, q_idx   : their transpose (dbst_transpose_block_mask)
+ *   scale       : the forward's scale (<= 0 selects 1/sqrt(D))
+ *   dq, dk, dv  : out, tiled [B,H,N,D] bf16; every element is written
+ *   workspace   : >= dbst_attn_backward_workspace_bytes(g) bytes, 16-byte aligned
+ * Two launches on `stream`.  List entries outside [0, NB) are skipped and
+ * reported as DBST_EBOUNDS through dbst_get_error.
+ */
+dbst_status dbst_block_sparse_attn_backward(const void* q, const void* k, const void* v, const float* lse,
+                                            const void* d_o, const dbst_geom* g,
+                                            const int32_t* kv_count, const int16_t* kv_idx,
+                                            const int32_t* q_count, const int16_t* q_idx, float scale,
+                                            void* dq, void* dk, void* dv,
+                                            void* workspace, size_t workspace_bytes, void* stream);
+/* The same on raster-order q, k, v, lse, d_o, dq, dk, dv (lists still indexed by tile-ordered block). */
+dbst_status dbst_block_sparse_attn_backward_raster(const void* q, const void* k, const void* v, const float* lse,
+                                                   const void* d_o, const dbst_geom* g,
+                                                   const int32_t* kv_count, const int16_t* kv_idx,
+                                                   const int32_t* q_count, const int16_t* q_idx, float scale,
+                                                   void* dq, void* dk, void* dv,
+                                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Synchronises `stream`, then reports (and clears) the first device-side
  * error any kernel of this library recorded since the last call, or a pending
  * CUDA error.  DBST_OK if there was none.

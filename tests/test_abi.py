@@ -128,3 +128,38 @@ def test_python_binding_validates_shapes_before_calling():
     x = torch.zeros((1, 2, g.N, 128), dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         dbst.tile_reorder(x, g)          # not a CUDA tensor
+
+
+def test_backward_entry_points_validate_arguments(lib):
+    g = geom()
+    a = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    ws = lib.dbst_attn_backward_workspace_bytes(ctypes.byref(g))
+    assert ws == (1 * 2 * g.N * 8 + 255) // 256 * 256
+    assert lib.dbst_attn_backward_workspace_bytes(ctypes.byref(geom(D=96))) == 0
+    for fn in (lib.dbst_block_sparse_attn_backward, lib.dbst_block_sparse_attn_backward_raster):
+        ok = [a, a, a, a, a, ctypes.byref(g), a, a, a, a, 0.0, a, a, a, a, ws, None]
+        for i in (0, 1, 2, 3, 4, 6, 7, 8, 9, 11, 12, 13, 14):          # each pointer null
+            args = list(ok)
+            args[i] = None
+            assert fn(*args) == dbst.DBST_EINVAL, i
+        for i in (0, 4, 7, 9, 11, 14):                                 # misaligned
+            args = list(ok)
+            args[i] = odd
+            assert fn(*args) == dbst.DBST_EINVAL, i
+        args = list(ok)
+        args[3] = ctypes.c_void_p((1 << 20) + 2)                       # lse not 4-byte aligned
+        assert fn(*args) == dbst.DBST_EINVAL
+        args = list(ok)
+        args[15] = ws - 1                                              # workspace too small
+        assert fn(*args) == dbst.DBST_EINVAL
+        args = list(ok)
+        args[10] = float("nan")
+        assert fn(*args) == dbst.DBST_EINVAL
+        args = list(ok)
+        args[5] = ctypes.byref(geom(D=96))
+        assert fn(*args) == dbst.DBST_EINVAL
+    assert lib.dbst_transpose_block_mask(a, ctypes.byref(g), a, a, a, None) == dbst.DBST_EINVAL   # in place
+    assert lib.dbst_transpose_block_mask(None, ctypes.byref(g), a, a, a, None) == dbst.DBST_EINVAL
+    assert lib.dbst_transpose_block_mask(a, ctypes.byref(g), ctypes.c_void_p(1 << 30), odd, a, None) == dbst.DBST_EINVAL
+    assert lib.dbst_transpose_block_mask(a, None, ctypes.c_void_p(1 << 30), a, a, None) == dbst.DBST_EINVAL
