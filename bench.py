@@ -293,6 +293,59 @@ def run_sweep(args, w):
     return 0
 
 
+def run_backward(args, w, p):
+    """Backward of the block-sparse attention (raster layout) on one GPU: mask, its transpose, forward
+    for the log-sum-exp, then the timed backward.  One JSON line, not the headline metric."""
+    import torch
+    import dynamic_block_sparse_tile_b200 as dbst
+    dbst.load()
+    g = dbst.Geom.make(w.B, w.H, w.D, w.grid, w.tile)
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()   # noqa: E731
+    q, k, v = (to_dev(a) for a in S.make_qkv(w))
+    do = to_dev(S.make_grad(w))
+    bits, cnt, idx = dbst.build_block_mask_raster(q, k, g, p, w.sta_radius)
+    pairs = dbst.pair_query_blocks(bits, g)
+    o, lse = dbst.block_sparse_attn_raster(q, k, v, g, cnt, idx, pairs=pairs)
+    out_t = dbst.transpose_block_mask(bits, g)
+    _, qcnt, qidx = out_t
+    ws = torch.empty(dbst.attn_backward_workspace_bytes(g), dtype=torch.uint8, device="cuda")
+    grads = tuple(torch.empty_like(q) for _ in range(3))
+
+    def timed(fn):
+        for _ in range(max(args.warmup, 3)):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(args.steps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    fwd_ms = timed(lambda: dbst.block_sparse_attn_raster(q, k, v, g, cnt, idx, 0.0, True, o, lse, pairs))
+    tr_ms = timed(lambda: dbst.transpose_block_mask(bits, g, out=out_t))
+    bwd_ms = timed(lambda: dbst.block_sparse_attn_backward(q, k, v, lse, do, g, cnt, idx, qcnt, qidx, raster=True,
+                                                           workspace=ws, out=grads))
+    dbst.get_error()
+    kept = int(cnt.sum().item())
+    unit = 2.0 * w.D * 64 * 64 * kept            # one 64x64xD product over every kept block pair
+    _, bf16, _, src = peaks()
+    out = {"backward": workload_desc(w, p), "kept_fraction": kept / (g.B * g.H * g.NB * g.NB),
+           "backward_ms": bwd_ms, "forward_attn_ms": fwd_ms, "transpose_ms": tr_ms,
+           "backward_tflops": 5 * unit / (bwd_ms * 1e-3) / 1e12,
+           "backward_tensor_tflops": 9 * unit / (bwd_ms * 1e-3) / 1e12,
+           "forward_tflops": 2 * unit / (fwd_ms * 1e-3) / 1e12,
+           "bf16_peak_tflops": bf16, "peak_source": src,
+           "note": "backward_tflops counts the 5 products of the gradient (S, dP, dV, dK, dQ); the kernels "
+                   "run 9 (S and dP twice more: the delta sweep of the dq pass and the dk/dv pass)"}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -307,6 +360,8 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="sparsity sweep: attention ms/call and kept-block TFLOP/s per p, dense crossover")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward (gradients over the same kept blocks) instead of the forward step")
     ap.add_argument("--path", default="fused", choices=["fused", "explicit"],
                     help="fused: tile reorder folded into the kernels (raster entry points); explicit: separate passes")
     args = ap.parse_args()
@@ -316,6 +371,8 @@ def main():
         return run_reference(args, w, p)
     if args.sweep:
         return run_sweep(args, S.workload("sweep") if args.workload == "wan" else w)
+    if args.backward:
+        return run_backward(args, w, p)
 
     import torch
     import torch.distributed as dist
