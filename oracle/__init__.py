@@ -36,6 +36,7 @@ from .nabla import (  # noqa: F401
     mask_to_lists,
     masked_attention,
     masked_attention_backward,
+    masked_attention_backward_blocks,
     dense_attention,
     kept_pair_flops,
 )

@@ -306,6 +306,61 @@ def masked_attention_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, mask:
     return dq, dk, dv
 
 
+def masked_attention_backward_blocks(q: np.ndarray, k: np.ndarray, v: np.ndarray, mask: np.ndarray, blk: int,
+                                     scale: float, do: np.ndarray, q_blocks, k_blocks):
+    """The gradients of :func:`masked_attention_backward` for chosen blocks only (reading R9).
+
+    ``q_blocks``: iterable of (b, h, i) -> dq of query block i, ``[blk, D]``.
+    ``k_blocks``: iterable of (b, h, j) -> (dk, dv) of key block j, each ``[blk, D]``; they sum
+    over every query block that keeps j, so each such row is computed in full.
+    Returns two dicts keyed by those tuples.  Same arithmetic as the full function, restricted.
+    """
+    dec = bf16_bits_to_f64 if q.dtype == np.uint16 else (lambda a: np.asarray(a, dtype=np.float64))
+    q_blocks = [tuple(int(x) for x in t) for t in q_blocks]
+    k_blocks = [tuple(int(x) for x in t) for t in k_blocks]
+    want_q = set(q_blocks)
+    want_k = {}
+    for b, h, j in k_blocks:
+        want_k.setdefault((b, h), set()).add(j)
+    D = q.shape[-1]
+    dq_out = {}
+    dkv = {t: (np.zeros((blk, D)), np.zeros((blk, D))) for t in k_blocks}
+    heads = {(b, h) for b, h, _ in q_blocks} | set(want_k)
+    for b, h in sorted(heads):
+        kj = want_k.get((b, h), set())
+        rows = {i for bb, hh, i in q_blocks if (bb, hh) == (b, h)}
+        for j in kj:
+            rows |= set(np.nonzero(mask[b, h, :, j])[0].tolist())
+        for i in sorted(rows):
+            kept = np.nonzero(mask[b, h, i])[0]
+            if kept.size == 0:
+                if (b, h, i) in want_q:
+                    dq_out[(b, h, i)] = np.zeros((blk, D))
+                continue
+            tok = (kept[:, None] * blk + np.arange(blk)[None, :]).reshape(-1)
+            r = slice(i * blk, (i + 1) * blk)
+            qi, ks, vs = dec(q[b, h, r]), dec(k[b, h, tok]), dec(v[b, h, tok])
+            doi = np.asarray(do[b, h, r], dtype=np.float64)
+            s = (qi @ ks.T) * scale
+            e = np.exp(s - s.max(axis=1, keepdims=True))
+            P = e / e.sum(axis=1, keepdims=True)
+            oi = P @ vs
+            dP = doi @ vs.T
+            delta = np.sum(doi * oi, axis=1, keepdims=True)
+            ds = P * (dP - delta)
+            if (b, h, i) in want_q:
+                dq_out[(b, h, i)] = scale * (ds @ ks)
+            for pos, j in enumerate(kept):
+                if int(j) in kj:
+                    c = slice(pos * blk, (pos + 1) * blk)
+                    dk_j, dv_j = dkv[(b, h, int(j))]
+                    dk_j += scale * (ds[:, c].T @ qi)
+                    dv_j += P[:, c].T @ doi
+    for t in q_blocks:
+        dq_out.setdefault(t, np.zeros((blk, D)))
+    return dq_out, dkv
+
+
 def dense_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float):
     """softmax(scale * q k^T) v over all tokens, fp64; returns (o, lse)."""
     if q.dtype == np.uint16:

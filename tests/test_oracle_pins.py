@@ -455,3 +455,23 @@ def test_backward_is_linear_in_do_and_reads_bf16_bits():
     for a, b, c, e in zip(g1, g2, g12, gf):
         np.testing.assert_allclose(c, 2 * a - 3 * b, rtol=1e-12, atol=1e-12)
         np.testing.assert_array_equal(a, e)
+
+
+def test_backward_blocks_equal_full_backward():
+    """The sampled-block form returns the full function's values for the chosen blocks (including
+    a query block with an empty list and a key block nobody keeps)."""
+    B, H, NB, blk, D = 2, 2, 5, 8, 4
+    q, k, v, do = (RNG.standard_normal((B, H, NB * blk, D)) for _ in range(4))
+    mask = RNG.random((B, H, NB, NB)) < 0.5
+    mask[0, 1, 3] = False
+    mask[1, 0, :, 2] = False
+    dq, dk, dv = O.masked_attention_backward(q, k, v, mask, blk, 0.4, do)
+    qs = [(0, 1, 3), (1, 1, 0), (0, 0, 4)]
+    ks = [(1, 0, 2), (0, 1, 1), (1, 1, 4), (0, 1, 0)]
+    gq, gkv = O.masked_attention_backward_blocks(q, k, v, mask, blk, 0.4, do, qs, ks)
+    for b, h, i in qs:
+        np.testing.assert_allclose(gq[(b, h, i)], dq[b, h, i * blk:(i + 1) * blk], rtol=1e-12, atol=1e-14)
+    for b, h, j in ks:
+        np.testing.assert_allclose(gkv[(b, h, j)][0], dk[b, h, j * blk:(j + 1) * blk], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(gkv[(b, h, j)][1], dv[b, h, j * blk:(j + 1) * blk], rtol=1e-12, atol=1e-14)
+    assert not gq[(0, 1, 3)].any() and not gkv[(1, 0, 2)][0].any() and not gkv[(1, 0, 2)][1].any()
