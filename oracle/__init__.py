@@ -19,8 +19,12 @@ Sources (cited by page title and section):
   "Les trois techniques": the kernel gathers the selected key/value blocks
   by index, which is why the mask is also emitted as per-row index lists.
 
+* "SQuad: Sub-Quadratic Attention Distillation for Efficient Video
+  Generation", section "Methodology: SQuad", item "1. SQuad-Attention
+  Operator": the two-pass operator (``oracle.squad``).
+
 Readings adopted where the pages are silent or garbled are listed in the
-module docstring of ``oracle.nabla``.
+module docstrings of ``oracle.nabla`` and ``oracle.squad``.
 """
 from .nabla import (  # noqa: F401
     Geometry,
@@ -40,3 +44,4 @@ from .nabla import (  # noqa: F401
     dense_attention,
     kept_pair_flops,
 )
+from .squad import squad_attention, squad_flops  # noqa: F401
