@@ -346,6 +346,47 @@ def run_backward(args, w, p):
     return 0
 
 
+def run_squad(args):
+    """SQuad two-pass attention against dense attention on the same tensors (B=2 H=16 N=16384 D=128,
+    w = sqrt(N) = 128).  One JSON line; not the headline metric."""
+    import torch
+    import dynamic_block_sparse_tile_b200 as dbst
+    dbst.load()
+    w = S.workload("sweep")
+    win = int(round(math.sqrt(w.N)))
+    g = dbst.Geom.make(w.B, w.H, w.D, w.grid, w.tile)
+    q, k, v = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda() for a in S.make_qkv(w))
+    ws = torch.empty(dbst.squad_workspace_bytes(w.B, w.H, w.N, w.D, win), dtype=torch.uint8, device="cuda")
+    o = torch.empty_like(q)
+
+    def timed(fn):
+        for _ in range(max(args.warmup, 3)):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(args.steps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    squad_ms = timed(lambda: dbst.squad_attn(q, k, v, win, workspace=ws, out=o))
+    dense_ms = timed(lambda: dbst.dense_attn_raster(q, k, v, g))
+    dbst.get_error()
+    flops = 4.0 * w.D * w.N * (win + w.N // win) * w.B * w.H
+    moved = 2 * 4 * w.B * w.H * w.N * w.D * 2      # four window transposes, each a read and a write
+    out = {"squad": f"B={w.B} H={w.H} N={w.N} D={w.D} w={win}", "squad_ms": squad_ms, "dense_attn_ms": dense_ms,
+           "speedup_vs_dense": dense_ms / squad_ms, "squad_tflops": flops / (squad_ms * 1e-3) / 1e12,
+           "squad_flop_fraction_of_dense": flops / (4.0 * w.D * w.N * w.N * w.B * w.H),
+           "transpose_bytes": moved, "launches": 6}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -360,6 +401,7 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="sparsity sweep: attention ms/call and kept-block TFLOP/s per p, dense crossover")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--squad", action="store_true", help="time SQuad two-pass attention against dense attention")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward (gradients over the same kept blocks) instead of the forward step")
     ap.add_argument("--path", default="fused", choices=["fused", "explicit"],
@@ -373,6 +415,8 @@ def main():
         return run_sweep(args, S.workload("sweep") if args.workload == "wan" else w)
     if args.backward:
         return run_backward(args, w, p)
+    if args.squad:
+        return run_squad(args)
 
     import torch
     import torch.distributed as dist

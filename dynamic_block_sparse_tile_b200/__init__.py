@@ -21,7 +21,7 @@ __all__ = ["Geom", "DbstError", "lib_path", "load", "tile_reorder", "tile_unreor
            "build_block_mask", "build_block_mask_noalloc", "mask_from_bits", "block_sparse_attn", "dense_attn",
            "build_block_mask_raster", "block_sparse_attn_raster", "dense_attn_raster", "pair_query_blocks",
            "transpose_block_mask", "attn_backward_workspace_bytes", "block_sparse_attn_backward",
-           "get_error", "EXPORTS"]
+           "squad_workspace_bytes", "squad_attn", "get_error", "EXPORTS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libdbst.so")
@@ -32,7 +32,7 @@ EXPORTS = ("dbst_status_string", "dbst_tile_reorder", "dbst_tile_unreorder", "db
            "dbst_get_error", "dbst_build_block_mask_noalloc", "dbst_build_block_mask_raster",
            "dbst_block_sparse_attn_raster", "dbst_dense_attn_raster", "dbst_pair_query_blocks",
            "dbst_transpose_block_mask", "dbst_attn_backward_workspace_bytes", "dbst_block_sparse_attn_backward",
-           "dbst_block_sparse_attn_backward_raster")
+           "dbst_block_sparse_attn_backward_raster", "dbst_squad_workspace_bytes", "dbst_squad_attn")
 
 DBST_OK, DBST_EINVAL, DBST_ECUDA, DBST_ETIMEOUT, DBST_EBOUNDS, DBST_ETOOLARGE = 0, 1, 2, 3, 4, 5
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -106,6 +106,10 @@ def load() -> ctypes.CDLL:
     for name in ("dbst_block_sparse_attn_backward", "dbst_block_sparse_attn_backward_raster"):
         getattr(lib, name).argtypes = [vp, vp, vp, vp, vp, gp, vp, vp, vp, vp, f32, vp, vp, vp, vp, ctypes.c_size_t, vp]
         getattr(lib, name).restype = i32
+    lib.dbst_squad_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
+    lib.dbst_squad_workspace_bytes.restype = ctypes.c_size_t
+    lib.dbst_squad_attn.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp, ctypes.c_size_t, vp]
+    lib.dbst_squad_attn.restype = i32
     _lib = lib
     return lib
 
@@ -340,6 +344,31 @@ def block_sparse_attn_backward(q, k, v, lse, d_o, g: Geom, kv_count, kv_idx, q_c
                                _ptr(kv_idx), _ptr(q_count), _ptr(q_idx), float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
                                _ptr(workspace), workspace.numel() * workspace.element_size(), _stream()), fn)
     return dq, dk, dv
+
+
+def squad_workspace_bytes(B: int, H: int, N: int, D: int, w: int) -> int:
+    return int(load().dbst_squad_workspace_bytes(B, H, N, D, w))
+
+
+def squad_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, w: int, scale: float = 0.0,
+               workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """SQuad two-pass attention with window w (``dbst_squad_attn``) on [B, H, N, D] bf16 -> o."""
+    if q.dim() != 4:
+        raise ValueError("q: expected [B, H, N, D]")
+    B, H, N, D = q.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, (B, H, N, D), n)
+    o = torch.empty_like(q) if out is None else out
+    _need(o, torch.bfloat16, (B, H, N, D), "out")
+    nbytes = squad_workspace_bytes(B, H, N, D, w)
+    if nbytes == 0:
+        raise ValueError(f"unsupported SQuad shape N={N} D={D} w={w}: w and N/w must be multiples of 64")
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    _check(load().dbst_squad_attn(_ptr(q), _ptr(k), _ptr(v), B, H, N, D, int(w), float(scale), _ptr(o),
+                                  _ptr(workspace), workspace.numel() * workspace.element_size(), _stream()),
+           "dbst_squad_attn")
+    return o
 
 
 def get_error() -> None:

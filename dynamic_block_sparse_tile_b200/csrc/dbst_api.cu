@@ -17,6 +17,7 @@
 #include "mask.cuh"
 #include "ptx.cuh"
 #include "reorder.cuh"
+#include "squad.cuh"
 
 namespace {
 
@@ -297,6 +298,39 @@ dbst_status bwd_common(const void* q, const void* k, const void* v, const float*
                      : launch_bwd<64, false>(q, k, v, lse, dout, g, kv_count, kv_idx, q_count, q_idx, scale, dq, dk, dv, stats, s);
 }
 
+// SQuad shapes: D in {64, 128}; the window w and the window count m = N / w both multiples of 64
+// (each pass's sequence is whole 64-token blocks), at most 4096 blocks per sequence.
+bool squad_ok(int B, int H, int N, int D, int w) {
+  if (B < 1 || H < 1 || N < 1 || (D != 64 && D != 128)) return false;
+  if (w < 64 || w % 64 || N % w) return false;
+  const int m = N / w;
+  if (m < 64 || m % 64) return false;
+  if (w / 64 > kMaxNB || m / 64 > kMaxNB) return false;
+  const long long rows = static_cast<long long>(B) * H * N;
+  if (rows >= (1ll << 31)) return false;
+  if (static_cast<long long>(H) * m >= (1ll << 31) || static_cast<long long>(H) * w >= (1ll << 31)) return false;
+  return true;
+}
+
+size_t squad_tensor_bytes(int B, int H, int N, int D) {
+  return align_up(static_cast<size_t>(B) * H * N * D * 2);
+}
+
+dbst_status window_transpose(const void* src, void* dst, long long heads, int A, int R, int D, cudaStream_t s) {
+  const int cpr_log2 = D == 128 ? 4 : 3;
+  const long long total = (heads * A * R) << cpr_log2;
+  long long grid = (total + 256 * dbst::kPermuteUnroll - 1) / (256 * dbst::kPermuteUnroll);
+  const long long cap = static_cast<long long>(sm_count()) * 16;
+  if (grid > cap) grid = cap;
+  const auto* in = static_cast<const uint4*>(src);
+  auto* out = static_cast<uint4*>(dst);
+  if (D == 128)
+    dbst::window_transpose_kernel<4><<<static_cast<unsigned>(grid), 256, 0, s>>>(in, out, A, R, total);
+  else
+    dbst::window_transpose_kernel<3><<<static_cast<unsigned>(grid), 256, 0, s>>>(in, out, A, R, total);
+  return cudaGetLastError() == cudaSuccess ? DBST_OK : DBST_ECUDA;
+}
+
 template <int NPT>
 bool launch_select(const double* S, const dbst::SelectGeo& sg, long long rows, uint32_t* bits, int32_t* cnt,
                    int16_t* idx, cudaStream_t s) {
@@ -522,6 +556,40 @@ dbst_status dbst_block_sparse_attn_backward_raster(const void* q, const void* k,
                                                    size_t workspace_bytes, void* stream) {
   return bwd_common(q, k, v, lse, d_o, g, kv_count, kv_idx, q_count, q_idx, scale, dq, dk, dv, workspace,
                     workspace_bytes, stream, true);
+}
+
+size_t dbst_squad_workspace_bytes(int B, int H, int N, int D, int w) {
+  if (!squad_ok(B, H, N, D, w)) return 0;
+  return 4 * squad_tensor_bytes(B, H, N, D);
+}
+
+dbst_status dbst_squad_attn(const void* q, const void* k, const void* v, int B, int H, int N, int D, int w,
+                            float scale, void* o, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!squad_ok(B, H, N, D, w) || !q || !k || !v || !o || !workspace) return DBST_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(workspace)) return DBST_EINVAL;
+  if (!std::isfinite(scale)) return DBST_EINVAL;
+  const size_t tb = squad_tensor_bytes(B, H, N, D);
+  if (workspace_bytes < 4 * tb) return DBST_EINVAL;
+  auto s = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  void* o_loc = ws;              // local output, later the global output in window-transposed order
+  void* qT = ws + tb;
+  void* kT = ws + 2 * tb;
+  void* o_locT = ws + 3 * tb;
+  const int m = N / w;
+  const long long heads = static_cast<long long>(B) * H;
+  // local pass: every window is a sequence of its own
+  const dbst_geom gl = {B, H * m, D, 1, 1, w, 1, 1, 64};
+  dbst_status st = attn_common(q, k, v, &gl, nullptr, nullptr, nullptr, scale, o_loc, nullptr, stream, false);
+  if (st != DBST_OK) return st;
+  // global pass: offset r of every window forms a sequence of m tokens
+  if ((st = window_transpose(q, qT, heads, m, w, D, s)) != DBST_OK) return st;
+  if ((st = window_transpose(k, kT, heads, m, w, D, s)) != DBST_OK) return st;
+  if ((st = window_transpose(o_loc, o_locT, heads, m, w, D, s)) != DBST_OK) return st;
+  const dbst_geom gg = {B, H * w, D, 1, 1, m, 1, 1, 64};
+  st = attn_common(qT, kT, o_locT, &gg, nullptr, nullptr, nullptr, scale, o_loc, nullptr, stream, false);
+  if (st != DBST_OK) return st;
+  return window_transpose(o_loc, o, heads, w, m, D, s);
 }
 
 dbst_status dbst_get_error(void* stream) {

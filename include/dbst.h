@@ -260,6 +260,27 @@ dbst_status dbst_block_sparse_attn_backward_raster(const void* q, const void* k,
                                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * SQuad two-pass attention (page "SQuad: Sub-Quadratic Attention Distillation
+ * for Efficient Video Generation", section "Methodology: SQuad", item
+ * "1. SQuad-Attention Operator").  The N tokens of each (b, h) are read as
+ * m = N / w windows of w consecutive tokens (token t: window t / w, offset
+ * t % w).  With softmax scale `scale` (<= 0 selects 1/sqrt(D)):
+ *   local  : o_L[t] = sum over t2 in window(t)      softmax(scale <q_t, k_t2>) v[t2]
+ *   global : o[t]   = sum over t2 with t2 % w = t % w  softmax(scale <q_t, k_t2>) o_L[t2]
+ * Both passes are the dense attention kernel (float32 softmax, bf16 output; o_L
+ * is rounded to bf16 before it feeds the global pass); the global pass runs on
+ * window-transposed copies of q, k and o_L.  Six launches on `stream`.
+ *   q, k, v, o : [B,H,N,D] bf16, sequence order as given by the caller
+ *   w          : window; w and N / w must be multiples of 64 (the page takes
+ *                w = sqrt(N), e.g. N = 16384, w = 128)
+ *   workspace  : >= dbst_squad_workspace_bytes(B,H,N,D,w) bytes (4 tensors)
+ * Unsupported shapes return DBST_EINVAL (and a workspace size of 0).
+ */
+size_t dbst_squad_workspace_bytes(int B, int H, int N, int D, int w);
+dbst_status dbst_squad_attn(const void* q, const void* k, const void* v, int B, int H, int N, int D, int w,
+                            float scale, void* o, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Synchronises `stream`, then reports (and clears) the first device-side
  * error any kernel of this library recorded since the last call, or a pending
  * CUDA error.  DBST_OK if there was none.

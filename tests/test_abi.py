@@ -163,3 +163,18 @@ def test_backward_entry_points_validate_arguments(lib):
     assert lib.dbst_transpose_block_mask(None, ctypes.byref(g), a, a, a, None) == dbst.DBST_EINVAL
     assert lib.dbst_transpose_block_mask(a, ctypes.byref(g), ctypes.c_void_p(1 << 30), odd, a, None) == dbst.DBST_EINVAL
     assert lib.dbst_transpose_block_mask(a, None, ctypes.c_void_p(1 << 30), a, a, None) == dbst.DBST_EINVAL
+
+
+def test_squad_entry_point_validates_shapes(lib):
+    a = ctypes.c_void_p(1 << 20)
+    tb = 2 * 16384 * 128 * 2
+    assert lib.dbst_squad_workspace_bytes(1, 2, 16384, 128, 128) == 4 * tb
+    for B, H, N, D, w in ((1, 2, 16384, 96, 128), (1, 2, 16384, 128, 100), (1, 2, 16384, 128, 32),
+                          (1, 2, 8192, 128, 256), (0, 2, 16384, 128, 128), (1, 2, 16000, 128, 128)):
+        assert lib.dbst_squad_workspace_bytes(B, H, N, D, w) == 0, (N, D, w)   # N/w=32 is rejected too
+        assert lib.dbst_squad_attn(a, a, a, B, H, N, D, w, 0.0, a, a, 1 << 40, None) == dbst.DBST_EINVAL
+    ok = (1, 2, 16384, 128, 128)
+    assert lib.dbst_squad_attn(a, a, a, *ok, 0.0, a, a, 4 * tb - 1, None) == dbst.DBST_EINVAL
+    assert lib.dbst_squad_attn(None, a, a, *ok, 0.0, a, a, 4 * tb, None) == dbst.DBST_EINVAL
+    assert lib.dbst_squad_attn(a, a, ctypes.c_void_p((1 << 20) + 8), *ok, 0.0, a, a, 4 * tb, None) == dbst.DBST_EINVAL
+    assert lib.dbst_squad_attn(a, a, a, *ok, float("nan"), a, a, 4 * tb, None) == dbst.DBST_EINVAL
