@@ -19,12 +19,15 @@ Sources (cited by page title and section):
   "Les trois techniques": the kernel gathers the selected key/value blocks
   by index, which is why the mask is also emitted as per-row index lists.
 
+* the same AB-Attention page, section "Les trois techniques", second
+  technique (SIP): sampled key blocks with inverse-probability logit
+  offsets (``oracle.sip``).
 * "SQuad: Sub-Quadratic Attention Distillation for Efficient Video
   Generation", section "Methodology: SQuad", item "1. SQuad-Attention
   Operator": the two-pass operator (``oracle.squad``).
 
 Readings adopted where the pages are silent or garbled are listed in the
-module docstrings of ``oracle.nabla`` and ``oracle.squad``.
+module docstrings of ``oracle.nabla``, ``oracle.sip`` and ``oracle.squad``.
 """
 from .nabla import (  # noqa: F401
     Geometry,
@@ -45,3 +48,4 @@ from .nabla import (  # noqa: F401
     kept_pair_flops,
 )
 from .squad import squad_attention, squad_flops  # noqa: F401
+from .sip import inclusion_probabilities, inclusion_probabilities_row, sip_attention, sip_sample  # noqa: F401
