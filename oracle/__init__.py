@@ -22,12 +22,15 @@ Sources (cited by page title and section):
 * the same AB-Attention page, section "Les trois techniques", second
   technique (SIP): sampled key blocks with inverse-probability logit
   offsets (``oracle.sip``).
+* the same section, third technique: key groups of 4 tokens gathered by
+  index into full tiles (``oracle.fine``).
 * "SQuad: Sub-Quadratic Attention Distillation for Efficient Video
   Generation", section "Methodology: SQuad", item "1. SQuad-Attention
   Operator": the two-pass operator (``oracle.squad``).
 
 Readings adopted where the pages are silent or garbled are listed in the
-module docstrings of ``oracle.nabla``, ``oracle.sip`` and ``oracle.squad``.
+module docstrings of ``oracle.nabla``, ``oracle.sip``, ``oracle.fine`` and
+``oracle.squad``.
 """
 from .nabla import (  # noqa: F401
     Geometry,
@@ -49,3 +52,4 @@ from .nabla import (  # noqa: F401
 )
 from .squad import squad_attention, squad_flops  # noqa: F401
 from .sip import inclusion_probabilities, inclusion_probabilities_row, sip_attention, sip_sample  # noqa: F401
+from .fine import build_fine_mask, fine_masked_attention, fine_score_map, kept_mass  # noqa: F401
