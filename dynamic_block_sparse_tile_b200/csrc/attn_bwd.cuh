@@ -1,8 +1,10 @@
 // Backward of block-sparse attention over the kept 64 x 64 tile pairs.
 //
 // The NABLA page ("NABLA: Neighborhood Adaptive Block-Level Attention",
-// sections on training and fine-tuning) uses the same adaptive mask in
-// training, which needs the gradient of the masked attention.  It is the exact
+// section "Contributions Clés", double-phase acceleration, and section
+// "Résultats Expérimentaux", items 1 and 2: fine-tuning and pre-training) uses
+// the same adaptive mask in training, which needs the gradient of the masked
+// attention.  It is the exact
 // gradient of the forward definition: for query block i with kept key tokens
 // S_i, P = softmax(scale * q_i k_S^T), dP = dO_i v_S^T, delta = rowsum(P * dP)
 // (one value per query row; it equals rowsum(dO_i * o_i)) and dS = P * (dP - delta):

@@ -221,8 +221,10 @@ size_t dbst_attn_backward_workspace_bytes(const dbst_geom* g);
 
 /*
  * Backward of dbst_block_sparse_attn over the same kept blocks.  The NABLA
- * page trains and fine-tunes with the same adaptive mask; this is the exact
- * gradient of the forward definition for an upstream gradient d_o of o.  For
+ * page (sections "Contributions Clés" and "Résultats Expérimentaux", items on
+ * fine-tuning and pre-training) trains with the same adaptive mask; this is
+ * the exact gradient of the forward definition for an upstream gradient d_o
+ * of o.  For
  * query block i with kept key tokens S_i, P = softmax(scale * q_i k_S^T):
  *   dP      = d_o_i v_S^T
  *   delta_n = sum_m P[n,m] * dP[n,m]       (per query token n; = d_o[n] . o[n])

@@ -33,7 +33,8 @@ R7  Token reorder ("Fractal Flattening") generalised from P x P spatial
     tokens inside a tile in raster order.  The time order of tiles is kept.
 R8  Blocks are the 64-token tiles: the pooling block of N tokens is one
     tile, so query block i and key block j both mean tile i / tile j.
-R9  Backward (the page claims faster training but prints no backward): the
+R9  Backward (the page claims faster training, sections "Contributions Clés"
+    and "Résultats Expérimentaux", but prints no backward): the
     exact gradient of the forward definition of :func:`masked_attention`
     with respect to q, k and v, for an upstream gradient do of o.  A key
     token receives gradient only from the query blocks that keep its block;
