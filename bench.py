@@ -346,6 +346,57 @@ def run_backward(args, w, p):
     return 0
 
 
+def run_sip(args, w, p):
+    """SIP on the Wan-like workload: sampled mask with inclusion-probability offsets at the
+    NABLA mask's mean kept count per row, then the offset attention; plus that attention
+    without offsets on the NABLA mask.  One JSON line; not the headline metric."""
+    import torch
+    import dynamic_block_sparse_tile_b200 as dbst
+    dbst.load()
+    g = dbst.Geom.make(w.B, w.H, w.D, w.grid, w.tile)
+    q, k, v = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda() for a in S.make_qkv(w))
+    bits, cnt, idx = dbst.build_block_mask_raster(q, k, g, p, w.sta_radius)
+    budget = float(cnt.double().mean().item())
+    gen = torch.Generator(device="cuda").manual_seed(1234)
+    u = torch.rand((g.B, g.H, g.NB, g.NB), dtype=torch.float64, device="cuda", generator=gen)
+    ws = torch.empty(dbst.mask_workspace_bytes(g), dtype=torch.uint8, device="cuda")
+    sip = dbst.build_sip_mask(q, k, g, budget, u, raster=True, workspace=ws)
+    o = torch.empty_like(q)
+    lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device="cuda")
+
+    def timed(fn):
+        for _ in range(max(args.warmup, 3)):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(args.steps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    sel_ms = timed(lambda: dbst.build_sip_mask(q, k, g, budget, u, raster=True, workspace=ws, out=sip))
+    attn_ms = timed(lambda: dbst.block_sparse_attn_offsets(q, k, v, g, sip[1], sip[2], sip[3], raster=True,
+                                                           out=o, lse=lse))
+    plain_ms = timed(lambda: dbst.block_sparse_attn_offsets(q, k, v, g, cnt, idx, None, raster=True, out=o, lse=lse))
+    dbst.get_error()
+    kept_sip = int(sip[1].sum().item())
+    kept = int(cnt.sum().item())
+    unit = 4.0 * w.D * 64 * 64
+    out = {"sip": workload_desc(w, p), "budget_blocks_per_row": budget,
+           "kept_fraction_sip": kept_sip / (g.B * g.H * g.NB * g.NB), "sip_mask_ms": sel_ms,
+           "sip_attn_ms": attn_ms, "sip_attn_tflops": unit * kept_sip / (attn_ms * 1e-3) / 1e12,
+           "two_sweep_attn_on_nabla_mask_ms": plain_ms,
+           "two_sweep_attn_tflops": unit * kept / (plain_ms * 1e-3) / 1e12,
+           "note": "TFLOP/s count the 2 products of attention per kept block pair; the two-sweep kernel runs 3"}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def run_squad(args):
     """SQuad two-pass attention against dense attention on the same tensors (B=2 H=16 N=16384 D=128,
     w = sqrt(N) = 128).  One JSON line; not the headline metric."""
@@ -402,6 +453,8 @@ def main():
                     help="sparsity sweep: attention ms/call and kept-block TFLOP/s per p, dense crossover")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--squad", action="store_true", help="time SQuad two-pass attention against dense attention")
+    ap.add_argument("--sip", action="store_true",
+                    help="time the SIP sampled mask and the attention with inclusion-probability offsets")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward (gradients over the same kept blocks) instead of the forward step")
     ap.add_argument("--path", default="fused", choices=["fused", "explicit"],
@@ -417,6 +470,8 @@ def main():
         return run_backward(args, w, p)
     if args.squad:
         return run_squad(args)
+    if args.sip:
+        return run_sip(args, w, p)
 
     import torch
     import torch.distributed as dist

@@ -21,7 +21,8 @@ __all__ = ["Geom", "DbstError", "lib_path", "load", "tile_reorder", "tile_unreor
            "build_block_mask", "build_block_mask_noalloc", "mask_from_bits", "block_sparse_attn", "dense_attn",
            "build_block_mask_raster", "block_sparse_attn_raster", "dense_attn_raster", "pair_query_blocks",
            "transpose_block_mask", "attn_backward_workspace_bytes", "block_sparse_attn_backward",
-           "squad_workspace_bytes", "squad_attn", "get_error", "EXPORTS"]
+           "squad_workspace_bytes", "squad_attn", "build_sip_mask", "block_sparse_attn_offsets", "get_error",
+           "EXPORTS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libdbst.so")
@@ -32,7 +33,9 @@ EXPORTS = ("dbst_status_string", "dbst_tile_reorder", "dbst_tile_unreorder", "db
            "dbst_get_error", "dbst_build_block_mask_noalloc", "dbst_build_block_mask_raster",
            "dbst_block_sparse_attn_raster", "dbst_dense_attn_raster", "dbst_pair_query_blocks",
            "dbst_transpose_block_mask", "dbst_attn_backward_workspace_bytes", "dbst_block_sparse_attn_backward",
-           "dbst_block_sparse_attn_backward_raster", "dbst_squad_workspace_bytes", "dbst_squad_attn")
+           "dbst_block_sparse_attn_backward_raster", "dbst_squad_workspace_bytes", "dbst_squad_attn",
+           "dbst_build_sip_mask", "dbst_build_sip_mask_raster", "dbst_block_sparse_attn_offsets",
+           "dbst_block_sparse_attn_offsets_raster")
 
 DBST_OK, DBST_EINVAL, DBST_ECUDA, DBST_ETIMEOUT, DBST_EBOUNDS, DBST_ETOOLARGE = 0, 1, 2, 3, 4, 5
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -110,6 +113,12 @@ def load() -> ctypes.CDLL:
     lib.dbst_squad_workspace_bytes.restype = ctypes.c_size_t
     lib.dbst_squad_attn.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp, ctypes.c_size_t, vp]
     lib.dbst_squad_attn.restype = i32
+    for name in ("dbst_build_sip_mask", "dbst_build_sip_mask_raster"):
+        getattr(lib, name).argtypes = [vp, vp, gp, ctypes.c_double, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        getattr(lib, name).restype = i32
+    for name in ("dbst_block_sparse_attn_offsets", "dbst_block_sparse_attn_offsets_raster"):
+        getattr(lib, name).argtypes = [vp, vp, vp, gp, vp, vp, vp, f32, vp, vp, vp]
+        getattr(lib, name).restype = i32
     _lib = lib
     return lib
 
@@ -344,6 +353,53 @@ def block_sparse_attn_backward(q, k, v, lse, d_o, g: Geom, kv_count, kv_idx, q_c
                                _ptr(kv_idx), _ptr(q_count), _ptr(q_idx), float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
                                _ptr(workspace), workspace.numel() * workspace.element_size(), _stream()), fn)
     return dq, dk, dv
+
+
+def build_sip_mask(q, k, g: Geom, budget: float, uniforms: torch.Tensor, raster: bool = False,
+                   workspace: Optional[torch.Tensor] = None, out=None):
+    """Sampled block mask with inclusion-probability offsets (``dbst_build_sip_mask[_raster]``).
+
+    ``uniforms``: float64 [B, H, NB, NB] in [0, 1).  Returns (mask_bits, kv_count, kv_idx, offsets),
+    offsets float32 [B, H, NB, NB] = log(1/pi) at kept blocks.
+    """
+    _need(q, torch.bfloat16, _qkv_shape(g), "q")
+    _need(k, torch.bfloat16, _qkv_shape(g), "k")
+    _need(uniforms, torch.float64, (g.B, g.H, g.NB, g.NB), "uniforms")
+    dev = q.device
+    if out is None:
+        bits = torch.empty((g.B, g.H, g.NB, g.NW), dtype=torch.int32, device=dev)
+        cnt = torch.empty((g.B, g.H, g.NB), dtype=torch.int32, device=dev)
+        idx = torch.empty((g.B, g.H, g.NB, g.NB), dtype=torch.int16, device=dev)
+        offsets = torch.empty((g.B, g.H, g.NB, g.NB), dtype=torch.float32, device=dev)
+    else:
+        bits, cnt, idx, offsets = out
+    if workspace is None:
+        workspace = torch.empty(mask_workspace_bytes(g), dtype=torch.uint8, device=dev)
+    fn = "dbst_build_sip_mask_raster" if raster else "dbst_build_sip_mask"
+    _check(getattr(load(), fn)(_ptr(q), _ptr(k), ctypes.byref(g), float(budget), _ptr(uniforms), _ptr(bits),
+                               _ptr(cnt), _ptr(idx), _ptr(offsets), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream()), fn)
+    return bits, cnt, idx, offsets
+
+
+def block_sparse_attn_offsets(q, k, v, g: Geom, kv_count, kv_idx, offsets: Optional[torch.Tensor] = None,
+                              scale: float = 0.0, raster: bool = False, want_lse: bool = True,
+                              out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None):
+    """Attention over kept blocks with a logit offset per (query block, key block)
+    (``dbst_block_sparse_attn_offsets[_raster]``) -> (o, lse or None)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, _qkv_shape(g), n)
+    _need(kv_count, torch.int32, (g.B, g.H, g.NB), "kv_count")
+    _need(kv_idx, torch.int16, (g.B, g.H, g.NB, g.NB), "kv_idx")
+    if offsets is not None:
+        _need(offsets, torch.float32, (g.B, g.H, g.NB, g.NB), "offsets")
+    o = torch.empty_like(q) if out is None else out
+    if want_lse and lse is None:
+        lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device=q.device)
+    fn = "dbst_block_sparse_attn_offsets_raster" if raster else "dbst_block_sparse_attn_offsets"
+    _check(getattr(load(), fn)(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(g), _ptr(kv_count), _ptr(kv_idx),
+                               _ptr(offsets), float(scale), _ptr(o), _ptr(lse if want_lse else None), _stream()), fn)
+    return o, (lse if want_lse else None)
 
 
 def squad_workspace_bytes(B: int, H: int, N: int, D: int, w: int) -> int:

@@ -1,0 +1,636 @@
+// Block-sparse attention kernels built on one tile walk: a CTA keeps its own 128 rows (two
+// 64-token blocks) in shared memory while the 64-row blocks of the other side stream through a
+// ring, one block per tile, over the union of the two own blocks' lists.  Three uses:
+//   MODE 0  backward, dq pass            MODE 1  backward, dk/dv pass
+//   MODE 2  forward with a logit offset per (query block, key block)
+//
+// ---- Backward (MODES 0 and 1)
+// The NABLA page ("NABLA: Neighborhood Adaptive Block-Level Attention",
+// section "Contributions Clés", double-phase acceleration, and section
+// "Résultats Expérimentaux", items 1 and 2: fine-tuning and pre-training) uses
+// the same adaptive mask in training, which needs the gradient of the masked
+// attention.  It is the exact
+// gradient of the forward definition: for query block i with kept key tokens
+// S_i, P = softmax(scale * q_i k_S^T), dP = dO_i v_S^T, delta = rowsum(P * dP)
+// (one value per query row; it equals rowsum(dO_i * o_i)) and dS = P * (dP - delta):
+//     dv_S += P^T dO_i,   dq_i = scale * dS k_S,   dk_S += scale * dS^T q_i.
+// P is recomputed from the forward's log-sum-exp (P = 2^(s * scale * log2 e -
+// lse * log2 e)), so no attention matrix is stored.
+//
+// delta is summed from the same float32 P and dP that form dS, not taken as
+// dO . o from the forward's output: o is bf16, and where a row's attention sits on
+// one key the true dq is close to zero while dO . (o_bf16 - o) is not, so that
+// shortcut leaves a relative error of order 10 % in such rows' dq.  Summing P * dP
+// keeps sum_j dS_ij = 0 to rounding, and the forward's o is not needed at all.
+//
+// Two launches:
+//   sweep_kernel<..., 0>  dq: one CTA per pair of query blocks, over the union of their kept key
+//                         blocks (the forward's lists), one key block per tile, in two sweeps:
+//                         the first sums delta, the second forms dS and dq; it also writes
+//                         (lse * log2 e, delta) of its rows to a tile-ordered stats array
+//   sweep_kernel<..., 1>  dk, dv: one CTA per pair of key blocks, over the union of the query
+//                         blocks that keep them (the transposed lists), one query block per tile
+// Both passes have one shape.  The CTA's own 128 rows X, X2 (dq: Q, dO; dk/dv: K, V) stay in
+// shared memory; per tile the 64 rows Y, Y2 of the other block (dq: K, V; dk/dv: Q, dO) arrive
+// through a ring, and
+//     A  = X . Y^T    [128 x 64]    (tcgen05 SS; dq: S, dk/dv: S^T)
+//     A2 = X2 . Y2^T  [128 x 64]    (tcgen05 SS; dq: dP, dk/dv: dP^T)
+// the softmax warps form P and dS from them in place in tensor memory (bf16 pairs), and
+//     dq pass:    acc0 += dS . Y            (dq; tcgen05 TS, Y = K read MN-major)
+//     dk/dv pass: acc0 += P^T . Y2          (dv; Y2 = dO)
+//                 acc1 += dS^T . Y          (dk; Y = Q)
+// A row (or column) whose block does not keep the tile's block gets P = dS = 0.
+//
+// ---- Forward with logit offsets (MODE 2)
+// AB-Attention's SIP ("AB-Attention accélère la génération vidéo…", section "Les trois
+// techniques", second technique) keeps a sampled set of key blocks and adds log(1/pi) to the
+// logits of each kept block, pi being its inclusion probability.  Here the offset is any
+// per-(query block, key block) value the caller supplies.  One CTA per pair of query blocks
+// (X = Q), the ring brings K and V (Y, Y2), two sweeps over the union: the first only forms
+// S = Q K^T and keeps each row's running max and sum of 2^(x - max), x = s * scale * log2 e +
+// offset * log2 e; the two column halves are merged into L = log2 of the row's normaliser; the
+// second sweep forms S again, P = 2^(x - L) (already normalised) as bf16 pairs in place, and
+//     acc0 += P . Y2                      (o; tcgen05 TS, V read MN-major)
+// so o needs no rescaling and comes out of tensor memory finished.  Three 128x64xD products per
+// tile against the two of pair_attn_kernel, for a kernel whose offsets cost nothing extra.
+//
+// TMEM (512 columns): acc0 at 0, acc1 at 128, two tile buffers at 256 and 384; in buffer b the
+// A product sits at +0 .. +63 and A2 at +64 .. +127.  Softmax warp (q, hc) reads columns
+// 32hc .. 32hc+31 of both and writes its 32 bf16 results of each, packed in pairs, back into
+// columns 32hc .. 32hc+15: inside the range it has itself read, so no other warp's input is
+// overwritten.  The TS product over K = 64 then takes, for its 16-wide step kk, columns
+// 32 * (kk >> 1) + 8 * (kk & 1) .. +7.
+//
+// Warp roles (320 threads):
+//   warps 0-7  softmax warps: warp w covers TMEM lanes (rows) 32*(w%4) .. +31 and tile columns
+//              32*(w/4) .. +31; then the epilogue of the same rows and half of the columns
+//   warp 8     TMEM owner and MMA issuer (whole warp, one elected lane issues)
+//   warp 9     TMA producer (lane 0): the own rows once, then the ring
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include "attn_pair.cuh"
+#include "ptx.cuh"
+#include "reorder.cuh"
+
+namespace dbst {
+
+constexpr int kSweepThreads = 320;
+constexpr int kSweepSlots = 3;
+
+struct SweepParams {
+  const int32_t* count;      // [BH*NB]: own block -> number of other blocks in its list
+  const int16_t* idx;        // [BH*NB*NB]: the lists, ascending
+  const float* lse;          // [BH*N] the forward's log-sum-exp, same layout as q (dq pass)
+  float2* stats;             // [BH*N] tile order: (lse * log2 e, delta); written by the dq pass
+  const float* offsets;      // MODE 2: [BH*NB*NB] natural-log offset of (query block, key block), or null
+  float* lse_out;            // MODE 2: [BH*N] log-sum-exp of the offset logits, same layout as q, or null
+  __nv_bfloat16* out0;       // dq pass: dq; dk/dv pass: dv; MODE 2: o
+  __nv_bfloat16* out1;       // dk/dv pass: dk
+  int NB, N;
+  int pair_stride;           // own blocks a and a + pair_stride share a CTA
+  int pairs_per_head;
+  float scale_log2;          // softmax scale * log2 e
+  float scale;               // softmax scale
+  TileGeo tg;                // token grid and tile shape (raster layout only)
+};
+
+struct SweepSmem {
+  static constexpr int kOwnX = 0;                         // X: D-halves x [128 rows x 128 B]
+  static constexpr int kOwnX2 = 32768;                    // X2, same layout
+  static constexpr int kRing = 65536;
+  static constexpr int kSlot = 33792;                     // Y: D-halves x [64 rows x 128 B]; Y2 at +16384;
+  static constexpr int kSlotY2 = 16384;                   //   64 float2 stats of Y's rows at +32768
+  static constexpr int kSlotStats = 32768;
+  static constexpr int kUnion = kRing + kSweepSlots * kSlot;   // int32 x 4096: j | inA<<16 | inB<<17
+  static constexpr int kWords = kUnion + 16384;           // u32 [2][128] bitmasks of the two lists
+  static constexpr int kScan = kWords + 1024;             // int [128] word offsets
+  static constexpr int kDelta = kScan + 512;              // float [2 quantities][2 column halves][128 rows]
+  static constexpr int kBars = kDelta + 2048;
+  static constexpr int kMisc = kBars + 256;
+  static constexpr int kBytes = kMisc + 64;
+};
+static_assert(SweepSmem::kSlot % 1024 == 0 && SweepSmem::kRing % 1024 == 0, "swizzled tiles need 1 KB alignment");
+
+enum {
+  BB_OWN = 0,
+  BB_RFULL = 1,                          // [kSweepSlots] ring slot loaded
+  BB_REMPTY = BB_RFULL + kSweepSlots,      // [kSweepSlots] ring slot's last reader (the TS products) done
+  BB_SFULL = BB_REMPTY + kSweepSlots,      // [2] A and A2 of tile t in buffer t&1 complete
+  BB_PFULL = BB_SFULL + 2,               // [2] 256 arrivals: P / dS of tile t written
+  BB_ACC = BB_PFULL + 2,                 // [2] TS products of tile t complete (buffer t&1 free)
+  BB_DRAIN = BB_ACC + 2,
+  BB_COUNT = BB_DRAIN + 1
+};
+static_assert(BB_COUNT * 8 <= 256, "barrier area");
+
+constexpr uint32_t kSweepAcc0 = 0, kSweepAcc1 = 128, kSweepBuf = 256;
+
+// 1-D bulk copy global -> shared, completing on `bar`; both addresses 16-byte aligned, bytes a
+// multiple of 16.
+__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+// bits_t[bh][j][w] bit i = bits[bh][32w + i][j / 32] bit (j % 32): key block j's row lists the
+// query blocks whose kept set contains j.
+__global__ void __launch_bounds__(256) transpose_bits_kernel(const uint32_t* __restrict__ bits,
+                                                             uint32_t* __restrict__ bits_t, int NB, int NW,
+                                                             long long words) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < words; e += stride) {
+    const long long bh = e / (static_cast<long long>(NB) * NW);
+    const int rem = static_cast<int>(e - bh * NB * NW);
+    const int j = rem / NW, w = rem % NW;
+    const uint32_t* head = bits + bh * NB * NW;
+    uint32_t word = 0u;
+    for (int i = 0; i < 32; ++i) {
+      const int qi = 32 * w + i;
+      if (qi >= NB) break;
+      word |= ((head[static_cast<long long>(qi) * NW + (j >> 5)] >> (j & 31)) & 1u) << i;
+    }
+    bits_t[e] = word;
+  }
+}
+
+// MODE 0: dq pass (X = Q, X2 = dO, Y = K, Y2 = V; lists = the forward's kept key blocks);
+//         virtual tiles v = 0 .. 2T-1 walk the union twice (tile v mod T).
+// MODE 1: dk/dv pass (X = K, X2 = V, Y = Q, Y2 = dO; lists = the transposed lists), T tiles.
+// MODE 2: forward with offsets (X = Q, Y = K, Y2 = V; the forward's lists), 2T virtual tiles; X2
+//         is not used, and the first sweep loads only Y.
+// RASTER: tensors in the caller's raster order, loaded with 5-D boxes (see pair_attn_kernel).
+template <int D, bool RASTER, int MODE>
+__global__ void __launch_bounds__(kSweepThreads, 1)
+    sweep_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmX2,
+               const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmY2,
+               const SweepParams prm) {
+  static_assert(D == 64 || D == 128, "head dim");
+  static_assert(MODE >= 0 && MODE <= 2, "mode");
+  constexpr bool DKDV = MODE == 1;
+  constexpr bool FWD = MODE == 2;
+  constexpr int DH = D / 64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(sm);
+  int32_t* s_union = reinterpret_cast<int32_t*>(sm + SweepSmem::kUnion);
+  uint32_t* s_words = reinterpret_cast<uint32_t*>(sm + SweepSmem::kWords);
+  int32_t* s_scan = reinterpret_cast<int32_t*>(sm + SweepSmem::kScan);
+  uint32_t* s_misc = reinterpret_cast<uint32_t*>(sm + SweepSmem::kMisc);
+  volatile uint32_t* s_abort = s_misc + 2;
+  auto bar = [&](int slot) -> uint32_t { return sbase + SweepSmem::kBars + 8u * slot; };
+  auto wait_live = [&](uint32_t mb, uint32_t parity, bool& live) {
+    if (!live || mbar_try(mb, parity)) return;
+    const long long t0 = clock64();
+    while (!mbar_try(mb, parity)) {
+      if (*s_abort) { live = false; return; }
+      if (clock64() - t0 > kWaitLimitCycles) {
+        record_error(kErrTimeout);
+        *s_abort = 1;
+        live = false;
+        return;
+      }
+    }
+  };
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int NB = prm.NB, NW = (NB + 31) >> 5;
+  const long long bh = blockIdx.x / prm.pairs_per_head;
+  const int pi = blockIdx.x - static_cast<int>(bh * prm.pairs_per_head);
+  const int ps = prm.pair_stride;
+  const int ba = (pi / ps) * 2 * ps + (pi % ps);
+  const int bb = ba + ps;
+  const bool has_b = bb < NB;
+  auto out_row = [&](int blk, int rr) -> long long {
+    if constexpr (RASTER) return bh * prm.N + tiled_to_raster(blk * 64 + rr, prm.tg);
+    else return bh * prm.N + static_cast<long long>(blk) * 64 + rr;
+  };
+  // TMA load of block blk's channels 64h .. 64h+63 (8 KB) into shared memory
+  auto load_block = [&](uint32_t dst, const CUtensorMap* map, uint32_t mbar, int blk, int h) {
+    if constexpr (RASTER) {
+      const int Tx = blk % prm.tg.nX, Ty = (blk / prm.tg.nX) % prm.tg.nY, Tt = blk / (prm.tg.nX * prm.tg.nY);
+      tma_load_5d(dst, map, mbar, 64 * h, Tx * prm.tg.tx, Ty * prm.tg.ty, Tt * prm.tg.tt, static_cast<int32_t>(bh));
+    } else {
+      tma_load_2d(dst, map, mbar, 64 * h, static_cast<int32_t>(bh * prm.N + static_cast<long long>(blk) * 64));
+    }
+  };
+
+  for (int w = tid; w < 2 * 128; w += kSweepThreads) s_words[w] = 0u;
+  if (tid == 0) {
+    for (int b = 0; b < BB_COUNT; ++b) mbar_init(bar(b), (b == BB_PFULL || b == BB_PFULL + 1) ? 256u : 1u);
+    fence_mbar_init();
+    for (int i = 1; i < 16; ++i) s_misc[i] = 0;
+  }
+  __syncthreads();
+  if (warp == 9 && lane == 0) {   // own rows: blocks ba (rows 0..63) and bb (rows 64..127; ba again if none)
+    tma_prefetch_desc(&tmX);
+    if constexpr (!FWD) tma_prefetch_desc(&tmX2);
+    mbar_expect_tx(bar(BB_OWN), (FWD ? 1 : 2) * 128 * D * 2);
+    for (int h = 0; h < DH; ++h) {
+      load_block(sbase + SweepSmem::kOwnX + h * 16384, &tmX, bar(BB_OWN), ba, h);
+      load_block(sbase + SweepSmem::kOwnX + h * 16384 + 8192, &tmX, bar(BB_OWN), has_b ? bb : ba, h);
+      if constexpr (!FWD) {
+        load_block(sbase + SweepSmem::kOwnX2 + h * 16384, &tmX2, bar(BB_OWN), ba, h);
+        load_block(sbase + SweepSmem::kOwnX2 + h * 16384 + 8192, &tmX2, bar(BB_OWN), has_b ? bb : ba, h);
+      }
+    }
+  }
+  if (warp == 8) {
+    tmem_alloc(sbase + SweepSmem::kMisc, 512);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  // ---- union of the two own blocks' lists -> ascending entries with membership flags
+  int n0 = prm.count[bh * NB + ba];
+  int n1 = has_b ? prm.count[bh * NB + bb] : 0;
+  if (n0 < 0 || n0 > NB || n1 < 0 || n1 > NB) {
+    if (tid == 0) record_error(kErrBounds);
+    n0 = min(max(n0, 0), NB);
+    n1 = min(max(n1, 0), NB);
+  }
+  const int16_t* g0 = prm.idx + (bh * NB + ba) * static_cast<long long>(NB);
+  const int16_t* g1 = prm.idx + (bh * NB + (has_b ? bb : ba)) * static_cast<long long>(NB);
+  for (int e = tid; e < n0 + n1; e += kSweepThreads) {
+    const int side = e >= n0;
+    const int j = static_cast<int>(side ? g1[e - n0] : g0[e]);
+    if (j < 0 || j >= NB) {
+      record_error(kErrBounds);
+      continue;
+    }
+    atomicOr(&s_words[side * 128 + (j >> 5)], 1u << (j & 31));
+  }
+  __syncthreads();
+  if (warp == 0) {   // exclusive scan of the union's popcounts over NW <= 128 words
+    int cnt[4], tot = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int w = 4 * lane + e;
+      cnt[e] = (w < NW) ? __popc(s_words[w] | s_words[128 + w]) : 0;
+      tot += cnt[e];
+    }
+    int incl = tot;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    int run = incl - tot;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      s_scan[4 * lane + e] = run;
+      run += cnt[e];
+    }
+    if (lane == 31) s_misc[1] = static_cast<uint32_t>(incl);
+  }
+  __syncthreads();
+  for (int w = tid; w < NW; w += kSweepThreads) {
+    const uint32_t wa = s_words[w], wb = s_words[128 + w];
+    uint32_t u = wa | wb;
+    int pos = s_scan[w];
+    while (u) {
+      const int b = __ffs(u) - 1;
+      u &= u - 1u;
+      s_union[pos++] = (32 * w + b) | (static_cast<int>((wa >> b) & 1u) << 16) | (static_cast<int>((wb >> b) & 1u) << 17);
+    }
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_misc[0];
+  const int T = static_cast<int>(s_misc[1]);
+  const int NV = DKDV ? T : 2 * T;       // virtual tiles
+  const int v_ts = DKDV ? 0 : T;         // first virtual tile with TS products
+  if (T == 0) {   // nothing in either list: zero gradients; MODE 2: o = 0 and lse = -inf
+    if (warp == 9 && lane == 0) mbar_wait(bar(BB_OWN), 0);
+    if (warp == 8) tmem_dealloc(tmem, 512);
+    for (int e = tid; e < 64 * D / 8; e += kSweepThreads) {
+      const int rr = e / (D / 8), c = e % (D / 8);
+      const uint4 z = make_uint4(0, 0, 0, 0);
+      reinterpret_cast<uint4*>(prm.out0 + out_row(ba, rr) * D)[c] = z;
+      if (has_b) reinterpret_cast<uint4*>(prm.out0 + out_row(bb, rr) * D)[c] = z;
+      if constexpr (DKDV) {
+        reinterpret_cast<uint4*>(prm.out1 + out_row(ba, rr) * D)[c] = z;
+        if (has_b) reinterpret_cast<uint4*>(prm.out1 + out_row(bb, rr) * D)[c] = z;
+      }
+    }
+    if constexpr (FWD) {
+      if (prm.lse_out && tid < 64) {
+        prm.lse_out[out_row(ba, tid)] = -INFINITY;
+        if (has_b) prm.lse_out[out_row(bb, tid)] = -INFINITY;
+      }
+    }
+    return;
+  }
+
+  if (warp == 9) {
+    // ------------------------------------------------------------ TMA producer of the ring
+    if (lane == 0) {
+      tma_prefetch_desc(&tmY);
+      tma_prefetch_desc(&tmY2);
+      int armed[kSweepSlots] = {0, 0, 0};
+      for (int t = 0; t < NV; ++t) {
+        if (*s_abort) break;
+        const int s = t % kSweepSlots;
+        if (t >= kSweepSlots && !mbar_wait(bar(BB_REMPTY + s), ((t / kSweepSlots) - 1) & 1)) {
+          *s_abort = 1;
+          break;
+        }
+        const int j = s_union[t < T ? t : t - T] & 0xFFFF;
+        const uint32_t dst = sbase + SweepSmem::kRing + s * SweepSmem::kSlot;
+        const bool withY2 = !(FWD && t < T);   // the offset forward's first sweep needs no values
+        mbar_expect_tx(bar(BB_RFULL + s), (withY2 ? 2 : 1) * 64 * D * 2 + (DKDV ? 512 : 0));
+        for (int h = 0; h < DH; ++h) {
+          load_block(dst + h * 8192, &tmY, bar(BB_RFULL + s), j, h);
+          if (withY2) load_block(dst + SweepSmem::kSlotY2 + h * 8192, &tmY2, bar(BB_RFULL + s), j, h);
+        }
+        if constexpr (DKDV)
+          bulk_load_1d(dst + SweepSmem::kSlotStats, prm.stats + bh * prm.N + static_cast<long long>(j) * 64, 512,
+                       bar(BB_RFULL + s));
+        armed[s] = t / kSweepSlots + 1;
+      }
+      // no copy may still be landing when the CTA exits
+      for (int s = 0; s < kSweepSlots; ++s)
+        if (armed[s] > 0) mbar_wait(bar(BB_RFULL + s), (armed[s] - 1) & 1);
+      mbar_wait(bar(BB_OWN), 0);
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer (whole warp)
+    constexpr uint32_t idSS = idesc_bf16(128, 64, 0, 0);   // A = own rows (K-major), B = ring rows (K-major)
+    constexpr uint32_t idTS = idesc_bf16(128, D, 0, 1);    // A = P or dS in TMEM, B = ring rows (MN-major)
+    const uint64_t dX = smem_desc(sbase + SweepSmem::kOwnX, 16, 1024);
+    const uint64_t dX2 = smem_desc(sbase + SweepSmem::kOwnX2, 16, 1024);
+    const uint64_t dRingK = smem_desc(sbase + SweepSmem::kRing, 16, 1024);
+    const uint64_t dRingMN = smem_desc(sbase + SweepSmem::kRing, 8192, 1024);
+    auto wait_all = [&](int slot, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar(slot), parity));
+    };
+    auto issue_ss = [&](int t) -> bool {
+      const int s = t % kSweepSlots, b = t & 1;
+      if (!wait_all(BB_RFULL + s, (t / kSweepSlots) & 1)) return false;
+      tc_fence_after();
+      const uint64_t y = dRingK + static_cast<uint64_t>((s * SweepSmem::kSlot) >> 4);
+      const uint64_t y2 = y + static_cast<uint64_t>(SweepSmem::kSlotY2 >> 4);
+      const uint32_t acc = tmem + kSweepBuf + 128u * b;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t oa = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+        const uint32_t ob = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
+        umma_f16_elect(acc, dX + oa, y + ob, idSS, kk > 0 ? 1u : 0u);
+        if constexpr (!FWD) umma_f16_elect(acc + 64u, dX2 + oa, y2 + ob, idSS, kk > 0 ? 1u : 0u);
+      }
+      umma_commit_elect(bar(BB_SFULL + b));
+      return true;
+    };
+    // Virtual tile u: once the softmax warps are done with buffer u&1, the TS products (second
+    // sweep of the dq pass, every tile of the dk/dv pass); the commits then also mark the buffer
+    // and the ring slot free in the first sweep, which has no TS products.
+    auto issue_ts = [&](int u) -> bool {
+      const int s = u % kSweepSlots, b = u & 1;
+      if (!wait_all(BB_PFULL + b, (u >> 1) & 1)) return false;
+      tc_fence_after();
+      const uint64_t y = dRingMN + static_cast<uint64_t>((s * SweepSmem::kSlot) >> 4);
+      const uint64_t y2 = y + static_cast<uint64_t>(SweepSmem::kSlotY2 >> 4);
+      const uint32_t buf = tmem + kSweepBuf + 128u * b;
+      if (u >= v_ts) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint32_t col = 32u * (kk >> 1) + 8u * (kk & 1);
+          const uint32_t accf = (u > v_ts || kk > 0) ? 1u : 0u;
+          if constexpr (DKDV) {
+            umma_ts_elect(tmem + kSweepAcc0, buf + col, y2 + kk * 128, idTS, accf);          // dv += P^T dO
+            umma_ts_elect(tmem + kSweepAcc1, buf + 64u + col, y + kk * 128, idTS, accf);     // dk += dS^T Q
+          } else if constexpr (FWD) {
+            umma_ts_elect(tmem + kSweepAcc0, buf + col, y2 + kk * 128, idTS, accf);          // o += P V
+          } else {
+            umma_ts_elect(tmem + kSweepAcc0, buf + 64u + col, y + kk * 128, idTS, accf);     // dq += dS K
+          }
+        }
+      }
+      umma_commit_elect(bar(BB_ACC + b));
+      umma_commit_elect(bar(BB_REMPTY + s));
+      return true;
+    };
+    bool ok = wait_all(BB_OWN, 0);
+    if (ok) ok = issue_ss(0);
+    if (ok && NV > 1) ok = issue_ss(1);
+    for (int u = 0; ok && u < NV; ++u) {
+      if (__any_sync(0xffffffffu, *s_abort != 0)) { ok = false; break; }
+      if (!issue_ts(u)) { ok = false; break; }
+      // buffer u&1 is rewritten by the products of tile u+2 only once the TS products of tile u,
+      // which read P and dS from it, have completed
+      if (u + 2 < NV) {
+        if (!wait_all(BB_ACC + (u & 1), (u >> 1) & 1) || !issue_ss(u + 2)) { ok = false; break; }
+      }
+    }
+    if (!ok && lane == 0) *s_abort = 1;
+    umma_commit_elect(bar(BB_DRAIN));
+    mbar_wait(bar(BB_DRAIN), 0);
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax warps 0-7
+    const int q = warp & 3;                   // TMEM lane quarter
+    const int hc = warp >> 2;                 // tile columns 32hc .. 32hc+31
+    const int r = 32 * q + lane;              // own row in the 128-row tile
+    const int side = r >> 6;                  // 0: block ba, 1: block bb (uniform per warp)
+    const uint32_t lrow = static_cast<uint32_t>(32 * q) << 16;
+    const float sc = prm.scale_log2;
+    float* s_delta = reinterpret_cast<float*>(sm + SweepSmem::kDelta);
+    if constexpr (FWD) {
+      // ---- forward with offsets: first sweep row max and sum, second sweep P = 2^(x - L) and o += P V
+      const int own = side ? bb : ba;
+      const float* offrow = prm.offsets ? prm.offsets + (bh * NB + own) * static_cast<long long>(NB) : nullptr;
+      float m = -INFINITY, l = 0.0f;          // first sweep, this warp's columns: running max of x, sum of 2^(x - m)
+      float L = -INFINITY;                    // log2 of the row's normaliser
+      bool live = true;
+      for (int v = 0; v < NV; ++v) {
+        const int b = v & 1;
+        const int t = v < T ? v : v - T;
+        wait_live(bar(BB_SFULL + b), (v >> 1) & 1, live);
+        tc_fence_after();
+        const int ent = s_union[t];
+        const bool vh = (ent >> (16 + side)) & 1;   // uniform per warp
+        const uint32_t buf = tmem + kSweepBuf + 128u * b + 32u * hc + lrow;
+        const float off = (vh && offrow != nullptr) ? offrow[ent & 0xFFFF] * 1.4426950408889634f : 0.0f;
+        if (v < T) {
+          if (vh) {
+            uint32_t sv[32];
+            tmem_ld32(buf, sv);
+            tmem_wait_ld();
+            float smax = __uint_as_float(sv[0]);
+#pragma unroll
+            for (int c = 1; c < 32; ++c) smax = fmaxf(smax, __uint_as_float(sv[c]));
+            const float mn = fmaxf(m, fmaf(smax, sc, off));   // finite: this tile is kept
+            float acc = 0.0f;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) acc += fast_exp2(fmaf(__uint_as_float(sv[c]), sc, off - mn));
+            l = fmaf(l, fast_exp2(m - mn), acc);               // m = -inf: 2^-inf = 0
+            m = mn;
+          }
+          tc_fence_before();
+          mbar_arrive(bar(BB_PFULL + b));
+          if (v == T - 1) {   // merge the two column halves of each row
+            s_delta[hc * 128 + r] = m;
+            s_delta[256 + hc * 128 + r] = l;
+            named_bar_sync(1u + static_cast<uint32_t>(q), 64);
+            const float m0 = s_delta[r], m1 = s_delta[128 + r];
+            const float M = fmaxf(m0, m1);
+            if (M != -INFINITY)
+              L = M + __log2f(s_delta[256 + r] * fast_exp2(m0 - M) + s_delta[384 + r] * fast_exp2(m1 - M));
+          }
+          continue;
+        }
+        uint32_t pp[16];
+        if (vh) {
+          uint32_t sv[32];
+          tmem_ld32(buf, sv);
+          tmem_wait_ld();
+          const float nb = off - L;
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            pp[c] = pack_bf16x2(fast_exp2(fmaf(__uint_as_float(sv[2 * c]), sc, nb)),
+                                fast_exp2(fmaf(__uint_as_float(sv[2 * c + 1]), sc, nb)));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) pp[c] = 0u;
+        }
+        tmem_st16(buf, pp);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(BB_PFULL + b));
+      }
+      // ---- epilogue: o is already normalised; this warp's rows, columns (D/2)hc .. +D/2
+      if (!mbar_wait(bar(BB_DRAIN), 0)) *s_abort = 1;   // every MMA of the CTA has completed
+      tc_fence_after();
+      if (side == 0 || has_b) {
+        const long long orow = out_row(own, r & 63);
+        uint4* dst = reinterpret_cast<uint4*>(prm.out0 + orow * D + (D / 2) * hc);
+#pragma unroll
+        for (int c0 = 0; c0 < D / 2; c0 += 32) {
+          uint32_t ov[32];
+          tmem_ld32(tmem + kSweepAcc0 + (D / 2) * hc + c0 + lrow, ov);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(__uint_as_float(ov[2 * c]), __uint_as_float(ov[2 * c + 1]));
+#pragma unroll
+          for (int u = 0; u < 4; ++u) dst[c0 / 8 + u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+        if (hc == 0 && prm.lse_out != nullptr)
+          prm.lse_out[orow] = (L == -INFINITY) ? -INFINITY : L * 0.69314718055994530942f;
+      }
+    } else {
+      float rowL = 0.0f, rowD = 0.0f;           // dq pass: this query row's (lse * log2 e, delta)
+      if constexpr (!DKDV) {
+        if (side == 0 || has_b) rowL = prm.lse[out_row(side ? bb : ba, r & 63)] * 1.4426950408889634f;
+      }
+      bool live = true;
+      float dsum = 0.0f;                        // dq pass, first sweep: sum of P * dP over this warp's columns
+      for (int v = 0; v < NV; ++v) {
+        const int b = v & 1, s = v % kSweepSlots;
+        const int t = v < T ? v : v - T;
+        wait_live(bar(BB_SFULL + b), (v >> 1) & 1, live);
+        // the ring slot cannot be refilled before this tile's TS products, which wait for this warp
+        if constexpr (DKDV) wait_live(bar(BB_RFULL + s), (v / kSweepSlots) & 1, live);
+        tc_fence_after();
+        const bool vh = (s_union[t] >> (16 + side)) & 1;   // uniform per warp
+        const uint32_t buf = tmem + kSweepBuf + 128u * b + 32u * hc + lrow;
+        if (v < v_ts) {   // dq pass, first sweep: delta only
+          if (vh) {
+            uint32_t sv[32], dv[32];
+            tmem_ld32(buf, sv);
+            tmem_ld32(buf + 64u, dv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              dsum = fmaf(fast_exp2(fmaf(__uint_as_float(sv[c]), sc, -rowL)), __uint_as_float(dv[c]), dsum);
+          }
+          tc_fence_before();
+          mbar_arrive(bar(BB_PFULL + b));
+          if (v == v_ts - 1) {   // combine the two column halves; publish (L, delta) for the dk/dv pass
+            s_delta[hc * 128 + r] = dsum;
+            named_bar_sync(1u + static_cast<uint32_t>(q), 64);
+            rowD = s_delta[r] + s_delta[128 + r];
+            if (hc == 0 && (side == 0 || has_b))
+              prm.stats[bh * prm.N + static_cast<long long>(side ? bb : ba) * 64 + (r & 63)] = make_float2(rowL, rowD);
+          }
+          continue;
+        }
+        uint32_t pp[16], pd[16];
+        if (vh) {
+          uint32_t sv[32], dv[32];
+          tmem_ld32(buf, sv);
+          tmem_ld32(buf + 64u, dv);
+          tmem_wait_ld();
+          if constexpr (DKDV) {
+            // column c of the tile is query row c of the ring block: (lse * log2 e, delta) per column
+            const float4* st4 = reinterpret_cast<const float4*>(sm + SweepSmem::kRing + s * SweepSmem::kSlot +
+                                                                SweepSmem::kSlotStats) + 16 * hc;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const float4 st = st4[c];
+              const float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * c]), sc, -st.x));
+              const float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * c + 1]), sc, -st.z));
+              const float d0 = p0 * (__uint_as_float(dv[2 * c]) - st.y);
+              const float d1 = p1 * (__uint_as_float(dv[2 * c + 1]) - st.w);
+              pp[c] = pack_bf16x2(p0, p1);
+              pd[c] = pack_bf16x2(d0, d1);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * c]), sc, -rowL));
+              const float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * c + 1]), sc, -rowL));
+              pd[c] = pack_bf16x2(p0 * (__uint_as_float(dv[2 * c]) - rowD), p1 * (__uint_as_float(dv[2 * c + 1]) - rowD));
+              pp[c] = 0u;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) pp[c] = pd[c] = 0u;
+        }
+        if constexpr (DKDV) tmem_st16(buf, pp);
+        tmem_st16(buf + 64u, pd);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(BB_PFULL + b));
+      }
+
+      // ---- epilogue: this warp's rows, columns (D/2)hc .. +D/2 of each accumulator, to bf16
+      if (!mbar_wait(bar(BB_DRAIN), 0)) *s_abort = 1;   // every MMA of the CTA has completed
+      tc_fence_after();
+      if (side == 0 || has_b) {
+        const long long orow = out_row(side ? bb : ba, r & 63);
+        auto store = [&](uint32_t acc, __nv_bfloat16* out, float f) {
+          uint4* dst = reinterpret_cast<uint4*>(out + orow * D + (D / 2) * hc);
+#pragma unroll
+          for (int c0 = 0; c0 < D / 2; c0 += 32) {
+            uint32_t ov[32];
+            tmem_ld32(tmem + acc + (D / 2) * hc + c0 + lrow, ov);
+            tmem_wait_ld();
+            uint32_t pk[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+              pk[c] = pack_bf16x2(__uint_as_float(ov[2 * c]) * f, __uint_as_float(ov[2 * c + 1]) * f);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[c0 / 8 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        };
+        if constexpr (DKDV) {
+          store(kSweepAcc0, prm.out0, 1.0f);        // dv
+          store(kSweepAcc1, prm.out1, prm.scale);   // dk
+        } else {
+          store(kSweepAcc0, prm.out0, prm.scale);   // dq
+        }
+      }
+      tc_fence_before();
+    }
+  }
+
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace dbst

@@ -11,12 +11,13 @@
 #include <mutex>
 
 #include "../../include/dbst.h"
-#include "attn_bwd.cuh"
+#include "attn_sweep.cuh"
 #include "attn_pair.cuh"
 #include "pairing.cuh"
 #include "mask.cuh"
 #include "ptx.cuh"
 #include "reorder.cuh"
+#include "sip.cuh"
 #include "squad.cuh"
 
 namespace {
@@ -239,7 +240,7 @@ dbst_status launch_bwd(const void* q, const void* k, const void* v, const float*
         !make_tmap(&tdo, dout, rows, D))
       return DBST_ECUDA;
   }
-  dbst::BwdParams p;
+  dbst::SweepParams p{};
   p.tg = tile_geo(g);
   p.lse = lse;
   p.stats = stats;
@@ -250,13 +251,13 @@ dbst_status launch_bwd(const void* q, const void* k, const void* v, const float*
   const float sc = scale > 0.0f ? scale : 1.0f / std::sqrt(static_cast<float>(D));
   p.scale = sc;
   p.scale_log2 = sc * 1.4426950408889634f;
-  const int smem = dbst::BwdSmem::kBytes + 1024;
+  const int smem = dbst::SweepSmem::kBytes + 1024;
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [&] {
-    attr = cudaFuncSetAttribute(dbst::bwd_kernel<D, RASTER, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    attr = cudaFuncSetAttribute(dbst::sweep_kernel<D, RASTER, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (attr == cudaSuccess)
-      attr = cudaFuncSetAttribute(dbst::bwd_kernel<D, RASTER, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      attr = cudaFuncSetAttribute(dbst::sweep_kernel<D, RASTER, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   });
   if (attr != cudaSuccess) return DBST_ECUDA;
   const long long grid = bh_count(g) * p.pairs_per_head;
@@ -265,13 +266,13 @@ dbst_status launch_bwd(const void* q, const void* k, const void* v, const float*
   p.idx = kv_idx;
   p.out0 = static_cast<__nv_bfloat16*>(dq);
   p.out1 = nullptr;
-  dbst::bwd_kernel<D, RASTER, false><<<static_cast<unsigned>(grid), dbst::kBwdThreads, smem, s>>>(tq, tdo, tk, tv, p);
+  dbst::sweep_kernel<D, RASTER, 0><<<static_cast<unsigned>(grid), dbst::kSweepThreads, smem, s>>>(tq, tdo, tk, tv, p);
   if (cudaGetLastError() != cudaSuccess) return DBST_ECUDA;
   p.count = q_count;
   p.idx = q_idx;
   p.out0 = static_cast<__nv_bfloat16*>(dv);
   p.out1 = static_cast<__nv_bfloat16*>(dk);
-  dbst::bwd_kernel<D, RASTER, true><<<static_cast<unsigned>(grid), dbst::kBwdThreads, smem, s>>>(tk, tv, tq, tdo, p);
+  dbst::sweep_kernel<D, RASTER, 1><<<static_cast<unsigned>(grid), dbst::kSweepThreads, smem, s>>>(tk, tv, tq, tdo, p);
   return launch_status();
 }
 
@@ -331,6 +332,63 @@ dbst_status window_transpose(const void* src, void* dst, long long heads, int A,
   return cudaGetLastError() == cudaSuccess ? DBST_OK : DBST_ECUDA;
 }
 
+// Forward with a logit offset per (query block, key block): the two-sweep kernel, MODE 2.
+template <int D, bool RASTER>
+dbst_status launch_offset_attn(const void* q, const void* k, const void* v, const dbst_geom* g, const int32_t* cnt,
+                               const int16_t* idx, const float* offsets, float scale, void* o, float* lse,
+                               cudaStream_t s) {
+  const long long rows = bh_count(g) * tokens(g);
+  CUtensorMap tq, tk, tv;
+  if (RASTER) {
+    if (!make_tmap_raster(&tq, q, g) || !make_tmap_raster(&tk, k, g) || !make_tmap_raster(&tv, v, g)) return DBST_ECUDA;
+  } else {
+    if (!make_tmap(&tq, q, rows, D) || !make_tmap(&tk, k, rows, D) || !make_tmap(&tv, v, rows, D)) return DBST_ECUDA;
+  }
+  dbst::SweepParams p{};
+  p.tg = tile_geo(g);
+  p.count = cnt;
+  p.idx = idx;
+  p.offsets = offsets;
+  p.lse_out = lse;
+  p.out0 = static_cast<__nv_bfloat16*>(o);
+  p.NB = nblocks(g);
+  p.N = static_cast<int>(tokens(g));
+  p.pair_stride = pair_stride(g);
+  p.pairs_per_head = ((p.NB + 2 * p.pair_stride - 1) / (2 * p.pair_stride)) * p.pair_stride;
+  const float sc = scale > 0.0f ? scale : 1.0f / std::sqrt(static_cast<float>(D));
+  p.scale = sc;
+  p.scale_log2 = sc * 1.4426950408889634f;
+  const int smem = dbst::SweepSmem::kBytes + 1024;
+  static std::once_flag once;
+  static cudaError_t attr = cudaSuccess;
+  std::call_once(once, [&] {
+    attr = cudaFuncSetAttribute(dbst::sweep_kernel<D, RASTER, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  if (attr != cudaSuccess) return DBST_ECUDA;
+  const long long grid = bh_count(g) * p.pairs_per_head;
+  if (grid >= (1ll << 31)) return DBST_EINVAL;
+  // the second tensor-map argument (X2) is not read in this mode
+  dbst::sweep_kernel<D, RASTER, 2><<<static_cast<unsigned>(grid), dbst::kSweepThreads, smem, s>>>(tq, tq, tk, tv, p);
+  return launch_status();
+}
+
+dbst_status offset_attn_common(const void* q, const void* k, const void* v, const dbst_geom* g, const int32_t* cnt,
+                               const int16_t* idx, const float* offsets, float scale, void* o, float* lse,
+                               void* stream, bool raster) {
+  if (!geom_ok(g) || !q || !k || !v || !o || !cnt || !idx) return DBST_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(cnt) || !aligned16(idx))
+    return DBST_EINVAL;
+  if ((lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) || (offsets && (reinterpret_cast<uintptr_t>(offsets) & 3u)))
+    return DBST_EINVAL;
+  if (!std::isfinite(scale)) return DBST_EINVAL;
+  auto s = static_cast<cudaStream_t>(stream);
+  if (raster)
+    return g->D == 128 ? launch_offset_attn<128, true>(q, k, v, g, cnt, idx, offsets, scale, o, lse, s)
+                       : launch_offset_attn<64, true>(q, k, v, g, cnt, idx, offsets, scale, o, lse, s);
+  return g->D == 128 ? launch_offset_attn<128, false>(q, k, v, g, cnt, idx, offsets, scale, o, lse, s)
+                     : launch_offset_attn<64, false>(q, k, v, g, cnt, idx, offsets, scale, o, lse, s);
+}
+
 template <int NPT>
 bool launch_select(const double* S, const dbst::SelectGeo& sg, long long rows, uint32_t* bits, int32_t* cnt,
                    int16_t* idx, cudaStream_t s) {
@@ -342,32 +400,23 @@ bool launch_select(const double* S, const dbst::SelectGeo& sg, long long rows, u
   return true;
 }
 
-// Mask build over tile-ordered (raster = false) or raster-ordered (raster = true) q and k.
-dbst_status build_mask(const void* q_tiled, const void* k_tiled, const dbst_geom* g, float p, int sta_radius,
-                       uint32_t* mask_bits, int32_t* kv_count, int16_t* kv_idx, void* workspace,
-                       size_t workspace_bytes, void* stream, bool raster) {
-  if (!geom_ok(g) || !q_tiled || !k_tiled || !mask_bits || !kv_count || !kv_idx || !workspace) return DBST_EINVAL;
-  if (!aligned16(q_tiled) || !aligned16(k_tiled) || !aligned16(mask_bits) || !aligned16(kv_count) ||
-      !aligned16(kv_idx) || !aligned16(workspace))
-    return DBST_EINVAL;
-  if (!(p > 0.0f && p <= 1.0f)) return DBST_EINVAL;   // also rejects NaN
-  const MaskWorkspace w = mask_workspace(g);
-  if (workspace_bytes < w.total) return DBST_EINVAL;
-  auto s = static_cast<cudaStream_t>(stream);
-  char* ws = static_cast<char*>(workspace);
+// Steps 1-2 of both mask builders: block means of q and k (tile-ordered or, with `raster`,
+// raster-ordered), then the float64 pooled logits S[b,h,i,j] = <qp_i, kp_j> / sqrt(D), into the
+// workspace.  The caller has validated the arguments (including B*H <= 65535).
+dbst_status pool_and_logits(const void* q, const void* k, const dbst_geom* g, const MaskWorkspace& w, char* ws,
+                            cudaStream_t s, bool raster) {
   double* qp = reinterpret_cast<double*>(ws + w.qp);
   double* kp = reinterpret_cast<double*>(ws + w.kp);
   double* S = reinterpret_cast<double*>(ws + w.s);
   const int NB = nblocks(g);
   const long long bh = bh_count(g);
   const long long nblk = bh * NB;
-
   {  // 1. block mean-pool of q and k
     long long grid = (2 * nblk * 32 + 255) / 256;
     const long long cap = static_cast<long long>(sm_count()) * 8;
     if (grid > cap) grid = cap;
-    const auto* qa = static_cast<const uint4*>(q_tiled);
-    const auto* ka = static_cast<const uint4*>(k_tiled);
+    const auto* qa = static_cast<const uint4*>(q);
+    const auto* ka = static_cast<const uint4*>(k);
     const unsigned gr = static_cast<unsigned>(grid);
     const dbst::TileGeo tg = tile_geo(g);
     if (g->D == 128) {
@@ -382,13 +431,34 @@ dbst_status build_mask(const void* q_tiled, const void* k_tiled, const dbst_geom
   {  // 2. pooled logits (float64)
     const double scale = 1.0 / std::sqrt(static_cast<double>(g->D));
     dim3 grid((NB + 63) / 64, (NB + 63) / 64, static_cast<unsigned>(bh));
-    if (bh > 65535) return DBST_EINVAL;
     if (g->D == 128)
       dbst::pooled_logits_kernel<128><<<grid, 256, 0, s>>>(qp, kp, S, NB, scale);
     else
       dbst::pooled_logits_kernel<64><<<grid, 256, 0, s>>>(qp, kp, S, NB, scale);
     if (cudaGetLastError() != cudaSuccess) return DBST_ECUDA;
   }
+  return DBST_OK;
+}
+
+// Mask build over tile-ordered (raster = false) or raster-ordered (raster = true) q and k.
+dbst_status build_mask(const void* q_tiled, const void* k_tiled, const dbst_geom* g, float p, int sta_radius,
+                       uint32_t* mask_bits, int32_t* kv_count, int16_t* kv_idx, void* workspace,
+                       size_t workspace_bytes, void* stream, bool raster) {
+  if (!geom_ok(g) || !q_tiled || !k_tiled || !mask_bits || !kv_count || !kv_idx || !workspace) return DBST_EINVAL;
+  if (!aligned16(q_tiled) || !aligned16(k_tiled) || !aligned16(mask_bits) || !aligned16(kv_count) ||
+      !aligned16(kv_idx) || !aligned16(workspace))
+    return DBST_EINVAL;
+  if (!(p > 0.0f && p <= 1.0f)) return DBST_EINVAL;   // also rejects NaN
+  const MaskWorkspace w = mask_workspace(g);
+  if (workspace_bytes < w.total) return DBST_EINVAL;
+  if (bh_count(g) > 65535) return DBST_EINVAL;        // grid.z of the pooled-logits launch
+  auto s = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  double* S = reinterpret_cast<double*>(ws + w.s);
+  const int NB = nblocks(g);
+  const long long nblk = bh_count(g) * NB;
+  const dbst_status st = pool_and_logits(q_tiled, k_tiled, g, w, ws, s, raster);
+  if (st != DBST_OK) return st;
   {  // 3. softmax + CDF selection + sliding-tile union + lists
     dbst::SelectGeo sg;
     sg.NB = NB;
@@ -410,6 +480,34 @@ dbst_status build_mask(const void* q_tiled, const void* k_tiled, const dbst_geom
     else ok = launch_select<16>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
     if (!ok) return DBST_ECUDA;
   }
+  return launch_status();
+}
+
+// SIP mask: pooled logits as for the CDF mask, then the sampled selection with offsets.
+dbst_status build_sip_mask(const void* q, const void* k, const dbst_geom* g, double budget, const double* uniforms,
+                           uint32_t* mask_bits, int32_t* kv_count, int16_t* kv_idx, float* offsets, void* workspace,
+                           size_t workspace_bytes, void* stream, bool raster) {
+  if (!geom_ok(g) || !q || !k || !uniforms || !mask_bits || !kv_count || !kv_idx || !offsets || !workspace)
+    return DBST_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(uniforms) || !aligned16(mask_bits) || !aligned16(kv_count) ||
+      !aligned16(kv_idx) || !aligned16(offsets) || !aligned16(workspace))
+    return DBST_EINVAL;
+  if (!(budget > 0.0) || !std::isfinite(budget)) return DBST_EINVAL;
+  const MaskWorkspace w = mask_workspace(g);
+  if (workspace_bytes < w.total) return DBST_EINVAL;
+  if (bh_count(g) > 65535) return DBST_EINVAL;
+  auto s = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  const dbst_status st = pool_and_logits(q, k, g, w, ws, s, raster);
+  if (st != DBST_OK) return st;
+  const int NB = nblocks(g);
+  const long long rows = bh_count(g) * NB;
+  long long grid = (rows + dbst::kSipWarps - 1) / dbst::kSipWarps;
+  const long long cap = static_cast<long long>(sm_count()) * 16;
+  if (grid > cap) grid = cap;
+  dbst::sip_select_kernel<<<static_cast<unsigned>(grid), 32 * dbst::kSipWarps, 0, s>>>(
+      reinterpret_cast<const double*>(ws + w.s), NB, (NB + 31) / 32, rows, budget, uniforms, mask_bits, kv_count,
+      kv_idx, offsets);
   return launch_status();
 }
 
@@ -556,6 +654,34 @@ dbst_status dbst_block_sparse_attn_backward_raster(const void* q, const void* k,
                                                    size_t workspace_bytes, void* stream) {
   return bwd_common(q, k, v, lse, d_o, g, kv_count, kv_idx, q_count, q_idx, scale, dq, dk, dv, workspace,
                     workspace_bytes, stream, true);
+}
+
+dbst_status dbst_build_sip_mask(const void* q_tiled, const void* k_tiled, const dbst_geom* g, double budget,
+                                const double* uniforms, uint32_t* mask_bits, int32_t* kv_count, int16_t* kv_idx,
+                                float* offsets, void* workspace, size_t workspace_bytes, void* stream) {
+  return build_sip_mask(q_tiled, k_tiled, g, budget, uniforms, mask_bits, kv_count, kv_idx, offsets, workspace,
+                        workspace_bytes, stream, false);
+}
+
+dbst_status dbst_build_sip_mask_raster(const void* q, const void* k, const dbst_geom* g, double budget,
+                                       const double* uniforms, uint32_t* mask_bits, int32_t* kv_count,
+                                       int16_t* kv_idx, float* offsets, void* workspace, size_t workspace_bytes,
+                                       void* stream) {
+  return build_sip_mask(q, k, g, budget, uniforms, mask_bits, kv_count, kv_idx, offsets, workspace,
+                        workspace_bytes, stream, true);
+}
+
+dbst_status dbst_block_sparse_attn_offsets(const void* q, const void* k, const void* v, const dbst_geom* g,
+                                           const int32_t* kv_count, const int16_t* kv_idx, const float* offsets,
+                                           float scale, void* o, float* lse, void* stream) {
+  return offset_attn_common(q, k, v, g, kv_count, kv_idx, offsets, scale, o, lse, stream, false);
+}
+
+dbst_status dbst_block_sparse_attn_offsets_raster(const void* q, const void* k, const void* v, const dbst_geom* g,
+                                                  const int32_t* kv_count, const int16_t* kv_idx,
+                                                  const float* offsets, float scale, void* o, float* lse,
+                                                  void* stream) {
+  return offset_attn_common(q, k, v, g, kv_count, kv_idx, offsets, scale, o, lse, stream, true);
 }
 
 size_t dbst_squad_workspace_bytes(int B, int H, int N, int D, int w) {

@@ -262,6 +262,56 @@ dbst_status dbst_block_sparse_attn_backward_raster(const void* q, const void* k,
                                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Sampled block mask with inclusion-probability weights: SIP on the page
+ * "AB-Attention accélère la génération vidéo jusqu'à 2,23× en sautant 92% de
+ * l'attention", section "Les trois techniques".  The scores of query block i
+ * are its row of the NABLA pooled map (softmax over key blocks of the pooled
+ * logits, computed as in dbst_build_block_mask).  Then
+ *   pi_ij  = min(1, c_i a_ij), c_i such that sum_j pi_ij = budget; blocks with
+ *            c_i a_ij >= 1 are fixed at 1 and c_i is recomputed over the rest
+ *            until none joins them; if budget covers every block with a_ij > 0,
+ *            all of those get pi = 1
+ *   keep   = uniforms[b,h,i,j] < pi_ij
+ *   offsets[b,h,i,j] = log(1 / pi_ij) for kept blocks, 0 elsewhere
+ * and the bitmask and lists of the kept blocks as dbst_build_block_mask writes
+ * them.  Pass offsets to dbst_block_sparse_attn_offsets.
+ *   budget   : expected kept blocks per row, > 0 (float64)
+ *   uniforms : [B,H,NB,NB] float64 in [0, 1), the caller's random draws
+ *   offsets  : out, [B,H,NB,NB] float32
+ *   workspace: dbst_mask_workspace_bytes(g) bytes
+ * q_tiled, k_tiled as for dbst_build_block_mask (the _raster form takes raster
+ * q, k like dbst_build_block_mask_raster).
+ */
+dbst_status dbst_build_sip_mask(const void* q_tiled, const void* k_tiled, const dbst_geom* g, double budget,
+                                const double* uniforms, uint32_t* mask_bits, int32_t* kv_count, int16_t* kv_idx,
+                                float* offsets, void* workspace, size_t workspace_bytes, void* stream);
+dbst_status dbst_build_sip_mask_raster(const void* q, const void* k, const dbst_geom* g, double budget,
+                                       const double* uniforms, uint32_t* mask_bits, int32_t* kv_count,
+                                       int16_t* kv_idx, float* offsets, void* workspace, size_t workspace_bytes,
+                                       void* stream);
+
+/*
+ * Block-sparse attention with a logit offset per (query block, key block), as
+ * SIP needs it (AB-Attention page, section "Les trois techniques"): for query
+ * block i with kept key blocks S_i and every query token n of block i,
+ *   o[n]   = sum_{m in tokens(S_i)} softmax_m(scale <q_n, k_m> + off[i, block(m)]) v[m]
+ *   lse[n] = log sum_{m in tokens(S_i)} exp(scale <q_n, k_m> + off[i, block(m)])
+ * offsets is [B,H,NB,NB] float32 (natural log; read only at kept blocks) or
+ * NULL for none.  The kernel walks the kept blocks twice (row statistics, then
+ * normalised P times V), so it forms S three times per two products of
+ * dbst_block_sparse_attn.  An empty row gives o = 0, lse = -inf.  Other
+ * arguments as for dbst_block_sparse_attn (the _raster form: raster q, k, v, o,
+ * lse); lse may be NULL.
+ */
+dbst_status dbst_block_sparse_attn_offsets(const void* q, const void* k, const void* v, const dbst_geom* g,
+                                           const int32_t* kv_count, const int16_t* kv_idx, const float* offsets,
+                                           float scale, void* o, float* lse, void* stream);
+dbst_status dbst_block_sparse_attn_offsets_raster(const void* q, const void* k, const void* v, const dbst_geom* g,
+                                                  const int32_t* kv_count, const int16_t* kv_idx,
+                                                  const float* offsets, float scale, void* o, float* lse,
+                                                  void* stream);
+
+/*
  * SQuad two-pass attention (page "SQuad: Sub-Quadratic Attention Distillation
  * for Efficient Video Generation", section "Methodology: SQuad", item
  * "1. SQuad-Attention Operator").  The N tokens of each (b, h) are read as

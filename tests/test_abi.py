@@ -178,3 +178,37 @@ def test_squad_entry_point_validates_shapes(lib):
     assert lib.dbst_squad_attn(None, a, a, *ok, 0.0, a, a, 4 * tb, None) == dbst.DBST_EINVAL
     assert lib.dbst_squad_attn(a, a, ctypes.c_void_p((1 << 20) + 8), *ok, 0.0, a, a, 4 * tb, None) == dbst.DBST_EINVAL
     assert lib.dbst_squad_attn(a, a, a, *ok, float("nan"), a, a, 4 * tb, None) == dbst.DBST_EINVAL
+
+
+def test_sip_and_offset_entry_points_validate_arguments(lib):
+    g = geom()
+    a = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    ws = lib.dbst_mask_workspace_bytes(ctypes.byref(g))
+    for fn in (lib.dbst_build_sip_mask, lib.dbst_build_sip_mask_raster):
+        ok = [a, a, ctypes.byref(g), 4.0, a, a, a, a, a, a, ws, None]
+        for i in (0, 1, 4, 5, 6, 7, 8, 9):
+            args = list(ok)
+            args[i] = None
+            assert fn(*args) == dbst.DBST_EINVAL, i
+            args[i] = odd
+            assert fn(*args) == dbst.DBST_EINVAL, i
+        for budget in (0.0, -1.0, float("nan"), float("inf")):
+            args = list(ok)
+            args[3] = budget
+            assert fn(*args) == dbst.DBST_EINVAL, budget
+        args = list(ok)
+        args[10] = ws - 1
+        assert fn(*args) == dbst.DBST_EINVAL
+    for fn in (lib.dbst_block_sparse_attn_offsets, lib.dbst_block_sparse_attn_offsets_raster):
+        ok = [a, a, a, ctypes.byref(g), a, a, None, 0.0, a, None, None]
+        for i in (0, 1, 2, 4, 5, 8):
+            args = list(ok)
+            args[i] = None
+            assert fn(*args) == dbst.DBST_EINVAL, i
+        args = list(ok)
+        args[6] = ctypes.c_void_p((1 << 20) + 2)                       # offsets not 4-byte aligned
+        assert fn(*args) == dbst.DBST_EINVAL
+        args = list(ok)
+        args[7] = float("nan")
+        assert fn(*args) == dbst.DBST_EINVAL
