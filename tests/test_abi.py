@@ -212,3 +212,15 @@ def test_sip_and_offset_entry_points_validate_arguments(lib):
         args = list(ok)
         args[7] = float("nan")
         assert fn(*args) == dbst.DBST_EINVAL
+
+
+def test_mask_builders_reject_too_many_heads_before_any_launch(lib):
+    """B*H above the pooled-logits grid limit is refused before anything is enqueued (the
+    refusal must not depend on a launch failing)."""
+    g = geom(B=1, H=70000, D=64, grid=(1, 8, 8), tile=(1, 8, 8))
+    a = ctypes.c_void_p(1 << 20)
+    ws = lib.dbst_mask_workspace_bytes(ctypes.byref(g))
+    assert ws > 0
+    assert lib.dbst_build_block_mask(a, a, ctypes.byref(g), 0.9, -1, a, a, a, a, ws, None) == dbst.DBST_EINVAL
+    assert lib.dbst_build_block_mask_raster(a, a, ctypes.byref(g), 0.9, -1, a, a, a, a, ws, None) == dbst.DBST_EINVAL
+    assert lib.dbst_build_sip_mask(a, a, ctypes.byref(g), 2.0, a, a, a, a, a, a, ws, None) == dbst.DBST_EINVAL
