@@ -21,7 +21,17 @@ def _cuda_available() -> bool:
         return False
 
 
+# Tests of the rows built on top of the core path (backward at full size, SIP, SQuad) run after
+# every test of the core path, so that a run stopping at the first failure (-x) never leaves a
+# core result unreported because of them.
+EXTENSION_MODULES = ("test_gpu_sip", "test_gpu_squad", "test_gpu_wan_backward")
+
+
 def pytest_collection_modifyitems(config, items):
+    def is_extension(item):
+        return item.module.__name__.rsplit(".", 1)[-1] in EXTENSION_MODULES
+
+    items[:] = [i for i in items if not is_extension(i)] + [i for i in items if is_extension(i)]
     if _cuda_available():
         return
     skip = pytest.mark.skip(reason="no CUDA device")

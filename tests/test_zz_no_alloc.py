@@ -9,8 +9,9 @@ point's output exactly, on two calls in a row (the second call reuses the
 scratch the first one left behind), and that a shape too large for the
 static scratch is refused before anything runs.
 
-Kept in a file of its own that sorts last, so that a run which stops at the
-first failure has already run every other test.
+Kept in a file of its own that sorts last among the core path's tests, so that
+a run which stops at the first failure has already run every other core test
+(tests/conftest.py runs the extension rows' tests after it).
 """
 import ctypes
 
