@@ -48,11 +48,14 @@
 // per-(query block, key block) value the caller supplies.  One CTA per pair of query blocks
 // (X = Q), the ring brings K and V (Y, Y2), two sweeps over the union: the first only forms
 // S = Q K^T and keeps each row's running max and sum of 2^(x - max), x = s * scale * log2 e +
-// offset * log2 e; the two column halves are merged into L = log2 of the row's normaliser; the
-// second sweep forms S again, P = 2^(x - L) (already normalised) as bf16 pairs in place, and
+// offset * log2 e; the two column halves are merged into the row max M and L = log2 of the
+// row's normaliser; the second sweep forms S again, P = 2^(x - M) as bf16 pairs in place, and
 //     acc0 += P . Y2                      (o; tcgen05 TS, V read MN-major)
-// so o needs no rescaling and comes out of tensor memory finished.  Three 128x64xD products per
-// tile against the two of pair_attn_kernel, for a kernel whose offsets cost nothing extra.
+// and the epilogue scales o by 2^(M - L).  Relative to the final max, the largest weight of a
+// row is exactly 1 in bf16 (as in pair_attn_kernel); normalising before the rounding instead
+// costs about 0.006 of max-abs error where a row sits on one key.  No rescaling of o between
+// tiles is needed.  Three 128x64xD products per tile against the two of pair_attn_kernel, for a
+// kernel whose offsets cost nothing extra.
 //
 // TMEM (512 columns): acc0 at 0, acc1 at 128, two tile buffers at 256 and 384; in buffer b the
 // A product sits at +0 .. +63 and A2 at +64 .. +127.  Softmax warp (q, hc) reads columns
@@ -436,11 +439,11 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
     const float sc = prm.scale_log2;
     float* s_delta = reinterpret_cast<float*>(sm + SweepSmem::kDelta);
     if constexpr (FWD) {
-      // ---- forward with offsets: first sweep row max and sum, second sweep P = 2^(x - L) and o += P V
+      // ---- forward with offsets: first sweep row max and sum, second sweep P = 2^(x - M) and o += P V
       const int own = side ? bb : ba;
       const float* offrow = prm.offsets ? prm.offsets + (bh * NB + own) * static_cast<long long>(NB) : nullptr;
       float m = -INFINITY, l = 0.0f;          // first sweep, this warp's columns: running max of x, sum of 2^(x - m)
-      float L = -INFINITY;                    // log2 of the row's normaliser
+      float M = -INFINITY, L = -INFINITY;     // the row's max of x and log2 of its normaliser
       bool live = true;
       for (int v = 0; v < NV; ++v) {
         const int b = v & 1;
@@ -473,7 +476,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             s_delta[256 + hc * 128 + r] = l;
             named_bar_sync(1u + static_cast<uint32_t>(q), 64);
             const float m0 = s_delta[r], m1 = s_delta[128 + r];
-            const float M = fmaxf(m0, m1);
+            M = fmaxf(m0, m1);
             if (M != -INFINITY)
               L = M + __log2f(s_delta[256 + r] * fast_exp2(m0 - M) + s_delta[384 + r] * fast_exp2(m1 - M));
           }
@@ -484,7 +487,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
           uint32_t sv[32];
           tmem_ld32(buf, sv);
           tmem_wait_ld();
-          const float nb = off - L;
+          const float nb = off - M;
 #pragma unroll
           for (int c = 0; c < 16; ++c)
             pp[c] = pack_bf16x2(fast_exp2(fmaf(__uint_as_float(sv[2 * c]), sc, nb)),
@@ -498,11 +501,12 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
         tc_fence_before();
         mbar_arrive(bar(BB_PFULL + b));
       }
-      // ---- epilogue: o is already normalised; this warp's rows, columns (D/2)hc .. +D/2
+      // ---- epilogue: o = acc * 2^(M - L); this warp's rows, columns (D/2)hc .. +D/2
       if (!mbar_wait(bar(BB_DRAIN), 0)) *s_abort = 1;   // every MMA of the CTA has completed
       tc_fence_after();
       if (side == 0 || has_b) {
         const long long orow = out_row(own, r & 63);
+        const float f = (L == -INFINITY) ? 0.0f : fast_exp2(M - L);
         uint4* dst = reinterpret_cast<uint4*>(prm.out0 + orow * D + (D / 2) * hc);
 #pragma unroll
         for (int c0 = 0; c0 < D / 2; c0 += 32) {
@@ -511,7 +515,8 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
           tmem_wait_ld();
           uint32_t pk[16];
 #pragma unroll
-          for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(__uint_as_float(ov[2 * c]), __uint_as_float(ov[2 * c + 1]));
+          for (int c = 0; c < 16; ++c)
+            pk[c] = pack_bf16x2(__uint_as_float(ov[2 * c]) * f, __uint_as_float(ov[2 * c + 1]) * f);
 #pragma unroll
           for (int u = 0; u < 4; ++u) dst[c0 / 8 + u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         }
