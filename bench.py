@@ -239,6 +239,25 @@ def run_reference(args, w, p):
     return 0
 
 
+def timed_median(fn, steps: int, warmup: int) -> float:
+    """Median CUDA-event time (ms) of fn() on the current stream over `steps` calls, after
+    max(warmup, 3) untimed calls."""
+    import torch
+    for _ in range(max(warmup, 3)):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(steps):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
 def run_sweep(args, w):
     """Attention time and kept-block TFLOP/s against the kept fraction; dense attention at the same shape."""
     import torch
@@ -251,19 +270,7 @@ def run_sweep(args, w):
     lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device="cuda")
 
     def timed(fn, reps):
-        for _ in range(3):
-            fn()
-        torch.cuda.synchronize()
-        ts = []
-        for _ in range(reps):
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record()
-            fn()
-            b.record()
-            torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b))
-        return statistics.median(ts)
+        return timed_median(fn, reps, 3)
 
     dense_ms = timed(lambda: dbst.dense_attn(qt, kt, vt, g), args.steps)
     dense_flops = 4.0 * w.D * w.N * w.N * w.B * w.H
@@ -293,15 +300,15 @@ def run_sweep(args, w):
     return 0
 
 
-def run_backward(args, w, p):
+def measure_backward(args, w, p, qkv=None) -> dict:
     """Backward of the block-sparse attention (raster layout) on one GPU: mask, its transpose, forward
-    for the log-sum-exp, then the timed backward.  One JSON line, not the headline metric."""
+    for the log-sum-exp, then the timed backward."""
     import torch
     import dynamic_block_sparse_tile_b200 as dbst
     dbst.load()
     g = dbst.Geom.make(w.B, w.H, w.D, w.grid, w.tile)
     to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()   # noqa: E731
-    q, k, v = (to_dev(a) for a in S.make_qkv(w))
+    q, k, v = qkv if qkv is not None else (to_dev(a) for a in S.make_qkv(w))
     do = to_dev(S.make_grad(w))
     bits, cnt, idx = dbst.build_block_mask_raster(q, k, g, p, w.sta_radius)
     pairs = dbst.pair_query_blocks(bits, g)
@@ -310,51 +317,41 @@ def run_backward(args, w, p):
     _, qcnt, qidx = out_t
     ws = torch.empty(dbst.attn_backward_workspace_bytes(g), dtype=torch.uint8, device="cuda")
     grads = tuple(torch.empty_like(q) for _ in range(3))
-
-    def timed(fn):
-        for _ in range(max(args.warmup, 3)):
-            fn()
-        torch.cuda.synchronize()
-        ts = []
-        for _ in range(args.steps):
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record()
-            fn()
-            b.record()
-            torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b))
-        return statistics.median(ts)
-
-    fwd_ms = timed(lambda: dbst.block_sparse_attn_raster(q, k, v, g, cnt, idx, 0.0, True, o, lse, pairs))
-    tr_ms = timed(lambda: dbst.transpose_block_mask(bits, g, out=out_t))
-    bwd_ms = timed(lambda: dbst.block_sparse_attn_backward(q, k, v, lse, do, g, cnt, idx, qcnt, qidx, raster=True,
-                                                           workspace=ws, out=grads))
+    fwd_ms = timed_median(lambda: dbst.block_sparse_attn_raster(q, k, v, g, cnt, idx, 0.0, True, o, lse, pairs),
+                          args.steps, args.warmup)
+    tr_ms = timed_median(lambda: dbst.transpose_block_mask(bits, g, out=out_t), args.steps, args.warmup)
+    bwd_ms = timed_median(lambda: dbst.block_sparse_attn_backward(q, k, v, lse, do, g, cnt, idx, qcnt, qidx,
+                                                                  raster=True, workspace=ws, out=grads),
+                          args.steps, args.warmup)
     dbst.get_error()
     kept = int(cnt.sum().item())
     unit = 2.0 * w.D * 64 * 64 * kept            # one 64x64xD product over every kept block pair
     _, bf16, _, src = peaks()
-    out = {"backward": workload_desc(w, p), "kept_fraction": kept / (g.B * g.H * g.NB * g.NB),
-           "backward_ms": bwd_ms, "forward_attn_ms": fwd_ms, "transpose_ms": tr_ms,
-           "backward_tflops": 5 * unit / (bwd_ms * 1e-3) / 1e12,
-           "backward_tensor_tflops": 9 * unit / (bwd_ms * 1e-3) / 1e12,
-           "forward_tflops": 2 * unit / (fwd_ms * 1e-3) / 1e12,
-           "bf16_peak_tflops": bf16, "peak_source": src,
-           "note": "backward_tflops counts the 5 products of the gradient (S, dP, dV, dK, dQ); the kernels "
-                   "run 9 (S and dP twice more: the delta sweep of the dq pass and the dk/dv pass)"}
-    print(json.dumps(out), flush=True)
+    return {"backward": workload_desc(w, p), "kept_fraction": kept / (g.B * g.H * g.NB * g.NB),
+            "backward_ms": bwd_ms, "forward_attn_ms": fwd_ms, "transpose_ms": tr_ms,
+            "backward_tflops": 5 * unit / (bwd_ms * 1e-3) / 1e12,
+            "backward_tensor_tflops": 9 * unit / (bwd_ms * 1e-3) / 1e12,
+            "forward_tflops": 2 * unit / (fwd_ms * 1e-3) / 1e12,
+            "bf16_peak_tflops": bf16, "peak_source": src,
+            "note": "backward_tflops counts the 5 products of the gradient (S, dP, dV, dK, dQ); the kernels "
+                    "run 9 (S and dP twice more: the delta sweep of the dq pass and the dk/dv pass)"}
+
+
+def run_backward(args, w, p):
+    print(json.dumps(measure_backward(args, w, p)), flush=True)
     return 0
 
 
-def run_sip(args, w, p):
-    """SIP on the Wan-like workload: sampled mask with inclusion-probability offsets at the
-    NABLA mask's mean kept count per row, then the offset attention; plus that attention
-    without offsets on the NABLA mask.  One JSON line; not the headline metric."""
+def measure_sip(args, w, p, qkv=None) -> dict:
+    """SIP on one workload: sampled mask with inclusion-probability offsets at the NABLA mask's mean
+    kept count per row, then the offset attention; plus that attention without offsets on the
+    NABLA mask."""
     import torch
     import dynamic_block_sparse_tile_b200 as dbst
     dbst.load()
     g = dbst.Geom.make(w.B, w.H, w.D, w.grid, w.tile)
-    q, k, v = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda() for a in S.make_qkv(w))
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()   # noqa: E731
+    q, k, v = qkv if qkv is not None else (to_dev(a) for a in S.make_qkv(w))
     bits, cnt, idx = dbst.build_block_mask_raster(q, k, g, p, w.sta_radius)
     budget = float(cnt.double().mean().item())
     gen = torch.Generator(device="cuda").manual_seed(1234)
@@ -363,43 +360,32 @@ def run_sip(args, w, p):
     sip = dbst.build_sip_mask(q, k, g, budget, u, raster=True, workspace=ws)
     o = torch.empty_like(q)
     lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device="cuda")
-
-    def timed(fn):
-        for _ in range(max(args.warmup, 3)):
-            fn()
-        torch.cuda.synchronize()
-        ts = []
-        for _ in range(args.steps):
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record()
-            fn()
-            b.record()
-            torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b))
-        return statistics.median(ts)
-
-    sel_ms = timed(lambda: dbst.build_sip_mask(q, k, g, budget, u, raster=True, workspace=ws, out=sip))
-    attn_ms = timed(lambda: dbst.block_sparse_attn_offsets(q, k, v, g, sip[1], sip[2], sip[3], raster=True,
-                                                           out=o, lse=lse))
-    plain_ms = timed(lambda: dbst.block_sparse_attn_offsets(q, k, v, g, cnt, idx, None, raster=True, out=o, lse=lse))
+    sel_ms = timed_median(lambda: dbst.build_sip_mask(q, k, g, budget, u, raster=True, workspace=ws, out=sip),
+                          args.steps, args.warmup)
+    attn_ms = timed_median(lambda: dbst.block_sparse_attn_offsets(q, k, v, g, sip[1], sip[2], sip[3], raster=True,
+                                                                  out=o, lse=lse), args.steps, args.warmup)
+    plain_ms = timed_median(lambda: dbst.block_sparse_attn_offsets(q, k, v, g, cnt, idx, None, raster=True, out=o,
+                                                                   lse=lse), args.steps, args.warmup)
     dbst.get_error()
     kept_sip = int(sip[1].sum().item())
     kept = int(cnt.sum().item())
     unit = 4.0 * w.D * 64 * 64
-    out = {"sip": workload_desc(w, p), "budget_blocks_per_row": budget,
-           "kept_fraction_sip": kept_sip / (g.B * g.H * g.NB * g.NB), "sip_mask_ms": sel_ms,
-           "sip_attn_ms": attn_ms, "sip_attn_tflops": unit * kept_sip / (attn_ms * 1e-3) / 1e12,
-           "two_sweep_attn_on_nabla_mask_ms": plain_ms,
-           "two_sweep_attn_tflops": unit * kept / (plain_ms * 1e-3) / 1e12,
-           "note": "TFLOP/s count the 2 products of attention per kept block pair; the two-sweep kernel runs 3"}
-    print(json.dumps(out), flush=True)
+    return {"sip": workload_desc(w, p), "budget_blocks_per_row": budget,
+            "kept_fraction_sip": kept_sip / (g.B * g.H * g.NB * g.NB), "sip_mask_ms": sel_ms,
+            "sip_attn_ms": attn_ms, "sip_attn_tflops": unit * kept_sip / (attn_ms * 1e-3) / 1e12,
+            "two_sweep_attn_on_nabla_mask_ms": plain_ms,
+            "two_sweep_attn_tflops": unit * kept / (plain_ms * 1e-3) / 1e12,
+            "note": "TFLOP/s count the 2 products of attention per kept block pair; the two-sweep kernel runs 3"}
+
+
+def run_sip(args, w, p):
+    print(json.dumps(measure_sip(args, w, p)), flush=True)
     return 0
 
 
-def run_squad(args):
+def measure_squad(args) -> dict:
     """SQuad two-pass attention against dense attention on the same tensors (B=2 H=16 N=16384 D=128,
-    w = sqrt(N) = 128).  One JSON line; not the headline metric."""
+    w = sqrt(N) = 128)."""
     import torch
     import dynamic_block_sparse_tile_b200 as dbst
     dbst.load()
@@ -409,32 +395,19 @@ def run_squad(args):
     q, k, v = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda() for a in S.make_qkv(w))
     ws = torch.empty(dbst.squad_workspace_bytes(w.B, w.H, w.N, w.D, win), dtype=torch.uint8, device="cuda")
     o = torch.empty_like(q)
-
-    def timed(fn):
-        for _ in range(max(args.warmup, 3)):
-            fn()
-        torch.cuda.synchronize()
-        ts = []
-        for _ in range(args.steps):
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record()
-            fn()
-            b.record()
-            torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b))
-        return statistics.median(ts)
-
-    squad_ms = timed(lambda: dbst.squad_attn(q, k, v, win, workspace=ws, out=o))
-    dense_ms = timed(lambda: dbst.dense_attn_raster(q, k, v, g))
+    squad_ms = timed_median(lambda: dbst.squad_attn(q, k, v, win, workspace=ws, out=o), args.steps, args.warmup)
+    dense_ms = timed_median(lambda: dbst.dense_attn_raster(q, k, v, g), args.steps, args.warmup)
     dbst.get_error()
     flops = 4.0 * w.D * w.N * (win + w.N // win) * w.B * w.H
     moved = 2 * 4 * w.B * w.H * w.N * w.D * 2      # four window transposes, each a read and a write
-    out = {"squad": f"B={w.B} H={w.H} N={w.N} D={w.D} w={win}", "squad_ms": squad_ms, "dense_attn_ms": dense_ms,
-           "speedup_vs_dense": dense_ms / squad_ms, "squad_tflops": flops / (squad_ms * 1e-3) / 1e12,
-           "squad_flop_fraction_of_dense": flops / (4.0 * w.D * w.N * w.N * w.B * w.H),
-           "transpose_bytes": moved, "launches": 6}
-    print(json.dumps(out), flush=True)
+    return {"squad": f"B={w.B} H={w.H} N={w.N} D={w.D} w={win}", "squad_ms": squad_ms, "dense_attn_ms": dense_ms,
+            "speedup_vs_dense": dense_ms / squad_ms, "squad_tflops": flops / (squad_ms * 1e-3) / 1e12,
+            "squad_flop_fraction_of_dense": flops / (4.0 * w.D * w.N * w.N * w.B * w.H),
+            "transpose_bytes": moved, "launches": 6}
+
+
+def run_squad(args):
+    print(json.dumps(measure_squad(args)), flush=True)
     return 0
 
 
@@ -453,6 +426,9 @@ def main():
                     help="sparsity sweep: attention ms/call and kept-block TFLOP/s per p, dense crossover")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--squad", action="store_true", help="time SQuad two-pass attention against dense attention")
+    ap.add_argument("--no-extensions", action="store_true",
+                    help="skip the extension measurements (backward, SIP, SQuad) after the timed step, e.g. "
+                         "under a profiler's launch list")
     ap.add_argument("--sip", action="store_true",
                     help="time the SIP sampled mask and the attention with inclusion-probability offsets")
     ap.add_argument("--backward", action="store_true",
@@ -652,6 +628,18 @@ def main():
                 "h2d_bytes_per_step": 3 * host[0].numel() * 2, "d2h_bytes_per_step": o_host.numel() * 2},
         "clocks": clk, "gpu_launches": launches_per_step * args.steps,
     }
+    if world == 1 and not args.no_extensions:
+        # The rows built on top of the path, each timed on its own after the step above (outside its
+        # timed region and launch count); a failure is recorded here and cannot touch the line.
+        ext = {}
+        for name, fn in (("backward", lambda: measure_backward(args, w, p, (q, k, v))),
+                         ("sip", lambda: measure_sip(args, w, p, (q, k, v))),
+                         ("squad", lambda: measure_squad(args))):
+            try:
+                ext[name] = fn()
+            except Exception as e:   # noqa: BLE001 - reported, not raised
+                ext[name] = {"error": f"{type(e).__name__}: {e}"}
+        line["extensions"] = ext
     if rank == 0 and not args.no_cpu_baseline:
         cv, cs, desc = oracle_sample(w, p, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": cv, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
