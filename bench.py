@@ -149,6 +149,23 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def cpu_model() -> str:
+    """The host CPU's model name, from /proc/cpuinfo where it exists."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+# NVIDIA's dense bf16 tensor figure for one B200 (its 4.5 PFLOP/s per-GPU figure assumes 2:4
+# sparsity); reported beside the measured peaks, never instead of them.
+NOMINAL_BF16_TFLOPS = 2250.0
+
+
 def cpu_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -233,7 +250,7 @@ def run_reference(args, w, p):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": workload_desc(w, p), "sample": "bounded oracle sample"},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
-                             "sample": desc},
+                             "sample": desc, "cpu_model": cpu_model(), "nproc": os.cpu_count()},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -383,6 +400,38 @@ def run_sip(args, w, p):
     return 0
 
 
+def measure_step(args, name: str) -> dict:
+    """The fused step (mask build + pairing + attention, raster in and out) on another workload,
+    timed call by call: the Wan-like latent in its 2x4x8 tiles."""
+    import torch
+    import dynamic_block_sparse_tile_b200 as dbst
+    dbst.load()
+    w = S.workload(name)
+    p = w.p_list[0]
+    g = dbst.Geom.make(w.B, w.H, w.D, w.grid, w.tile)
+    q, k, v = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda() for a in S.make_qkv(w))
+    ws = torch.empty(dbst.mask_workspace_bytes(g), dtype=torch.uint8, device="cuda")
+    mask = dbst.build_block_mask_raster(q, k, g, p, w.sta_radius, workspace=ws)
+    pairs = dbst.pair_query_blocks(mask[0], g)
+    o = torch.empty_like(q)
+    lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device="cuda")
+
+    def mask_and_pairs():
+        dbst.build_block_mask_raster(q, k, g, p, w.sta_radius, workspace=ws, out=mask)
+        dbst.pair_query_blocks(mask[0], g, out=pairs)
+
+    mask_ms = timed_median(mask_and_pairs, args.steps, args.warmup)
+    attn_ms = timed_median(lambda: dbst.block_sparse_attn_raster(q, k, v, g, mask[1], mask[2], 0.0, True, o, lse,
+                                                                 pairs), args.steps, args.warmup)
+    dbst.get_error()
+    kept = int(mask[1].sum().item())
+    flops = 4.0 * w.D * 64 * 64 * kept
+    return {"workload": workload_desc(w, p), "kept_fraction": kept / (g.B * g.H * g.NB * g.NB),
+            "mask_and_pairing_ms": mask_ms, "sparse_attn_ms": attn_ms,
+            "sparse_attn_tflops": flops / (attn_ms * 1e-3) / 1e12,
+            "step_tflops": flops / ((mask_ms + attn_ms) * 1e-3) / 1e12}
+
+
 def measure_squad(args) -> dict:
     """SQuad two-pass attention against dense attention on the same tensors (B=2 H=16 N=16384 D=128,
     w = sqrt(N) = 128)."""
@@ -427,8 +476,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--squad", action="store_true", help="time SQuad two-pass attention against dense attention")
     ap.add_argument("--no-extensions", action="store_true",
-                    help="skip the extension measurements (backward, SIP, SQuad) after the timed step, e.g. "
-                         "under a profiler's launch list")
+                    help="skip the extension measurements (backward, SIP, SQuad, the 2x4x8-tile Wan variant) "
+                         "after the timed step, e.g. under a profiler's launch list")
     ap.add_argument("--sip", action="store_true",
                     help="time the SIP sampled mask and the attention with inclusion-probability offsets")
     ap.add_argument("--backward", action="store_true",
@@ -620,6 +669,8 @@ def main():
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": bf16, "unit": "TFLOP/s",
                      "frac": attn_tflops / bf16, "traffic": measured_traffic(w.name, p, "raster" if fused else "tiled"),
                      "peak_source": f"{src} bf16 burst; frac of sustained {attn_tflops / bf16_sus:.3f}",
+                     "frac_of_sustained": attn_tflops / bf16_sus,
+                     "frac_of_nominal_dense_bf16": attn_tflops / NOMINAL_BF16_TFLOPS,
                      "kernel": "pair_attn_kernel<128, raster>" if fused else "pair_attn_kernel<128, tiled>"},
         "mask_roofline": {"bound": "hbm", "achieved": mask_bytes / (mask_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
                           "frac": mask_bytes / (mask_ms * 1e-3) / 1e9 / hbm},
@@ -634,7 +685,8 @@ def main():
         ext = {}
         for name, fn in (("backward", lambda: measure_backward(args, w, p, (q, k, v))),
                          ("sip", lambda: measure_sip(args, w, p, (q, k, v))),
-                         ("squad", lambda: measure_squad(args))):
+                         ("squad", lambda: measure_squad(args)),
+                         ("wan_tiles_2x4x8", lambda: measure_step(args, "wan_2x4x8"))):
             try:
                 ext[name] = fn()
             except Exception as e:   # noqa: BLE001 - reported, not raised
@@ -643,7 +695,7 @@ def main():
     if rank == 0 and not args.no_cpu_baseline:
         cv, cs, desc = oracle_sample(w, p, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": cv, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
-                                "sample": desc}
+                                "sample": desc, "cpu_model": cpu_model(), "nproc": os.cpu_count()}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

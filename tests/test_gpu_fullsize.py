@@ -120,6 +120,12 @@ def test_wan_like_full_size_bench_path(built):
     assert np.max(np.abs(lse_gpu - lse_ref_t)) <= P.LSE_MAX_ABS
 
 
+def test_wan_like_2x4x8_variant_full_size(built):
+    """The Wan-like latent in 2x4x8 tiles on the grid padded to 22 frames (616 blocks)."""
+    kept, excused = check_full("wan_2x4x8", 0.9, per_head=8)
+    assert 0.05 < kept < 0.15
+
+
 def test_hunyuan_like_full_size(built):
     kept, excused = check_full("hunyuan", 0.9, per_head=64)
     assert 0.03 < kept < 0.15

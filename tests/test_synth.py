@@ -36,6 +36,7 @@ def test_workload_geometry():
     assert S.workload("wan").NB == 588 and S.workload("wan").N == 37632
     assert S.workload("hunyuan").NB == 2040 and S.workload("hunyuan").N == 130560
     assert S.workload("sweep").NB == 256
+    assert S.workload("wan_2x4x8").NB == 616 and S.workload("wan_2x4x8").N == 39424
 
 
 def test_field_statistics():
