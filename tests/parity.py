@@ -87,6 +87,16 @@ def mask_mismatches(gpu: np.ndarray, ref: np.ndarray, A: np.ndarray, p: float, s
     return hard, excused
 
 
+def rows_where_masks_agree(got: np.ndarray, ref: np.ndarray, rows=None):
+    """Query blocks (b, h, i) whose GPU mask row equals the oracle's row; from `rows`, or all.
+
+    Attention parity feeds the oracle its own mask only.  A GPU output computed on the GPU's
+    mask is therefore compared only where the two masks agree (they can differ only at
+    near-threshold blocks, which the mask checks excuse)."""
+    cand = rows if rows is not None else list(np.ndindex(*got.shape[:3]))
+    return [tuple(int(x) for x in r) for r in cand if np.array_equal(got[tuple(r)], ref[tuple(r)])]
+
+
 def lists_match_bits(cnt: np.ndarray, idx: np.ndarray, mask: np.ndarray) -> bool:
     if not np.array_equal(cnt, mask.sum(-1)):
         return False

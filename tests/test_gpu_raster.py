@@ -93,13 +93,17 @@ def test_raster_against_oracle(built):
     og, (q, k, v), _, raster = both_paths(w, 0.9, 1)
     qt, kt, vt = (O.tile_reorder(a, og) for a in (q, k, v))
     got = P.unpack_mask(raster["mask"][0].cpu().numpy().view(np.uint32), og.NB)
-    o_ref_t, lse_ref_t = O.masked_attention(qt, kt, vt, got, 64, 1.0 / math.sqrt(w.D))
-    o_ref = O.tile_unreorder(o_ref_t, og)
-    lse_ref = O.tile_unreorder(lse_ref_t[..., None], og)[..., 0]
-    o = raster["o"].float().cpu().numpy().astype(np.float64)
-    max_abs, rel = P.attn_errors(o, o_ref)
+    # the oracle on its own mask; outputs compared on the query blocks whose mask rows agree
+    ref = O.build_block_mask(qt, kt, og, 0.9, 1)
+    agree = (got == ref).all(-1)
+    assert agree.mean() >= 0.9
+    sel = np.repeat(agree, 64, axis=-1)
+    o_ref_t, lse_ref_t = O.masked_attention(qt, kt, vt, ref, 64, 1.0 / math.sqrt(w.D))
+    o_t = O.tile_reorder(raster["o"].float().cpu().numpy().astype(np.float64), og)
+    lse_t = O.tile_reorder(raster["lse"].cpu().numpy()[..., None], og)[..., 0]
+    max_abs, rel = P.attn_errors(o_t[sel], o_ref_t[sel])
     assert max_abs <= P.ATTN_MAX_ABS and rel <= P.ATTN_REL_L2, (max_abs, rel)
-    assert np.max(np.abs(raster["lse"].cpu().numpy() - lse_ref)) <= P.LSE_MAX_ABS
+    assert np.max(np.abs(lse_t[sel] - lse_ref_t[sel])) <= P.LSE_MAX_ABS
 
 
 @pytest.mark.slow

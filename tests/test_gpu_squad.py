@@ -50,13 +50,14 @@ def test_squad_matches_oracle(built, B, H, D, grid, w):
 
 def test_squad_explicit_scale_and_repeat_is_identical(built):
     wl = workload(1, 2, 128, (4, 32, 32))
-    q, k, v = (P.bits_to_torch(a) for a in S.make_qkv(wl))
+    qh, kh, vh = S.make_qkv(wl)
+    q, k, v = (P.bits_to_torch(a) for a in (qh, kh, vh))
     ws = torch.empty(dbst.squad_workspace_bytes(1, 2, wl.N, 128, 64), dtype=torch.uint8, device="cuda")
     first = dbst.squad_attn(q, k, v, 64, scale=0.05, workspace=ws)
     again = dbst.squad_attn(q, k, v, 64, scale=0.05, workspace=ws)
     dbst.get_error()
     assert torch.equal(first, again)
-    ref, _ = O.squad_attention(*(P.torch_to_bits(t) for t in (q, k, v)), 64, 0.05)
+    ref, _ = O.squad_attention(qh, kh, vh, 64, 0.05)
     got = S.f32_from_bf16_bits(P.torch_to_bits(first)).astype(np.float64)
     assert np.abs(got - ref).max() <= SQUAD_MAX_ABS
 
