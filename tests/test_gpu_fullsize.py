@@ -4,8 +4,10 @@ Same call sequence as bench.py's explicit path (reorder -> mask -> attention
 -> unreorder), and the bench's default path in its own test.  The mask is
 compared with the oracle on every row of every head, with the near-threshold
 exemption.  Attention is compared on seeded query blocks in every head (plus
-the first and the last block), against the oracle given the mask the GPU built
-and given the oracle's own mask.
+the first and the last block); the oracle always runs on its own mask.  The
+GPU's output on its own mask is compared on the blocks whose mask rows equal
+the oracle's, and the GPU's output on the oracle's mask (expanded to lists on
+the GPU) on every sampled block.
 """
 import dataclasses
 import math
