@@ -87,6 +87,33 @@ def mask_mismatches(gpu: np.ndarray, ref: np.ndarray, A: np.ndarray, p: float, s
     return hard, excused
 
 
+def near_tie(A: np.ndarray, p: float, b: int, h: int, i: int, j: int, tol: float = 1e-6) -> bool:
+    """Whether block j of row (b, h, i) ties (within `tol` in pooled mass) with the row's boundary
+    block, the last one the oracle keeps.  Such disagreements are reported on their own; they are
+    not excused."""
+    a = A[b, h, i]
+    order = np.argsort(-a, kind="stable")
+    c = np.cumsum(a[order])
+    k = min(int(np.searchsorted(c, p)), len(a) - 1) if p < 1.0 else len(a) - 1
+    return abs(a[j] - a[order[k]]) <= tol
+
+
+def write_mask_report(name: str, p: float, hard, excused, A: np.ndarray) -> None:
+    """With DBST_PARITY_REPORT_DIR set, list every excused mask block (and every non-excused one,
+    with its near-tie flag) in <dir>/mask_parity_<name>_p<p>.json."""
+    import json
+    import os
+    out = os.environ.get("DBST_PARITY_REPORT_DIR")
+    if not out:
+        return
+    os.makedirs(out, exist_ok=True)
+    rep = {"workload": name, "p": p, "cdf_exemption": CDF_EXEMPT,
+           "excused": [[int(x) for x in t] for t in excused],
+           "not_excused": [[int(x) for x in t] + [bool(near_tie(A, p, *(int(x) for x in t)))] for t in hard]}
+    with open(os.path.join(out, f"mask_parity_{name}_p{p}.json"), "w") as f:
+        json.dump(rep, f)
+
+
 def rows_where_masks_agree(got: np.ndarray, ref: np.ndarray, rows=None):
     """Query blocks (b, h, i) whose GPU mask row equals the oracle's row; from `rows`, or all.
 

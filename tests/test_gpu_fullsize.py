@@ -57,7 +57,9 @@ def check_full(name, p, per_head=8):
     ref, A = P.oracle_mask_per_head(qt, kt, og, p, w.sta_radius)
     got = P.unpack_mask(bits.cpu().numpy().view(np.uint32), og.NB)
     hard, excused = P.mask_mismatches(got, ref, A, p, O.sta_mask(og, w.sta_radius))
-    assert not hard, f"{len(hard)} non-excused mask disagreements, first {hard[:5]}"
+    P.write_mask_report(name, p, hard, excused, A)
+    ties = sum(P.near_tie(A, p, *t) for t in hard)
+    assert not hard, f"{len(hard)} non-excused mask disagreements ({ties} at a near-tie), first {hard[:5]}"
     cnt_h, idx_h = cnt.cpu().numpy(), idx.cpu().numpy()
     assert np.array_equal(cnt_h, got.sum(-1))
     # attention on sampled query blocks computed on the GPU's own lists, against the oracle on its
