@@ -21,8 +21,8 @@ __all__ = ["Geom", "DbstError", "lib_path", "load", "tile_reorder", "tile_unreor
            "build_block_mask", "build_block_mask_noalloc", "mask_from_bits", "block_sparse_attn", "dense_attn",
            "build_block_mask_raster", "block_sparse_attn_raster", "dense_attn_raster", "pair_query_blocks",
            "transpose_block_mask", "attn_backward_workspace_bytes", "block_sparse_attn_backward",
-           "squad_workspace_bytes", "squad_attn", "build_sip_mask", "block_sparse_attn_offsets", "get_error",
-           "EXPORTS"]
+           "squad_workspace_bytes", "squad_attn", "build_sip_mask", "block_sparse_attn_offsets",
+           "fine_mask_workspace_bytes", "build_fine_mask", "block_sparse_attn_groups", "get_error", "EXPORTS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libdbst.so")
@@ -35,7 +35,8 @@ EXPORTS = ("dbst_status_string", "dbst_tile_reorder", "dbst_tile_unreorder", "db
            "dbst_transpose_block_mask", "dbst_attn_backward_workspace_bytes", "dbst_block_sparse_attn_backward",
            "dbst_block_sparse_attn_backward_raster", "dbst_squad_workspace_bytes", "dbst_squad_attn",
            "dbst_build_sip_mask", "dbst_build_sip_mask_raster", "dbst_block_sparse_attn_offsets",
-           "dbst_block_sparse_attn_offsets_raster")
+           "dbst_block_sparse_attn_offsets_raster", "dbst_fine_mask_workspace_bytes", "dbst_build_fine_mask",
+           "dbst_build_fine_mask_raster", "dbst_block_sparse_attn_groups", "dbst_block_sparse_attn_groups_raster")
 
 DBST_OK, DBST_EINVAL, DBST_ECUDA, DBST_ETIMEOUT, DBST_EBOUNDS, DBST_ETOOLARGE = 0, 1, 2, 3, 4, 5
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -117,6 +118,14 @@ def load() -> ctypes.CDLL:
         getattr(lib, name).argtypes = [vp, vp, gp, ctypes.c_double, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
         getattr(lib, name).restype = i32
     for name in ("dbst_block_sparse_attn_offsets", "dbst_block_sparse_attn_offsets_raster"):
+        getattr(lib, name).argtypes = [vp, vp, vp, gp, vp, vp, vp, f32, vp, vp, vp]
+        getattr(lib, name).restype = i32
+    lib.dbst_fine_mask_workspace_bytes.argtypes = [gp]
+    lib.dbst_fine_mask_workspace_bytes.restype = ctypes.c_size_t
+    for name in ("dbst_build_fine_mask", "dbst_build_fine_mask_raster"):
+        getattr(lib, name).argtypes = [vp, vp, gp, f32, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        getattr(lib, name).restype = i32
+    for name in ("dbst_block_sparse_attn_groups", "dbst_block_sparse_attn_groups_raster"):
         getattr(lib, name).argtypes = [vp, vp, vp, gp, vp, vp, vp, f32, vp, vp, vp]
         getattr(lib, name).restype = i32
     _lib = lib
@@ -399,6 +408,54 @@ def block_sparse_attn_offsets(q, k, v, g: Geom, kv_count, kv_idx, offsets: Optio
     fn = "dbst_block_sparse_attn_offsets_raster" if raster else "dbst_block_sparse_attn_offsets"
     _check(getattr(load(), fn)(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(g), _ptr(kv_count), _ptr(kv_idx),
                                _ptr(offsets), float(scale), _ptr(o), _ptr(lse if want_lse else None), _stream()), fn)
+    return o, (lse if want_lse else None)
+
+
+def fine_mask_workspace_bytes(g: Geom) -> int:
+    return int(load().dbst_fine_mask_workspace_bytes(ctypes.byref(g)))
+
+
+def build_fine_mask(q, k, g: Geom, p: float, raster: bool = False, workspace: Optional[torch.Tensor] = None,
+                    out=None):
+    """Mask of kept 4-token key groups (``dbst_build_fine_mask[_raster]``) -> (group_mask, kv_count, kv_idx).
+
+    group_mask: int16 [B, H, NB, NB], bit r of [.., i, j] = group r (tokens 4r .. 4r+3) of key block j.
+    """
+    _need(q, torch.bfloat16, _qkv_shape(g), "q")
+    _need(k, torch.bfloat16, _qkv_shape(g), "k")
+    dev = q.device
+    if out is None:
+        gm = torch.empty((g.B, g.H, g.NB, g.NB), dtype=torch.int16, device=dev)
+        cnt = torch.empty((g.B, g.H, g.NB), dtype=torch.int32, device=dev)
+        idx = torch.empty((g.B, g.H, g.NB, g.NB), dtype=torch.int16, device=dev)
+    else:
+        gm, cnt, idx = out
+    nbytes = fine_mask_workspace_bytes(g)
+    if nbytes == 0:
+        raise ValueError("fine mask: unsupported geometry (at most 1024 blocks per head)")
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    fn = "dbst_build_fine_mask_raster" if raster else "dbst_build_fine_mask"
+    _check(getattr(load(), fn)(_ptr(q), _ptr(k), ctypes.byref(g), float(p), _ptr(gm), _ptr(cnt), _ptr(idx),
+                               _ptr(workspace), workspace.numel() * workspace.element_size(), _stream()), fn)
+    return gm, cnt, idx
+
+
+def block_sparse_attn_groups(q, k, v, g: Geom, kv_count, kv_idx, group_mask, scale: float = 0.0,
+                             raster: bool = False, want_lse: bool = True, out: Optional[torch.Tensor] = None,
+                             lse: Optional[torch.Tensor] = None):
+    """Attention over the kept 4-token key groups (``dbst_block_sparse_attn_groups[_raster]``) -> (o, lse)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, _qkv_shape(g), n)
+    _need(kv_count, torch.int32, (g.B, g.H, g.NB), "kv_count")
+    _need(kv_idx, torch.int16, (g.B, g.H, g.NB, g.NB), "kv_idx")
+    _need(group_mask, torch.int16, (g.B, g.H, g.NB, g.NB), "group_mask")
+    o = torch.empty_like(q) if out is None else out
+    if want_lse and lse is None:
+        lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device=q.device)
+    fn = "dbst_block_sparse_attn_groups_raster" if raster else "dbst_block_sparse_attn_groups"
+    _check(getattr(load(), fn)(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(g), _ptr(kv_count), _ptr(kv_idx),
+                               _ptr(group_mask), float(scale), _ptr(o), _ptr(lse if want_lse else None), _stream()), fn)
     return o, (lse if want_lse else None)
 
 

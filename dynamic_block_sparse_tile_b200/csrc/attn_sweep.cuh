@@ -55,7 +55,9 @@
 // row is exactly 1 in bf16 (as in pair_attn_kernel); normalising before the rounding instead
 // costs about 0.006 of max-abs error where a row sits on one key.  No rescaling of o between
 // tiles is needed.  Three 128x64xD products per tile against the two of pair_attn_kernel, for a
-// kernel whose offsets cost nothing extra.
+// kernel whose offsets cost nothing extra.  With a group mask (AB-Attention's third technique,
+// key groups of 4 tokens), bit r of mask[i][j] keeps tokens 4r .. 4r+3 of key block j for query
+// block i; the other columns get P = 0 in both sweeps.
 //
 // TMEM (512 columns): acc0 at 0, acc1 at 128, two tile buffers at 256 and 384; in buffer b the
 // A product sits at +0 .. +63 and A2 at +64 .. +127.  Softmax warp (q, hc) reads columns
@@ -87,6 +89,7 @@ struct SweepParams {
   const float* lse;          // [BH*N] the forward's log-sum-exp, same layout as q (dq pass)
   float2* stats;             // [BH*N] tile order: (lse * log2 e, delta); written by the dq pass
   const float* offsets;      // MODE 2: [BH*NB*NB] natural-log offset of (query block, key block), or null
+  const uint16_t* gmask;     // MODE 2: [BH*NB*NB] kept 4-token groups of (query block, key block), or null
   float* lse_out;            // MODE 2: [BH*N] log-sum-exp of the offset logits, same layout as q, or null
   __nv_bfloat16* out0;       // dq pass: dq; dk/dv pass: dv; MODE 2: o
   __nv_bfloat16* out1;       // dk/dv pass: dk
@@ -442,6 +445,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
       // ---- forward with offsets: first sweep row max and sum, second sweep P = 2^(x - M) and o += P V
       const int own = side ? bb : ba;
       const float* offrow = prm.offsets ? prm.offsets + (bh * NB + own) * static_cast<long long>(NB) : nullptr;
+      const uint16_t* gmrow = prm.gmask ? prm.gmask + (bh * NB + own) * static_cast<long long>(NB) : nullptr;
       float m = -INFINITY, l = 0.0f;          // first sweep, this warp's columns: running max of x, sum of 2^(x - m)
       float M = -INFINITY, L = -INFINITY;     // the row's max of x and log2 of its normaliser
       bool live = true;
@@ -451,7 +455,10 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
         wait_live(bar(BB_SFULL + b), (v >> 1) & 1, live);
         tc_fence_after();
         const int ent = s_union[t];
-        const bool vh = (ent >> (16 + side)) & 1;   // uniform per warp
+        // this warp's 32 columns are the groups 8hc .. 8hc+7 of the tile's key block
+        const uint32_t gbits = (((ent >> (16 + side)) & 1) == 0) ? 0u
+                               : (gmrow != nullptr) ? ((gmrow[ent & 0xFFFF] >> (8 * hc)) & 0xFFu) : 0xFFu;
+        const bool vh = gbits != 0u;                 // uniform per warp
         const uint32_t buf = tmem + kSweepBuf + 128u * b + 32u * hc + lrow;
         const float off = (vh && offrow != nullptr) ? offrow[ent & 0xFFFF] * 1.4426950408889634f : 0.0f;
         if (v < T) {
@@ -459,13 +466,15 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             uint32_t sv[32];
             tmem_ld32(buf, sv);
             tmem_wait_ld();
-            float smax = __uint_as_float(sv[0]);
+            float smax = -INFINITY;
 #pragma unroll
-            for (int c = 1; c < 32; ++c) smax = fmaxf(smax, __uint_as_float(sv[c]));
-            const float mn = fmaxf(m, fmaf(smax, sc, off));   // finite: this tile is kept
+            for (int c = 0; c < 32; ++c)
+              if ((gbits >> (c >> 2)) & 1u) smax = fmaxf(smax, __uint_as_float(sv[c]));
+            const float mn = fmaxf(m, fmaf(smax, sc, off));   // finite: a kept group is here
             float acc = 0.0f;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) acc += fast_exp2(fmaf(__uint_as_float(sv[c]), sc, off - mn));
+            for (int c = 0; c < 32; ++c)
+              if ((gbits >> (c >> 2)) & 1u) acc += fast_exp2(fmaf(__uint_as_float(sv[c]), sc, off - mn));
             l = fmaf(l, fast_exp2(m - mn), acc);               // m = -inf: 2^-inf = 0
             m = mn;
           }
@@ -489,9 +498,12 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
           tmem_wait_ld();
           const float nb = off - M;
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
-            pp[c] = pack_bf16x2(fast_exp2(fmaf(__uint_as_float(sv[2 * c]), sc, nb)),
-                                fast_exp2(fmaf(__uint_as_float(sv[2 * c + 1]), sc, nb)));
+          for (int c = 0; c < 16; ++c) {   // columns 2c and 2c+1 share group c/2
+            const bool keep = (gbits >> (c >> 1)) & 1u;
+            pp[c] = keep ? pack_bf16x2(fast_exp2(fmaf(__uint_as_float(sv[2 * c]), sc, nb)),
+                                       fast_exp2(fmaf(__uint_as_float(sv[2 * c + 1]), sc, nb)))
+                         : 0u;
+          }
         } else {
 #pragma unroll
           for (int c = 0; c < 16; ++c) pp[c] = 0u;

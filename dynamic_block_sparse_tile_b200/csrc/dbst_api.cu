@@ -12,6 +12,7 @@
 
 #include "../../include/dbst.h"
 #include "attn_sweep.cuh"
+#include "fine.cuh"
 #include "attn_pair.cuh"
 #include "pairing.cuh"
 #include "mask.cuh"
@@ -335,8 +336,8 @@ dbst_status window_transpose(const void* src, void* dst, long long heads, int A,
 // Forward with a logit offset per (query block, key block): the two-sweep kernel, MODE 2.
 template <int D, bool RASTER>
 dbst_status launch_offset_attn(const void* q, const void* k, const void* v, const dbst_geom* g, const int32_t* cnt,
-                               const int16_t* idx, const float* offsets, float scale, void* o, float* lse,
-                               cudaStream_t s) {
+                               const int16_t* idx, const float* offsets, const uint16_t* gmask, float scale, void* o,
+                               float* lse, cudaStream_t s) {
   const long long rows = bh_count(g) * tokens(g);
   CUtensorMap tq, tk, tv;
   if (RASTER) {
@@ -349,6 +350,7 @@ dbst_status launch_offset_attn(const void* q, const void* k, const void* v, cons
   p.count = cnt;
   p.idx = idx;
   p.offsets = offsets;
+  p.gmask = gmask;
   p.lse_out = lse;
   p.out0 = static_cast<__nv_bfloat16*>(o);
   p.NB = nblocks(g);
@@ -373,20 +375,21 @@ dbst_status launch_offset_attn(const void* q, const void* k, const void* v, cons
 }
 
 dbst_status offset_attn_common(const void* q, const void* k, const void* v, const dbst_geom* g, const int32_t* cnt,
-                               const int16_t* idx, const float* offsets, float scale, void* o, float* lse,
-                               void* stream, bool raster) {
+                               const int16_t* idx, const float* offsets, const uint16_t* gmask, float scale, void* o,
+                               float* lse, void* stream, bool raster) {
   if (!geom_ok(g) || !q || !k || !v || !o || !cnt || !idx) return DBST_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(cnt) || !aligned16(idx))
     return DBST_EINVAL;
-  if ((lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) || (offsets && (reinterpret_cast<uintptr_t>(offsets) & 3u)))
+  if ((lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) || (offsets && (reinterpret_cast<uintptr_t>(offsets) & 3u)) ||
+      (gmask && (reinterpret_cast<uintptr_t>(gmask) & 1u)))
     return DBST_EINVAL;
   if (!std::isfinite(scale)) return DBST_EINVAL;
   auto s = static_cast<cudaStream_t>(stream);
   if (raster)
-    return g->D == 128 ? launch_offset_attn<128, true>(q, k, v, g, cnt, idx, offsets, scale, o, lse, s)
-                       : launch_offset_attn<64, true>(q, k, v, g, cnt, idx, offsets, scale, o, lse, s);
-  return g->D == 128 ? launch_offset_attn<128, false>(q, k, v, g, cnt, idx, offsets, scale, o, lse, s)
-                     : launch_offset_attn<64, false>(q, k, v, g, cnt, idx, offsets, scale, o, lse, s);
+    return g->D == 128 ? launch_offset_attn<128, true>(q, k, v, g, cnt, idx, offsets, gmask, scale, o, lse, s)
+                       : launch_offset_attn<64, true>(q, k, v, g, cnt, idx, offsets, gmask, scale, o, lse, s);
+  return g->D == 128 ? launch_offset_attn<128, false>(q, k, v, g, cnt, idx, offsets, gmask, scale, o, lse, s)
+                     : launch_offset_attn<64, false>(q, k, v, g, cnt, idx, offsets, gmask, scale, o, lse, s);
 }
 
 template <int NPT>
@@ -480,6 +483,79 @@ dbst_status build_mask(const void* q_tiled, const void* k_tiled, const dbst_geom
     else ok = launch_select<16>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
     if (!ok) return DBST_ECUDA;
   }
+  return launch_status();
+}
+
+// Fine mask (4-token key groups): float64 query-block and key-group means, the float64 logits of
+// every (query block, key group), then one CTA per row for the CDF selection over groups.
+constexpr int kFineMaxNB = dbst::kFineMaxGroups / 16;
+struct FineWorkspace {
+  size_t qp, kp, s, total;
+};
+FineWorkspace fine_workspace(const dbst_geom* g) {
+  const size_t nb = static_cast<size_t>(nblocks(g)), ng = 16 * nb, bh = static_cast<size_t>(bh_count(g));
+  FineWorkspace w;
+  w.qp = 0;
+  w.kp = align_up(bh * nb * g->D * sizeof(double));
+  w.s = w.kp + align_up(bh * ng * g->D * sizeof(double));
+  w.total = w.s + align_up(bh * nb * ng * sizeof(double));
+  return w;
+}
+
+dbst_status build_fine_mask(const void* q, const void* k, const dbst_geom* g, float p, uint16_t* gmask,
+                            int32_t* kv_count, int16_t* kv_idx, void* workspace, size_t workspace_bytes, void* stream,
+                            bool raster) {
+  if (!geom_ok(g) || !q || !k || !gmask || !kv_count || !kv_idx || !workspace) return DBST_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(gmask) || !aligned16(kv_count) || !aligned16(kv_idx) ||
+      !aligned16(workspace))
+    return DBST_EINVAL;
+  if (!(p > 0.0f && p <= 1.0f)) return DBST_EINVAL;
+  if (nblocks(g) > kFineMaxNB || bh_count(g) > 65535) return DBST_EINVAL;
+  const FineWorkspace w = fine_workspace(g);
+  if (workspace_bytes < w.total) return DBST_EINVAL;
+  auto s = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  double* qp = reinterpret_cast<double*>(ws + w.qp);
+  double* kp = reinterpret_cast<double*>(ws + w.kp);
+  double* S = reinterpret_cast<double*>(ws + w.s);
+  const int NB = nblocks(g), NG = 16 * NB;
+  const long long bh = bh_count(g);
+  const dbst::TileGeo tg = tile_geo(g);
+  const long long cap = static_cast<long long>(sm_count()) * 8;
+  auto grid_for = [&](long long warps) {
+    long long grid = (warps * 32 + 255) / 256;
+    return static_cast<unsigned>(grid > cap ? cap : grid);
+  };
+  const auto* qa = static_cast<const uint4*>(q);
+  const auto* ka = static_cast<const uint4*>(k);
+  const long long nq = bh * NB, nk = bh * NG;
+  if (g->D == 128) {
+    if (raster) {
+      dbst::group_pool_kernel<128, true, 64><<<grid_for(nq), 256, 0, s>>>(qa, qp, nq, tg);
+      dbst::group_pool_kernel<128, true, 4><<<grid_for(nk), 256, 0, s>>>(ka, kp, nk, tg);
+    } else {
+      dbst::group_pool_kernel<128, false, 64><<<grid_for(nq), 256, 0, s>>>(qa, qp, nq, tg);
+      dbst::group_pool_kernel<128, false, 4><<<grid_for(nk), 256, 0, s>>>(ka, kp, nk, tg);
+    }
+  } else {
+    if (raster) {
+      dbst::group_pool_kernel<64, true, 64><<<grid_for(nq), 256, 0, s>>>(qa, qp, nq, tg);
+      dbst::group_pool_kernel<64, true, 4><<<grid_for(nk), 256, 0, s>>>(ka, kp, nk, tg);
+    } else {
+      dbst::group_pool_kernel<64, false, 64><<<grid_for(nq), 256, 0, s>>>(qa, qp, nq, tg);
+      dbst::group_pool_kernel<64, false, 4><<<grid_for(nk), 256, 0, s>>>(ka, kp, nk, tg);
+    }
+  }
+  if (cudaGetLastError() != cudaSuccess) return DBST_ECUDA;
+  const double scale = 1.0 / std::sqrt(static_cast<double>(g->D));
+  dim3 lgrid((NG + 63) / 64, (NB + 63) / 64, static_cast<unsigned>(bh));
+  if (g->D == 128)
+    dbst::fine_logits_kernel<128><<<lgrid, 256, 0, s>>>(qp, kp, S, NB, NG, scale);
+  else
+    dbst::fine_logits_kernel<64><<<lgrid, 256, 0, s>>>(qp, kp, S, NB, NG, scale);
+  if (cudaGetLastError() != cudaSuccess) return DBST_ECUDA;
+  dbst::fine_select_kernel<<<static_cast<unsigned>(bh * NB), dbst::kFineThreads, 0, s>>>(
+      S, NB, static_cast<double>(p), gmask, kv_count, kv_idx);
   return launch_status();
 }
 
@@ -671,17 +747,50 @@ dbst_status dbst_build_sip_mask_raster(const void* q, const void* k, const dbst_
                         workspace_bytes, stream, true);
 }
 
+size_t dbst_fine_mask_workspace_bytes(const dbst_geom* g) {
+  if (!geom_ok(g) || nblocks(g) > kFineMaxNB) return 0;
+  return fine_workspace(g).total;
+}
+
+dbst_status dbst_build_fine_mask(const void* q_tiled, const void* k_tiled, const dbst_geom* g, float p,
+                                 uint16_t* group_mask, int32_t* kv_count, int16_t* kv_idx, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  return build_fine_mask(q_tiled, k_tiled, g, p, group_mask, kv_count, kv_idx, workspace, workspace_bytes, stream,
+                         false);
+}
+
+dbst_status dbst_build_fine_mask_raster(const void* q, const void* k, const dbst_geom* g, float p,
+                                        uint16_t* group_mask, int32_t* kv_count, int16_t* kv_idx, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  return build_fine_mask(q, k, g, p, group_mask, kv_count, kv_idx, workspace, workspace_bytes, stream, true);
+}
+
+dbst_status dbst_block_sparse_attn_groups(const void* q, const void* k, const void* v, const dbst_geom* g,
+                                          const int32_t* kv_count, const int16_t* kv_idx, const uint16_t* group_mask,
+                                          float scale, void* o, float* lse, void* stream) {
+  if (!group_mask) return DBST_EINVAL;
+  return offset_attn_common(q, k, v, g, kv_count, kv_idx, nullptr, group_mask, scale, o, lse, stream, false);
+}
+
+dbst_status dbst_block_sparse_attn_groups_raster(const void* q, const void* k, const void* v, const dbst_geom* g,
+                                                 const int32_t* kv_count, const int16_t* kv_idx,
+                                                 const uint16_t* group_mask, float scale, void* o, float* lse,
+                                                 void* stream) {
+  if (!group_mask) return DBST_EINVAL;
+  return offset_attn_common(q, k, v, g, kv_count, kv_idx, nullptr, group_mask, scale, o, lse, stream, true);
+}
+
 dbst_status dbst_block_sparse_attn_offsets(const void* q, const void* k, const void* v, const dbst_geom* g,
                                            const int32_t* kv_count, const int16_t* kv_idx, const float* offsets,
                                            float scale, void* o, float* lse, void* stream) {
-  return offset_attn_common(q, k, v, g, kv_count, kv_idx, offsets, scale, o, lse, stream, false);
+  return offset_attn_common(q, k, v, g, kv_count, kv_idx, offsets, nullptr, scale, o, lse, stream, false);
 }
 
 dbst_status dbst_block_sparse_attn_offsets_raster(const void* q, const void* k, const void* v, const dbst_geom* g,
                                                   const int32_t* kv_count, const int16_t* kv_idx,
                                                   const float* offsets, float scale, void* o, float* lse,
                                                   void* stream) {
-  return offset_attn_common(q, k, v, g, kv_count, kv_idx, offsets, scale, o, lse, stream, true);
+  return offset_attn_common(q, k, v, g, kv_count, kv_idx, offsets, nullptr, scale, o, lse, stream, true);
 }
 
 size_t dbst_squad_workspace_bytes(int B, int H, int N, int D, int w) {

@@ -312,6 +312,49 @@ dbst_status dbst_block_sparse_attn_offsets_raster(const void* q, const void* k, 
                                                   void* stream);
 
 /*
+ * Fine-grained mask with key groups of 4 tokens (AB-Attention page, section
+ * "Les trois techniques", third technique).  Scoring and selection follow
+ * dbst_build_block_mask with a finer key unit: each 64-token query block and
+ * each run of 4 consecutive tile-ordered key tokens (a "group"; 16 per block)
+ * is mean-pooled in float64, the pooled logits (scale 1/sqrt(D)) are
+ * soft-maxed over all N/4 groups of the row, and the row keeps the smallest
+ * descending prefix of groups whose mass reaches p (ties to the lower group;
+ * p = 1 keeps all).  No sliding-tile union.  Outputs, per (b, h, query block i):
+ *   group_mask[b,h,i,j] : uint16, bit r set if group r of key block j (its
+ *                         tokens 4r .. 4r+3) is kept
+ *   kv_count, kv_idx    : the key blocks with any kept group, ascending (the
+ *                         layout of dbst_build_block_mask)
+ * NB must be at most 1024.  workspace: dbst_fine_mask_workspace_bytes(g)
+ * (float64 means and the [B,H,NB,N/4] float64 logits).  The _raster form
+ * takes raster q, k.
+ */
+size_t dbst_fine_mask_workspace_bytes(const dbst_geom* g);
+dbst_status dbst_build_fine_mask(const void* q_tiled, const void* k_tiled, const dbst_geom* g, float p,
+                                 uint16_t* group_mask, int32_t* kv_count, int16_t* kv_idx, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+dbst_status dbst_build_fine_mask_raster(const void* q, const void* k, const dbst_geom* g, float p,
+                                        uint16_t* group_mask, int32_t* kv_count, int16_t* kv_idx, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
+/*
+ * Attention over the kept 4-token groups: for query block i, the keys are the
+ * tokens of the groups that group_mask[b,h,i,:] keeps in the blocks listed by
+ * (kv_count, kv_idx); exact softmax over those tokens, o bf16, lse float32
+ * (NULL allowed).  Runs the two-sweep kernel of dbst_block_sparse_attn_offsets
+ * over the listed blocks with the other groups' columns masked, so it costs
+ * whole blocks; gathering the kept groups into full tiles is not done here.
+ * group_mask must be 2-byte aligned and is required.  The _raster form takes
+ * raster q, k, v, o, lse.
+ */
+dbst_status dbst_block_sparse_attn_groups(const void* q, const void* k, const void* v, const dbst_geom* g,
+                                          const int32_t* kv_count, const int16_t* kv_idx, const uint16_t* group_mask,
+                                          float scale, void* o, float* lse, void* stream);
+dbst_status dbst_block_sparse_attn_groups_raster(const void* q, const void* k, const void* v, const dbst_geom* g,
+                                                 const int32_t* kv_count, const int16_t* kv_idx,
+                                                 const uint16_t* group_mask, float scale, void* o, float* lse,
+                                                 void* stream);
+
+/*
  * SQuad two-pass attention (page "SQuad: Sub-Quadratic Attention Distillation
  * for Efficient Video Generation", section "Methodology: SQuad", item
  * "1. SQuad-Attention Operator").  The N tokens of each (b, h) are read as

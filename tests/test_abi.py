@@ -224,3 +224,39 @@ def test_mask_builders_reject_too_many_heads_before_any_launch(lib):
     assert lib.dbst_build_block_mask(a, a, ctypes.byref(g), 0.9, -1, a, a, a, a, ws, None) == dbst.DBST_EINVAL
     assert lib.dbst_build_block_mask_raster(a, a, ctypes.byref(g), 0.9, -1, a, a, a, a, ws, None) == dbst.DBST_EINVAL
     assert lib.dbst_build_sip_mask(a, a, ctypes.byref(g), 2.0, a, a, a, a, a, a, ws, None) == dbst.DBST_EINVAL
+
+
+def test_fine_mask_and_group_attention_validate_arguments(lib):
+    g = geom()
+    a = ctypes.c_void_p(1 << 20)
+    ws = lib.dbst_fine_mask_workspace_bytes(ctypes.byref(g))
+    nb, ng, bh = g.N // 64, g.N // 4, 2
+    up = lambda x: (x + 255) // 256 * 256   # noqa: E731
+    assert ws == up(bh * nb * 128 * 8) + up(bh * ng * 128 * 8) + up(bh * nb * ng * 8)
+    big = geom(grid=(8, 128, 128), tile=(1, 8, 8))          # 2048 blocks: above the 1024 limit
+    assert lib.dbst_fine_mask_workspace_bytes(ctypes.byref(big)) == 0
+    for fn in (lib.dbst_build_fine_mask, lib.dbst_build_fine_mask_raster):
+        ok = [a, a, ctypes.byref(g), 0.9, a, a, a, a, ws, None]
+        for i in (0, 1, 4, 5, 6, 7):
+            args = list(ok)
+            args[i] = None
+            assert fn(*args) == dbst.DBST_EINVAL, i
+        for p in (0.0, 1.5, float("nan")):
+            args = list(ok)
+            args[3] = p
+            assert fn(*args) == dbst.DBST_EINVAL
+        args = list(ok)
+        args[8] = ws - 1
+        assert fn(*args) == dbst.DBST_EINVAL
+        args = list(ok)
+        args[2] = ctypes.byref(big)
+        assert fn(*args) == dbst.DBST_EINVAL
+    for fn in (lib.dbst_block_sparse_attn_groups, lib.dbst_block_sparse_attn_groups_raster):
+        ok = [a, a, a, ctypes.byref(g), a, a, a, 0.0, a, None, None]
+        for i in (0, 1, 2, 4, 5, 6, 8):
+            args = list(ok)
+            args[i] = None
+            assert fn(*args) == dbst.DBST_EINVAL, i
+        args = list(ok)
+        args[6] = ctypes.c_void_p((1 << 20) + 1)                      # group mask not 2-byte aligned
+        assert fn(*args) == dbst.DBST_EINVAL
