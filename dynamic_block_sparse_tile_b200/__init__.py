@@ -22,7 +22,8 @@ __all__ = ["Geom", "DbstError", "lib_path", "load", "tile_reorder", "tile_unreor
            "build_block_mask_raster", "block_sparse_attn_raster", "dense_attn_raster", "pair_query_blocks",
            "transpose_block_mask", "attn_backward_workspace_bytes", "block_sparse_attn_backward",
            "squad_workspace_bytes", "squad_attn", "build_sip_mask", "block_sparse_attn_offsets",
-           "fine_mask_workspace_bytes", "build_fine_mask", "block_sparse_attn_groups", "get_error", "EXPORTS"]
+           "fine_mask_workspace_bytes", "build_fine_mask", "block_sparse_attn_groups", "block_sparse_attn_gather",
+           "get_error", "EXPORTS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libdbst.so")
@@ -36,7 +37,8 @@ EXPORTS = ("dbst_status_string", "dbst_tile_reorder", "dbst_tile_unreorder", "db
            "dbst_block_sparse_attn_backward_raster", "dbst_squad_workspace_bytes", "dbst_squad_attn",
            "dbst_build_sip_mask", "dbst_build_sip_mask_raster", "dbst_block_sparse_attn_offsets",
            "dbst_block_sparse_attn_offsets_raster", "dbst_fine_mask_workspace_bytes", "dbst_build_fine_mask",
-           "dbst_build_fine_mask_raster", "dbst_block_sparse_attn_groups", "dbst_block_sparse_attn_groups_raster")
+           "dbst_build_fine_mask_raster", "dbst_block_sparse_attn_groups", "dbst_block_sparse_attn_groups_raster",
+           "dbst_block_sparse_attn_gather", "dbst_block_sparse_attn_gather_raster")
 
 DBST_OK, DBST_EINVAL, DBST_ECUDA, DBST_ETIMEOUT, DBST_EBOUNDS, DBST_ETOOLARGE = 0, 1, 2, 3, 4, 5
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -124,6 +126,9 @@ def load() -> ctypes.CDLL:
     lib.dbst_fine_mask_workspace_bytes.restype = ctypes.c_size_t
     for name in ("dbst_build_fine_mask", "dbst_build_fine_mask_raster"):
         getattr(lib, name).argtypes = [vp, vp, gp, f32, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        getattr(lib, name).restype = i32
+    for name in ("dbst_block_sparse_attn_gather", "dbst_block_sparse_attn_gather_raster"):
+        getattr(lib, name).argtypes = [vp, vp, vp, gp, vp, f32, vp, vp, vp]
         getattr(lib, name).restype = i32
     for name in ("dbst_block_sparse_attn_groups", "dbst_block_sparse_attn_groups_raster"):
         getattr(lib, name).argtypes = [vp, vp, vp, gp, vp, vp, vp, f32, vp, vp, vp]
@@ -456,6 +461,23 @@ def block_sparse_attn_groups(q, k, v, g: Geom, kv_count, kv_idx, group_mask, sca
     fn = "dbst_block_sparse_attn_groups_raster" if raster else "dbst_block_sparse_attn_groups"
     _check(getattr(load(), fn)(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(g), _ptr(kv_count), _ptr(kv_idx),
                                _ptr(group_mask), float(scale), _ptr(o), _ptr(lse if want_lse else None), _stream()), fn)
+    return o, (lse if want_lse else None)
+
+
+def block_sparse_attn_gather(q, k, v, g: Geom, group_mask, scale: float = 0.0, raster: bool = False,
+                             want_lse: bool = True, out: Optional[torch.Tensor] = None,
+                             lse: Optional[torch.Tensor] = None):
+    """Attention over the kept 4-token key groups, gathered 16 to a tile
+    (``dbst_block_sparse_attn_gather[_raster]``) -> (o, lse)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, _qkv_shape(g), n)
+    _need(group_mask, torch.int16, (g.B, g.H, g.NB, g.NB), "group_mask")
+    o = torch.empty_like(q) if out is None else out
+    if want_lse and lse is None:
+        lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device=q.device)
+    fn = "dbst_block_sparse_attn_gather_raster" if raster else "dbst_block_sparse_attn_gather"
+    _check(getattr(load(), fn)(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(g), _ptr(group_mask), float(scale), _ptr(o),
+                               _ptr(lse if want_lse else None), _stream()), fn)
     return o, (lse if want_lse else None)
 
 

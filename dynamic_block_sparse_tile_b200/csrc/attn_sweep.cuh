@@ -101,22 +101,32 @@ struct SweepParams {
   TileGeo tg;                // token grid and tile shape (raster layout only)
 };
 
-struct SweepSmem {
+// Shared-memory layout.  Modes 0-2 walk key (or query) blocks: at most 4096 union entries over
+// 128 words of 32 blocks.  Mode 3 walks 4-token key groups, 16 per block: up to 16384 entries over
+// 512 words, and it has no second own tile, so its ring starts right after X.
+template <int MODE>
+struct SweepLayout {
+  static constexpr int kUnionCap = MODE == 3 ? 16384 : 4096;
+  static constexpr int kMaxWords = kUnionCap / 32;
   static constexpr int kOwnX = 0;                         // X: D-halves x [128 rows x 128 B]
-  static constexpr int kOwnX2 = 32768;                    // X2, same layout
-  static constexpr int kRing = 65536;
+  static constexpr int kOwnX2 = 32768;                    // X2, same layout (modes 0 and 1)
+  static constexpr int kRing = MODE == 3 ? 32768 : 65536;
   static constexpr int kSlot = 33792;                     // Y: D-halves x [64 rows x 128 B]; Y2 at +16384;
   static constexpr int kSlotY2 = 16384;                   //   64 float2 stats of Y's rows at +32768
   static constexpr int kSlotStats = 32768;
-  static constexpr int kUnion = kRing + kSweepSlots * kSlot;   // int32 x 4096: j | inA<<16 | inB<<17
-  static constexpr int kWords = kUnion + 16384;           // u32 [2][128] bitmasks of the two lists
-  static constexpr int kScan = kWords + 1024;             // int [128] word offsets
-  static constexpr int kDelta = kScan + 512;              // float [2 quantities][2 column halves][128 rows]
+  static constexpr int kUnion = kRing + kSweepSlots * kSlot;   // int32 x kUnionCap: j | inA<<16 | inB<<17
+  static constexpr int kWords = kUnion + 4 * kUnionCap;   // u32 [2][kMaxWords] bitmasks of the two lists
+  static constexpr int kScan = kWords + 8 * kMaxWords;    // int [kMaxWords] word offsets
+  static constexpr int kDelta = kScan + 4 * kMaxWords;    // float [2 quantities][2 column halves][128 rows]
   static constexpr int kBars = kDelta + 2048;
   static constexpr int kMisc = kBars + 256;
   static constexpr int kBytes = kMisc + 64;
+  static_assert(kSlot % 1024 == 0 && kRing % 1024 == 0, "swizzled tiles need 1 KB alignment");
+  static_assert(kBytes + 1024 <= 227 * 1024, "shared memory per CTA");
 };
-static_assert(SweepSmem::kSlot % 1024 == 0 && SweepSmem::kRing % 1024 == 0, "swizzled tiles need 1 KB alignment");
+using SweepSmem = SweepLayout<0>;
+static_assert(SweepLayout<0>::kBytes == SweepLayout<1>::kBytes && SweepLayout<0>::kBytes == SweepLayout<2>::kBytes,
+              "modes 0-2 share one layout");
 
 enum {
   BB_OWN = 0,
@@ -173,19 +183,21 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmY2,
                const SweepParams prm) {
   static_assert(D == 64 || D == 128, "head dim");
-  static_assert(MODE >= 0 && MODE <= 2, "mode");
+  static_assert(MODE >= 0 && MODE <= 3, "mode");
+  using L = SweepLayout<MODE>;
   constexpr bool DKDV = MODE == 1;
-  constexpr bool FWD = MODE == 2;
+  constexpr bool GATHER = MODE == 3;            // the forward over gathered 4-token key groups
+  constexpr bool FWD = MODE == 2 || GATHER;     // the forward sweeps (offsets, group masks, gather)
   constexpr int DH = D / 64;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(sm);
-  int32_t* s_union = reinterpret_cast<int32_t*>(sm + SweepSmem::kUnion);
-  uint32_t* s_words = reinterpret_cast<uint32_t*>(sm + SweepSmem::kWords);
-  int32_t* s_scan = reinterpret_cast<int32_t*>(sm + SweepSmem::kScan);
-  uint32_t* s_misc = reinterpret_cast<uint32_t*>(sm + SweepSmem::kMisc);
+  int32_t* s_union = reinterpret_cast<int32_t*>(sm + L::kUnion);
+  uint32_t* s_words = reinterpret_cast<uint32_t*>(sm + L::kWords);
+  int32_t* s_scan = reinterpret_cast<int32_t*>(sm + L::kScan);
+  uint32_t* s_misc = reinterpret_cast<uint32_t*>(sm + L::kMisc);
   volatile uint32_t* s_abort = s_misc + 2;
-  auto bar = [&](int slot) -> uint32_t { return sbase + SweepSmem::kBars + 8u * slot; };
+  auto bar = [&](int slot) -> uint32_t { return sbase + L::kBars + 8u * slot; };
   auto wait_live = [&](uint32_t mb, uint32_t parity, bool& live) {
     if (!live || mbar_try(mb, parity)) return;
     const long long t0 = clock64();
@@ -221,8 +233,21 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
       tma_load_2d(dst, map, mbar, 64 * h, static_cast<int32_t>(bh * prm.N + static_cast<long long>(blk) * 64));
     }
   };
+  // Mode 3: TMA load of 4-token group grp's channels 64h .. 64h+63 (4 rows, 512 B); the map's box
+  // is 4 rows high (RASTER: 4 tokens along x, which the host requires tx to allow)
+  auto load_group = [&](uint32_t dst, const CUtensorMap* map, uint32_t mbar, int grp, int h) {
+    if constexpr (RASTER) {
+      const int blk = grp >> 4, off = (grp & 15) * 4;
+      const int Tx = blk % prm.tg.nX, Ty = (blk / prm.tg.nX) % prm.tg.nY, Tt = blk / (prm.tg.nX * prm.tg.nY);
+      const int dx = off % prm.tg.tx, dy = (off / prm.tg.tx) % prm.tg.ty, dt = off / (prm.tg.tx * prm.tg.ty);
+      tma_load_5d(dst, map, mbar, 64 * h, Tx * prm.tg.tx + dx, Ty * prm.tg.ty + dy, Tt * prm.tg.tt + dt,
+                  static_cast<int32_t>(bh));
+    } else {
+      tma_load_2d(dst, map, mbar, 64 * h, static_cast<int32_t>(bh * prm.N + static_cast<long long>(grp) * 4));
+    }
+  };
 
-  for (int w = tid; w < 2 * 128; w += kSweepThreads) s_words[w] = 0u;
+  for (int w = tid; w < 2 * L::kMaxWords; w += kSweepThreads) s_words[w] = 0u;
   if (tid == 0) {
     for (int b = 0; b < BB_COUNT; ++b) mbar_init(bar(b), (b == BB_PFULL || b == BB_PFULL + 1) ? 256u : 1u);
     fence_mbar_init();
@@ -234,20 +259,34 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
     if constexpr (!FWD) tma_prefetch_desc(&tmX2);
     mbar_expect_tx(bar(BB_OWN), (FWD ? 1 : 2) * 128 * D * 2);
     for (int h = 0; h < DH; ++h) {
-      load_block(sbase + SweepSmem::kOwnX + h * 16384, &tmX, bar(BB_OWN), ba, h);
-      load_block(sbase + SweepSmem::kOwnX + h * 16384 + 8192, &tmX, bar(BB_OWN), has_b ? bb : ba, h);
+      load_block(sbase + L::kOwnX + h * 16384, &tmX, bar(BB_OWN), ba, h);
+      load_block(sbase + L::kOwnX + h * 16384 + 8192, &tmX, bar(BB_OWN), has_b ? bb : ba, h);
       if constexpr (!FWD) {
-        load_block(sbase + SweepSmem::kOwnX2 + h * 16384, &tmX2, bar(BB_OWN), ba, h);
-        load_block(sbase + SweepSmem::kOwnX2 + h * 16384 + 8192, &tmX2, bar(BB_OWN), has_b ? bb : ba, h);
+        load_block(sbase + L::kOwnX2 + h * 16384, &tmX2, bar(BB_OWN), ba, h);
+        load_block(sbase + L::kOwnX2 + h * 16384 + 8192, &tmX2, bar(BB_OWN), has_b ? bb : ba, h);
       }
     }
   }
   if (warp == 8) {
-    tmem_alloc(sbase + SweepSmem::kMisc, 512);
+    tmem_alloc(sbase + L::kMisc, 512);
     tmem_relinquish();
     tc_fence_before();
   }
   // ---- union of the two own blocks' lists -> ascending entries with membership flags
+  // (mode 3: of their kept 4-token groups, read from the group masks: word w holds blocks 2w, 2w+1)
+  const int NWu = GATHER ? (16 * NB + 31) >> 5 : NW;
+  if constexpr (GATHER) {
+    const uint16_t* m0 = prm.gmask + (bh * NB + ba) * static_cast<long long>(NB);
+    const uint16_t* m1 = prm.gmask + (bh * NB + (has_b ? bb : ba)) * static_cast<long long>(NB);
+    for (int e = tid; e < 2 * NWu; e += kSweepThreads) {
+      const int side = e >= NWu;
+      const int w = side ? e - NWu : e;
+      if (side && !has_b) continue;
+      const uint16_t* m = side ? m1 : m0;
+      const uint32_t lo = m[2 * w], hi = (2 * w + 1 < NB) ? m[2 * w + 1] : 0u;
+      s_words[side * L::kMaxWords + w] = lo | (hi << 16);
+    }
+  } else {
   int n0 = prm.count[bh * NB + ba];
   int n1 = has_b ? prm.count[bh * NB + bb] : 0;
   if (n0 < 0 || n0 > NB || n1 < 0 || n1 > NB) {
@@ -264,15 +303,17 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
       record_error(kErrBounds);
       continue;
     }
-    atomicOr(&s_words[side * 128 + (j >> 5)], 1u << (j & 31));
+    atomicOr(&s_words[side * L::kMaxWords + (j >> 5)], 1u << (j & 31));
+  }
   }
   __syncthreads();
-  if (warp == 0) {   // exclusive scan of the union's popcounts over NW <= 128 words
-    int cnt[4], tot = 0;
+  if (warp == 0) {   // exclusive scan of the union's popcounts over NWu <= kMaxWords words
+    constexpr int WPL = L::kMaxWords / 32;
+    int cnt[WPL], tot = 0;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int w = 4 * lane + e;
-      cnt[e] = (w < NW) ? __popc(s_words[w] | s_words[128 + w]) : 0;
+    for (int e = 0; e < WPL; ++e) {
+      const int w = WPL * lane + e;
+      cnt[e] = (w < NWu) ? __popc(s_words[w] | s_words[L::kMaxWords + w]) : 0;
       tot += cnt[e];
     }
     int incl = tot;
@@ -283,15 +324,15 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
     }
     int run = incl - tot;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      s_scan[4 * lane + e] = run;
+    for (int e = 0; e < WPL; ++e) {
+      s_scan[WPL * lane + e] = run;
       run += cnt[e];
     }
     if (lane == 31) s_misc[1] = static_cast<uint32_t>(incl);
   }
   __syncthreads();
-  for (int w = tid; w < NW; w += kSweepThreads) {
-    const uint32_t wa = s_words[w], wb = s_words[128 + w];
+  for (int w = tid; w < NWu; w += kSweepThreads) {
+    const uint32_t wa = s_words[w], wb = s_words[L::kMaxWords + w];
     uint32_t u = wa | wb;
     int pos = s_scan[w];
     while (u) {
@@ -303,7 +344,8 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_misc[0];
-  const int T = static_cast<int>(s_misc[1]);
+  const int nu = static_cast<int>(s_misc[1]);   // union entries (blocks; mode 3: groups)
+  const int T = GATHER ? (nu + 15) >> 4 : nu;   // tiles: one block, or 16 groups
   const int NV = DKDV ? T : 2 * T;       // virtual tiles
   const int v_ts = DKDV ? 0 : T;         // first virtual tile with TS products
   if (T == 0) {   // nothing in either list: zero gradients; MODE 2: o = 0 and lse = -inf
@@ -328,7 +370,48 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
     return;
   }
 
-  if (warp == 9) {
+  if (warp == 9 && GATHER) {
+    // ------------------------------------------------------------ mode 3 producer: 16 groups per tile
+    // Lane 0 waits for the slot and arms its barrier; then lanes 0-15 each load one group (the
+    // first group of the tile stands in past the end of the union; its columns are masked).
+    if (lane == 0) {
+      tma_prefetch_desc(&tmY);
+      tma_prefetch_desc(&tmY2);
+    }
+    int armed[kSweepSlots] = {0, 0, 0};
+    for (int v = 0; v < NV; ++v) {
+      const int s = v % kSweepSlots;
+      int ok = 1;
+      if (lane == 0) {
+        if (*s_abort) {
+          ok = 0;
+        } else if (v >= kSweepSlots && !mbar_wait(bar(BB_REMPTY + s), ((v / kSweepSlots) - 1) & 1)) {
+          *s_abort = 1;
+          ok = 0;
+        } else {
+          mbar_expect_tx(bar(BB_RFULL + s), (v >= T ? 2 : 1) * 64 * D * 2);   // values in the second sweep
+          armed[s] = v / kSweepSlots + 1;
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      __syncwarp();
+      if (lane < 16) {
+        const int t = v < T ? v : v - T;
+        const int u = 16 * t + lane;
+        const int grp = (u < nu ? s_union[u] : s_union[16 * t]) & 0xFFFF;
+        const uint32_t dst = sbase + L::kRing + s * L::kSlot + 512u * lane;
+        for (int h = 0; h < DH; ++h) {
+          load_group(dst + h * 8192, &tmY, bar(BB_RFULL + s), grp, h);
+          if (v >= T) load_group(dst + L::kSlotY2 + h * 8192, &tmY2, bar(BB_RFULL + s), grp, h);
+        }
+      }
+    }
+    if (lane == 0) {   // no copy may still be landing when the CTA exits
+      for (int s = 0; s < kSweepSlots; ++s)
+        if (armed[s] > 0) mbar_wait(bar(BB_RFULL + s), (armed[s] - 1) & 1);
+      mbar_wait(bar(BB_OWN), 0);
+    }
+  } else if (warp == 9) {
     // ------------------------------------------------------------ TMA producer of the ring
     if (lane == 0) {
       tma_prefetch_desc(&tmY);
@@ -342,15 +425,15 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
           break;
         }
         const int j = s_union[t < T ? t : t - T] & 0xFFFF;
-        const uint32_t dst = sbase + SweepSmem::kRing + s * SweepSmem::kSlot;
+        const uint32_t dst = sbase + L::kRing + s * L::kSlot;
         const bool withY2 = !(FWD && t < T);   // the offset forward's first sweep needs no values
         mbar_expect_tx(bar(BB_RFULL + s), (withY2 ? 2 : 1) * 64 * D * 2 + (DKDV ? 512 : 0));
         for (int h = 0; h < DH; ++h) {
           load_block(dst + h * 8192, &tmY, bar(BB_RFULL + s), j, h);
-          if (withY2) load_block(dst + SweepSmem::kSlotY2 + h * 8192, &tmY2, bar(BB_RFULL + s), j, h);
+          if (withY2) load_block(dst + L::kSlotY2 + h * 8192, &tmY2, bar(BB_RFULL + s), j, h);
         }
         if constexpr (DKDV)
-          bulk_load_1d(dst + SweepSmem::kSlotStats, prm.stats + bh * prm.N + static_cast<long long>(j) * 64, 512,
+          bulk_load_1d(dst + L::kSlotStats, prm.stats + bh * prm.N + static_cast<long long>(j) * 64, 512,
                        bar(BB_RFULL + s));
         armed[s] = t / kSweepSlots + 1;
       }
@@ -363,10 +446,10 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
     // ------------------------------------------------------------ MMA issuer (whole warp)
     constexpr uint32_t idSS = idesc_bf16(128, 64, 0, 0);   // A = own rows (K-major), B = ring rows (K-major)
     constexpr uint32_t idTS = idesc_bf16(128, D, 0, 1);    // A = P or dS in TMEM, B = ring rows (MN-major)
-    const uint64_t dX = smem_desc(sbase + SweepSmem::kOwnX, 16, 1024);
-    const uint64_t dX2 = smem_desc(sbase + SweepSmem::kOwnX2, 16, 1024);
-    const uint64_t dRingK = smem_desc(sbase + SweepSmem::kRing, 16, 1024);
-    const uint64_t dRingMN = smem_desc(sbase + SweepSmem::kRing, 8192, 1024);
+    const uint64_t dX = smem_desc(sbase + L::kOwnX, 16, 1024);
+    const uint64_t dX2 = smem_desc(sbase + L::kOwnX2, 16, 1024);
+    const uint64_t dRingK = smem_desc(sbase + L::kRing, 16, 1024);
+    const uint64_t dRingMN = smem_desc(sbase + L::kRing, 8192, 1024);
     auto wait_all = [&](int slot, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar(slot), parity));
     };
@@ -374,8 +457,8 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
       const int s = t % kSweepSlots, b = t & 1;
       if (!wait_all(BB_RFULL + s, (t / kSweepSlots) & 1)) return false;
       tc_fence_after();
-      const uint64_t y = dRingK + static_cast<uint64_t>((s * SweepSmem::kSlot) >> 4);
-      const uint64_t y2 = y + static_cast<uint64_t>(SweepSmem::kSlotY2 >> 4);
+      const uint64_t y = dRingK + static_cast<uint64_t>((s * L::kSlot) >> 4);
+      const uint64_t y2 = y + static_cast<uint64_t>(L::kSlotY2 >> 4);
       const uint32_t acc = tmem + kSweepBuf + 128u * b;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
@@ -394,8 +477,8 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
       const int s = u % kSweepSlots, b = u & 1;
       if (!wait_all(BB_PFULL + b, (u >> 1) & 1)) return false;
       tc_fence_after();
-      const uint64_t y = dRingMN + static_cast<uint64_t>((s * SweepSmem::kSlot) >> 4);
-      const uint64_t y2 = y + static_cast<uint64_t>(SweepSmem::kSlotY2 >> 4);
+      const uint64_t y = dRingMN + static_cast<uint64_t>((s * L::kSlot) >> 4);
+      const uint64_t y2 = y + static_cast<uint64_t>(L::kSlotY2 >> 4);
       const uint32_t buf = tmem + kSweepBuf + 128u * b;
       if (u >= v_ts) {
 #pragma unroll
@@ -440,7 +523,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
     const int side = r >> 6;                  // 0: block ba, 1: block bb (uniform per warp)
     const uint32_t lrow = static_cast<uint32_t>(32 * q) << 16;
     const float sc = prm.scale_log2;
-    float* s_delta = reinterpret_cast<float*>(sm + SweepSmem::kDelta);
+    float* s_delta = reinterpret_cast<float*>(sm + L::kDelta);
     if constexpr (FWD) {
       // ---- forward with offsets: first sweep row max and sum, second sweep P = 2^(x - M) and o += P V
       const int own = side ? bb : ba;
@@ -454,13 +537,24 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
         const int t = v < T ? v : v - T;
         wait_live(bar(BB_SFULL + b), (v >> 1) & 1, live);
         tc_fence_after();
-        const int ent = s_union[t];
-        // this warp's 32 columns are the groups 8hc .. 8hc+7 of the tile's key block
-        const uint32_t gbits = (((ent >> (16 + side)) & 1) == 0) ? 0u
-                               : (gmrow != nullptr) ? ((gmrow[ent & 0xFFFF] >> (8 * hc)) & 0xFFu) : 0xFFu;
+        // this warp's 32 columns are the groups 8hc .. 8hc+7 of the tile: of the tile's key block,
+        // or (mode 3) union entries 16t + 8hc .. +7
+        uint32_t gbits = 0u;
+        float off = 0.0f;
+        if constexpr (GATHER) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int u = 16 * t + 8 * hc + e;
+            if (u < nu && ((s_union[u] >> (16 + side)) & 1)) gbits |= 1u << e;
+          }
+        } else {
+          const int ent = s_union[t];
+          gbits = (((ent >> (16 + side)) & 1) == 0) ? 0u
+                  : (gmrow != nullptr) ? ((gmrow[ent & 0xFFFF] >> (8 * hc)) & 0xFFu) : 0xFFu;
+          if (gbits != 0u && offrow != nullptr) off = offrow[ent & 0xFFFF] * 1.4426950408889634f;
+        }
         const bool vh = gbits != 0u;                 // uniform per warp
         const uint32_t buf = tmem + kSweepBuf + 128u * b + 32u * hc + lrow;
-        const float off = (vh && offrow != nullptr) ? offrow[ent & 0xFFFF] * 1.4426950408889634f : 0.0f;
         if (v < T) {
           if (vh) {
             uint32_t sv[32];
@@ -580,8 +674,8 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
           tmem_wait_ld();
           if constexpr (DKDV) {
             // column c of the tile is query row c of the ring block: (lse * log2 e, delta) per column
-            const float4* st4 = reinterpret_cast<const float4*>(sm + SweepSmem::kRing + s * SweepSmem::kSlot +
-                                                                SweepSmem::kSlotStats) + 16 * hc;
+            const float4* st4 = reinterpret_cast<const float4*>(sm + L::kRing + s * L::kSlot +
+                                                                L::kSlotStats) + 16 * hc;
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
               const float4 st = st4[c];

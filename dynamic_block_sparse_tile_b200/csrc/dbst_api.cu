@@ -24,6 +24,7 @@
 namespace {
 
 constexpr int kMaxNB = 4096;   // selection and list kernels keep one row on chip
+constexpr int kFineMaxNB = dbst::kFineMaxGroups / 16;   // 4-token groups: 16384 per row at most
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -166,6 +167,33 @@ bool make_tmap_raster(CUtensorMap* m, const void* base, const dbst_geom* g) {
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Boxes of 4 token rows (one 4-token key group) x 64 channels: a [rows, D] matrix, or the raster
+// [B*H, T, Y, X, D] tensor with the 4 tokens along x.
+bool make_tmap_group(CUtensorMap* m, const void* base, long long rows, int D) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  cuuint32_t box[2] = {64, 4};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+bool make_tmap_raster_group(CUtensorMap* m, const void* base, const dbst_geom* g) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t D = static_cast<cuuint64_t>(g->D);
+  cuuint64_t dims[5] = {D, static_cast<cuuint64_t>(g->X), static_cast<cuuint64_t>(g->Y), static_cast<cuuint64_t>(g->T),
+                        static_cast<cuuint64_t>(bh_count(g))};
+  cuuint64_t strides[4] = {D * 2, D * 2 * dims[1], D * 2 * dims[1] * dims[2], D * 2 * dims[1] * dims[2] * dims[3]};
+  cuuint32_t box[5] = {64, 4, 1, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int D, bool RASTER>
@@ -374,6 +402,62 @@ dbst_status launch_offset_attn(const void* q, const void* k, const void* v, cons
   return launch_status();
 }
 
+// Attention over the kept 4-token groups, gathered 16 to a 64-key tile: the sweep kernel, MODE 3.
+template <int D, bool RASTER>
+dbst_status launch_gather_attn(const void* q, const void* k, const void* v, const dbst_geom* g, const uint16_t* gmask,
+                               float scale, void* o, float* lse, cudaStream_t s) {
+  const long long rows = bh_count(g) * tokens(g);
+  CUtensorMap tq, tk, tv;
+  if (RASTER) {
+    if (!make_tmap_raster(&tq, q, g) || !make_tmap_raster_group(&tk, k, g) || !make_tmap_raster_group(&tv, v, g))
+      return DBST_ECUDA;
+  } else {
+    if (!make_tmap(&tq, q, rows, D) || !make_tmap_group(&tk, k, rows, D) || !make_tmap_group(&tv, v, rows, D))
+      return DBST_ECUDA;
+  }
+  dbst::SweepParams p{};
+  p.tg = tile_geo(g);
+  p.gmask = gmask;
+  p.lse_out = lse;
+  p.out0 = static_cast<__nv_bfloat16*>(o);
+  p.NB = nblocks(g);
+  p.N = static_cast<int>(tokens(g));
+  p.pair_stride = pair_stride(g);
+  p.pairs_per_head = ((p.NB + 2 * p.pair_stride - 1) / (2 * p.pair_stride)) * p.pair_stride;
+  const float sc = scale > 0.0f ? scale : 1.0f / std::sqrt(static_cast<float>(D));
+  p.scale = sc;
+  p.scale_log2 = sc * 1.4426950408889634f;
+  const int smem = dbst::SweepLayout<3>::kBytes + 1024;
+  static std::once_flag once;
+  static cudaError_t attr = cudaSuccess;
+  std::call_once(once, [&] {
+    attr = cudaFuncSetAttribute(dbst::sweep_kernel<D, RASTER, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
+  if (attr != cudaSuccess) return DBST_ECUDA;
+  const long long grid = bh_count(g) * p.pairs_per_head;
+  if (grid >= (1ll << 31)) return DBST_EINVAL;
+  // the second tensor-map argument (X2) is not read in this mode
+  dbst::sweep_kernel<D, RASTER, 3><<<static_cast<unsigned>(grid), dbst::kSweepThreads, smem, s>>>(tq, tq, tk, tv, p);
+  return launch_status();
+}
+
+dbst_status gather_common(const void* q, const void* k, const void* v, const dbst_geom* g, const uint16_t* gmask,
+                          float scale, void* o, float* lse, void* stream, bool raster) {
+  if (!geom_ok(g) || !q || !k || !v || !o || !gmask) return DBST_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (reinterpret_cast<uintptr_t>(gmask) & 1u))
+    return DBST_EINVAL;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return DBST_EINVAL;
+  if (!std::isfinite(scale)) return DBST_EINVAL;
+  if (nblocks(g) > kFineMaxNB) return DBST_EINVAL;    // group union of a pair: at most 16384 entries
+  if (raster && g->tx % 4 != 0) return DBST_EINVAL;   // a group must be 4 tokens along x
+  auto s = static_cast<cudaStream_t>(stream);
+  if (raster)
+    return g->D == 128 ? launch_gather_attn<128, true>(q, k, v, g, gmask, scale, o, lse, s)
+                       : launch_gather_attn<64, true>(q, k, v, g, gmask, scale, o, lse, s);
+  return g->D == 128 ? launch_gather_attn<128, false>(q, k, v, g, gmask, scale, o, lse, s)
+                     : launch_gather_attn<64, false>(q, k, v, g, gmask, scale, o, lse, s);
+}
+
 dbst_status offset_attn_common(const void* q, const void* k, const void* v, const dbst_geom* g, const int32_t* cnt,
                                const int16_t* idx, const float* offsets, const uint16_t* gmask, float scale, void* o,
                                float* lse, void* stream, bool raster) {
@@ -488,7 +572,6 @@ dbst_status build_mask(const void* q_tiled, const void* k_tiled, const dbst_geom
 
 // Fine mask (4-token key groups): float64 query-block and key-group means, the float64 logits of
 // every (query block, key group), then one CTA per row for the CDF selection over groups.
-constexpr int kFineMaxNB = dbst::kFineMaxGroups / 16;
 struct FineWorkspace {
   size_t qp, kp, s, total;
 };
@@ -778,6 +861,18 @@ dbst_status dbst_block_sparse_attn_groups_raster(const void* q, const void* k, c
                                                  void* stream) {
   if (!group_mask) return DBST_EINVAL;
   return offset_attn_common(q, k, v, g, kv_count, kv_idx, nullptr, group_mask, scale, o, lse, stream, true);
+}
+
+dbst_status dbst_block_sparse_attn_gather(const void* q, const void* k, const void* v, const dbst_geom* g,
+                                          const uint16_t* group_mask, float scale, void* o, float* lse,
+                                          void* stream) {
+  return gather_common(q, k, v, g, group_mask, scale, o, lse, stream, false);
+}
+
+dbst_status dbst_block_sparse_attn_gather_raster(const void* q, const void* k, const void* v, const dbst_geom* g,
+                                                 const uint16_t* group_mask, float scale, void* o, float* lse,
+                                                 void* stream) {
+  return gather_common(q, k, v, g, group_mask, scale, o, lse, stream, true);
 }
 
 dbst_status dbst_block_sparse_attn_offsets(const void* q, const void* k, const void* v, const dbst_geom* g,

@@ -355,6 +355,21 @@ dbst_status dbst_block_sparse_attn_groups_raster(const void* q, const void* k, c
                                                  void* stream);
 
 /*
+ * The same attention with the kept groups gathered, the page's own design:
+ * each 64-key tile is assembled from 16 kept 4-token groups of the union of a
+ * query-block pair's group masks (loaded by index, 4 rows at a time), so only
+ * kept groups are computed.  The group masks alone define the keys (no block
+ * lists).  NB must be at most 1024; the _raster form also needs tx divisible by
+ * 4 (a group is 4 tokens along x).
+ */
+dbst_status dbst_block_sparse_attn_gather(const void* q, const void* k, const void* v, const dbst_geom* g,
+                                          const uint16_t* group_mask, float scale, void* o, float* lse,
+                                          void* stream);
+dbst_status dbst_block_sparse_attn_gather_raster(const void* q, const void* k, const void* v, const dbst_geom* g,
+                                                 const uint16_t* group_mask, float scale, void* o, float* lse,
+                                                 void* stream);
+
+/*
  * SQuad two-pass attention (page "SQuad: Sub-Quadratic Attention Distillation
  * for Efficient Video Generation", section "Methodology: SQuad", item
  * "1. SQuad-Attention Operator").  The N tokens of each (b, h) are read as

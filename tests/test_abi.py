@@ -260,3 +260,23 @@ def test_fine_mask_and_group_attention_validate_arguments(lib):
         args = list(ok)
         args[6] = ctypes.c_void_p((1 << 20) + 1)                      # group mask not 2-byte aligned
         assert fn(*args) == dbst.DBST_EINVAL
+
+
+def test_gathered_group_attention_validates_arguments(lib):
+    g = geom()
+    a = ctypes.c_void_p(1 << 20)
+    for fn in (lib.dbst_block_sparse_attn_gather, lib.dbst_block_sparse_attn_gather_raster):
+        ok = [a, a, a, ctypes.byref(g), a, 0.0, a, None, None]
+        for i in (0, 1, 2, 4, 6):
+            args = list(ok)
+            args[i] = None
+            assert fn(*args) == dbst.DBST_EINVAL, i
+        args = list(ok)
+        args[4] = ctypes.c_void_p((1 << 20) + 1)
+        assert fn(*args) == dbst.DBST_EINVAL
+        args = list(ok)
+        args[3] = ctypes.byref(geom(grid=(8, 128, 128), tile=(1, 8, 8)))   # 2048 blocks
+        assert fn(*args) == dbst.DBST_EINVAL
+    narrow = geom(grid=(4, 16, 16), tile=(4, 8, 2))                       # tx = 2: no 4-token run along x
+    assert lib.dbst_block_sparse_attn_gather_raster(a, a, a, ctypes.byref(narrow), a, 0.0, a, None,
+                                                    None) == dbst.DBST_EINVAL

@@ -110,3 +110,29 @@ def test_group_attention_matches_oracle(built, name, p, D):
     ro, rlse = dbst.block_sparse_attn_groups(*(P.bits_to_torch(a) for a in (q, k, v)), g, cnt, idx, gm, raster=True)
     dbst.get_error()
     np.testing.assert_array_equal(O.tile_reorder(P.torch_to_bits(ro), og), P.torch_to_bits(o))
+
+
+@pytest.mark.parametrize("name,p,D", [("tiny", 0.9, 64), ("small", 0.9, 64), ("small", 0.7, 128)])
+def test_gathered_group_attention_matches_oracle(built, name, p, D):
+    """The page's design: kept groups gathered 16 to a 64-key tile by 4-row loads."""
+    w = dataclasses.replace(S.workload(name), D=D)
+    og = P.geometry(w)
+    g = gpu_geom(w)
+    q, k, v = S.make_qkv(w)
+    qt, kt, vt = (O.tile_reorder(a, og) for a in (q, k, v))
+    keep = O.build_fine_mask(qt, kt, og, p, G=4)
+    keep[0, 0, 1] = False                                     # an empty row
+    gm = torch.from_numpy(masks_from_groups(keep)).cuda()
+    o, lse = dbst.block_sparse_attn_gather(*(P.bits_to_torch(a) for a in (qt, kt, vt)), g, gm)
+    dbst.get_error()
+    ref_o, ref_lse = O.fine_masked_attention(qt, kt, vt, keep, 64, 4, 1.0 / math.sqrt(D))
+    got = S.f32_from_bf16_bits(P.torch_to_bits(o)).astype(np.float64)
+    max_abs, rel = P.attn_errors(got, ref_o)
+    assert max_abs <= P.ATTN_MAX_ABS and rel <= P.ATTN_REL_L2, (max_abs, rel)
+    lse = lse.cpu().numpy()
+    fin = np.isfinite(ref_lse)
+    assert (np.isneginf(lse) == ~fin).all()
+    assert np.abs(lse[fin] - ref_lse[fin]).max() <= P.LSE_MAX_ABS
+    ro, _ = dbst.block_sparse_attn_gather(*(P.bits_to_torch(a) for a in (q, k, v)), g, gm, raster=True)
+    dbst.get_error()
+    np.testing.assert_array_equal(O.tile_reorder(P.torch_to_bits(ro), og), P.torch_to_bits(o))
