@@ -432,6 +432,36 @@ def measure_step(args, name: str) -> dict:
             "step_tflops": flops / ((mask_ms + attn_ms) * 1e-3) / 1e12}
 
 
+def measure_fine(args, w, p, qkv=None) -> dict:
+    """Fine-grained 4-token key groups on one workload: the group mask, then the attention over the
+    kept groups, on whole blocks with the other groups masked and gathered 16 groups to a tile."""
+    import torch
+    import dynamic_block_sparse_tile_b200 as dbst
+    dbst.load()
+    g = dbst.Geom.make(w.B, w.H, w.D, w.grid, w.tile)
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()   # noqa: E731
+    q, k, v = qkv if qkv is not None else (to_dev(a) for a in S.make_qkv(w))
+    ws = torch.empty(dbst.fine_mask_workspace_bytes(g), dtype=torch.uint8, device="cuda")
+    mask = dbst.build_fine_mask(q, k, g, p, raster=True, workspace=ws)
+    o = torch.empty_like(q)
+    lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device="cuda")
+    mask_ms = timed_median(lambda: dbst.build_fine_mask(q, k, g, p, raster=True, workspace=ws, out=mask),
+                           args.steps, args.warmup)
+    blocks_ms = timed_median(lambda: dbst.block_sparse_attn_groups(q, k, v, g, mask[1], mask[2], mask[0], raster=True,
+                                                                   out=o, lse=lse), args.steps, args.warmup)
+    gather_ms = timed_median(lambda: dbst.block_sparse_attn_gather(q, k, v, g, mask[0], raster=True, out=o, lse=lse),
+                             args.steps, args.warmup)
+    dbst.get_error()
+    gm = mask[0].cpu().numpy().view(np.uint16)
+    kept_groups = int(np.unpackbits(gm.view(np.uint8)).sum())
+    ng = g.N // 4
+    flops = 4.0 * w.D * 64 * 4 * kept_groups          # 64 queries x 4 keys per kept (query block, group)
+    return {"fine": workload_desc(w, p), "kept_group_fraction": kept_groups / (g.B * g.H * g.NB * ng),
+            "kept_block_fraction": int(mask[1].sum().item()) / (g.B * g.H * g.NB * g.NB), "mask_ms": mask_ms,
+            "attn_whole_blocks_ms": blocks_ms, "attn_gathered_ms": gather_ms,
+            "gathered_tflops_on_kept_groups": flops / (gather_ms * 1e-3) / 1e12}
+
+
 def measure_squad(args) -> dict:
     """SQuad two-pass attention against dense attention on the same tensors (B=2 H=16 N=16384 D=128,
     w = sqrt(N) = 128)."""
@@ -478,6 +508,8 @@ def main():
     ap.add_argument("--no-extensions", action="store_true",
                     help="skip the extension measurements (backward, SIP, SQuad, the 2x4x8-tile Wan variant) "
                          "after the timed step, e.g. under a profiler's launch list")
+    ap.add_argument("--fine", action="store_true",
+                    help="time the 4-token key-group mask and attention (whole blocks, and gathered groups)")
     ap.add_argument("--sip", action="store_true",
                     help="time the SIP sampled mask and the attention with inclusion-probability offsets")
     ap.add_argument("--backward", action="store_true",
@@ -497,6 +529,9 @@ def main():
         return run_squad(args)
     if args.sip:
         return run_sip(args, w, p)
+    if args.fine:
+        print(json.dumps(measure_fine(args, w, p)), flush=True)
+        return 0
 
     import torch
     import torch.distributed as dist
