@@ -8,8 +8,8 @@ arithmetic is float64.  Library primitives used as steps: ``numpy.matmul``,
 
 Readings adopted where the page is silent, ambiguous or garbled:
 
-R1  CDF threshold ("Seuil CDF").  The page keeps the blocks "where the
-    cumulative probability exceeds a threshold (1 - thr)".  Read with the
+R1  CDF threshold ("Seuil CDF").  The page thresholds the row's cumulative
+    probability at 1 - thr without fixing the sort direction.  Read with the
     row sorted ascending and cumulative mass c_j up to and including block j,
     block j is kept iff c_j > 1 - p.  Equivalently (and this is the form
     computed here): sort the row descending, ties to the lower key-block
