@@ -14,7 +14,7 @@ Sources (cited by page title and section):
   the per-row CDF threshold ("Seuil CDF"), expansion of the block mask
   ("Expansion") and the union with Sliding Tile Attention ("Intégration
   Hybride avec STA"); the lay section "L'ancienne solution" describes STA as
-  a tile attending to itself and the immediately adjacent tiles.
+  a tile attending to itself and its direct neighbours.
 * "AB-Attention accélère la génération vidéo…" (news.hamidun.com), section
   "Les trois techniques": the kernel gathers the selected key/value blocks
   by index, which is why the mask is also emitted as per-row index lists.

@@ -24,7 +24,7 @@ R4  p must lie in (0, 1]; every row then keeps at least one block.
 R5  A query block with no kept key block (only possible with a mask the
     caller supplies) produces output 0 and log-sum-exp -inf.
 R6  Sliding-tile neighbourhood ("Intégration Hybride avec STA"; the lay
-    section describes the own tile plus the immediately adjacent tiles):
+    section describes the own tile plus its direct neighbours):
     key tile j is a neighbour of query tile i iff the Chebyshev distance of
     their tile coordinates is <= r, clipped at the grid edges (no wrap, no
     shifting of the window).
