@@ -462,6 +462,19 @@ def measure_fine(args, w, p, qkv=None) -> dict:
             "gathered_tflops_on_kept_groups": flops / (gather_ms * 1e-3) / 1e12}
 
 
+def measure_dense(args, w, qkv) -> dict:
+    """Dense attention from the same library on the same raster tensors (the comparator)."""
+    import torch
+    import dynamic_block_sparse_tile_b200 as dbst
+    g = dbst.Geom.make(w.B, w.H, w.D, w.grid, w.tile)
+    q, k, v = qkv
+    dense_ms = timed_median(lambda: dbst.dense_attn_raster(q, k, v, g), args.steps, args.warmup)
+    dbst.get_error()
+    flops = 4.0 * w.D * w.N * w.N * w.B * w.H
+    return {"workload": workload_desc(w, float("nan")), "dense_attn_ms": dense_ms,
+            "dense_tflops": flops / (dense_ms * 1e-3) / 1e12}
+
+
 def measure_squad(args) -> dict:
     """SQuad two-pass attention against dense attention on the same tensors (B=2 H=16 N=16384 D=128,
     w = sqrt(N) = 128)."""
@@ -718,7 +731,8 @@ def main():
         # The rows built on top of the path, each timed on its own after the step above (outside its
         # timed region and launch count); a failure is recorded here and cannot touch the line.
         ext = {}
-        for name, fn in (("backward", lambda: measure_backward(args, w, p, (q, k, v))),
+        for name, fn in (("dense_same_shape", lambda: measure_dense(args, w, (q, k, v))),
+                         ("backward", lambda: measure_backward(args, w, p, (q, k, v))),
                          ("sip", lambda: measure_sip(args, w, p, (q, k, v))),
                          ("squad", lambda: measure_squad(args)),
                          ("wan_tiles_2x4x8", lambda: measure_step(args, "wan_2x4x8"))):
