@@ -464,7 +464,6 @@ def measure_fine(args, w, p, qkv=None) -> dict:
 
 def measure_dense(args, w, qkv) -> dict:
     """Dense attention from the same library on the same raster tensors (the comparator)."""
-    import torch
     import dynamic_block_sparse_tile_b200 as dbst
     g = dbst.Geom.make(w.B, w.H, w.D, w.grid, w.tile)
     q, k, v = qkv
