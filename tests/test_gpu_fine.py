@@ -2,9 +2,6 @@
 techniques", third technique: key groups of 4 tokens) against the float64
 oracle ``oracle.fine``.
 
-Marked ``unverified``: these kernels have not yet run on a B200, so the tests
-are kept out of ``-m gpu`` until they have; run them with ``-m unverified``.
-
 Selection: the kept groups must match the oracle's, a disagreement being
 excused only where the oracle's cumulative pooled mass at that group's rank,
 or the rank before it, lies within 1e-4 of p (the rule of the block mask).
@@ -22,7 +19,7 @@ import oracle as O
 import dynamic_block_sparse_tile_b200 as dbst
 from tests import parity as P
 
-pytestmark = pytest.mark.unverified
+pytestmark = pytest.mark.gpu
 
 
 @pytest.fixture(scope="module")

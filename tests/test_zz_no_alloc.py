@@ -52,12 +52,17 @@ def test_noalloc_matches_regular_entry_point_twice(lib, name, p, sta, heads):
     for call in range(2):
         out = (torch.full_like(torch.from_numpy(ref[0]), -1).cuda(), torch.full_like(torch.from_numpy(ref[1]), -1).cuda(),
                torch.full_like(torch.from_numpy(ref[2]), -1).cuda())
+        torch.cuda.synchronize()
+        before = (torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated(), torch.cuda.memory_reserved())
         status = lib.dbst_build_block_mask_noalloc(
             ctypes.c_void_p(qt.data_ptr()), ctypes.c_void_p(kt.data_ptr()), ctypes.byref(g), ctypes.c_float(p),
             ctypes.c_int(sta), ctypes.c_void_p(out[0].data_ptr()), ctypes.c_void_p(out[1].data_ptr()),
             ctypes.c_void_p(out[2].data_ptr()), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
         assert status == dbst.DBST_OK, status
         dbst.get_error()
+        # nothing was allocated: the device's free memory (cudaMemGetInfo) and torch's pools are as before
+        after = (torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated(), torch.cuda.memory_reserved())
+        assert after == before, f"call {call}: device memory changed from {before} to {after}"
         bits, cnt, idx = (t.cpu().numpy() for t in out)
         np.testing.assert_array_equal(bits, ref[0], err_msg=f"call {call}: mask bits")
         np.testing.assert_array_equal(cnt, ref[1], err_msg=f"call {call}: kv_count")
