@@ -23,7 +23,7 @@ __all__ = ["Geom", "DbstError", "lib_path", "load", "tile_reorder", "tile_unreor
            "transpose_block_mask", "attn_backward_workspace_bytes", "block_sparse_attn_backward",
            "squad_workspace_bytes", "squad_attn", "build_sip_mask", "block_sparse_attn_offsets",
            "fine_mask_workspace_bytes", "build_fine_mask", "block_sparse_attn_groups", "block_sparse_attn_gather",
-           "get_error", "EXPORTS"]
+           "get_error", "set_wait_limit", "EXPORTS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libdbst.so")
@@ -38,7 +38,7 @@ EXPORTS = ("dbst_status_string", "dbst_tile_reorder", "dbst_tile_unreorder", "db
            "dbst_build_sip_mask", "dbst_build_sip_mask_raster", "dbst_block_sparse_attn_offsets",
            "dbst_block_sparse_attn_offsets_raster", "dbst_fine_mask_workspace_bytes", "dbst_build_fine_mask",
            "dbst_build_fine_mask_raster", "dbst_block_sparse_attn_groups", "dbst_block_sparse_attn_groups_raster",
-           "dbst_block_sparse_attn_gather", "dbst_block_sparse_attn_gather_raster")
+           "dbst_block_sparse_attn_gather", "dbst_block_sparse_attn_gather_raster", "dbst_set_wait_limit")
 
 DBST_OK, DBST_EINVAL, DBST_ECUDA, DBST_ETIMEOUT, DBST_EBOUNDS, DBST_ETOOLARGE = 0, 1, 2, 3, 4, 5
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -133,6 +133,7 @@ def load() -> ctypes.CDLL:
     for name in ("dbst_block_sparse_attn_groups", "dbst_block_sparse_attn_groups_raster"):
         getattr(lib, name).argtypes = [vp, vp, vp, gp, vp, vp, vp, f32, vp, vp, vp]
         getattr(lib, name).restype = i32
+    lib.dbst_set_wait_limit.argtypes, lib.dbst_set_wait_limit.restype = [ctypes.c_longlong], None
     _lib = lib
     return lib
 
@@ -509,3 +510,8 @@ def squad_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, w: int, scale:
 def get_error() -> None:
     """Synchronise the current stream and raise if a kernel recorded an error."""
     _check(load().dbst_get_error(_stream()), "device")
+
+
+def set_wait_limit(cycles: int) -> None:
+    """Limit (SM cycles) of the attention kernels' waits between roles (``dbst_set_wait_limit``); <= 0: default."""
+    load().dbst_set_wait_limit(int(cycles))

@@ -28,6 +28,14 @@
 //   warp 13     TMA producer of Q and the K ring (lane 0)
 //   warp 14     TMA producer of the V ring (lane 0); a warp of its own, so that its waits for
 //               free V slots never hold up the K loads
+//
+// Waits between roles are bounded by a run-time limit (PairParams::wait_limit, default about one
+// second); one that runs out records DBST_ETIMEOUT and the CTA abandons its work: producers stop
+// issuing, the softmax roles run out their loops without waiting, and each role waits (with the
+// default limit) for the copies and products it issued itself before the CTA frees TMEM and exits.
+//
+// CTAs run in grid order: head by head, each head's pairs in the order of the pair list (the
+// pairing lists them longest first, so the short pairs fill the end of the launch).
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -54,6 +62,7 @@ struct PairParams {
   int pair_stride;           // without a pair list: qb = qa + pair_stride
   int pairs_per_head;
   float scale_log2;          // softmax scale * log2(e)
+  long long wait_limit;      // cycles a wait between roles may take before the CTA gives up (0: default)
   TileGeo tg;                // token grid and tile shape (raster layout only)
 };
 
@@ -123,6 +132,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   uint32_t* s_misc = reinterpret_cast<uint32_t*>(sm + PairSmem::kMisc);
   volatile uint32_t* s_abort = s_misc + 2;
   auto bar = [&](int slot) -> uint32_t { return sbase + PairSmem::kBars + 8u * slot; };
+  // limit of a wait between roles; read only on a wait's slow path, so it holds no register in the loops
+  auto limit = [&]() -> long long { return prm.wait_limit > 0 ? prm.wait_limit : kWaitLimitCycles; };
   // Bounded wait used inside the softmax loops.  The abort flag is read only when the phase is
   // not already complete, so a wait that succeeds at once costs one barrier test; `live` turns
   // false for good once this warp times out or sees another role's abort, and later waits are
@@ -132,7 +143,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const long long t0 = clock64();
     while (!mbar_try(mb, parity)) {
       if (*s_abort) { live = false; return; }
-      if (clock64() - t0 > kWaitLimitCycles) {
+      if (clock64() - t0 > limit()) {
         record_error(kErrTimeout);
         *s_abort = 1;
         live = false;
@@ -298,7 +309,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       for (int t = 0; t < T; ++t) {
         if (*s_abort) break;
         const int s = t % slots;
-        if (t >= slots && !mbar_wait(bar(empty0 + s), ((t / slots) - 1) & 1)) {
+        if (t >= slots && !mbar_wait_lim(bar(empty0 + s), ((t / slots) - 1) & 1, limit())) {
           *s_abort = 1;
           break;
         }
@@ -324,7 +335,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const uint64_t dK = smem_desc(sbase + PairSmem::kK, 16, 1024);
     const uint64_t dV = smem_desc(sbase + PairSmem::kV, 16384, 1024);
     auto wait_all = [&](int slot, uint32_t parity) -> bool {
-      return __all_sync(0xffffffffu, mbar_wait(bar(slot), parity));
+      return __all_sync(0xffffffffu, mbar_wait_lim(bar(slot), parity, limit()));
     };
     // S(t) -> S buffer t&1, once the softmax has read S(t-2) out of it.
     auto issue_s = [&](int t) -> bool {

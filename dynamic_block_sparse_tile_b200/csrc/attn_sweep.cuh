@@ -98,6 +98,7 @@ struct SweepParams {
   int pairs_per_head;
   float scale_log2;          // softmax scale * log2 e
   float scale;               // softmax scale
+  long long wait_limit;      // cycles a wait between roles may take before the CTA gives up (0: default)
   TileGeo tg;                // token grid and tile shape (raster layout only)
 };
 
@@ -198,12 +199,15 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
   uint32_t* s_misc = reinterpret_cast<uint32_t*>(sm + L::kMisc);
   volatile uint32_t* s_abort = s_misc + 2;
   auto bar = [&](int slot) -> uint32_t { return sbase + L::kBars + 8u * slot; };
+  // waits between roles run out after `limit` cycles; the drains of a CTA's own copies and
+  // products keep the default limit
+  const long long limit = prm.wait_limit > 0 ? prm.wait_limit : kWaitLimitCycles;
   auto wait_live = [&](uint32_t mb, uint32_t parity, bool& live) {
     if (!live || mbar_try(mb, parity)) return;
     const long long t0 = clock64();
     while (!mbar_try(mb, parity)) {
       if (*s_abort) { live = false; return; }
-      if (clock64() - t0 > kWaitLimitCycles) {
+      if (clock64() - t0 > limit) {
         record_error(kErrTimeout);
         *s_abort = 1;
         live = false;
@@ -385,7 +389,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
       if (lane == 0) {
         if (*s_abort) {
           ok = 0;
-        } else if (v >= kSweepSlots && !mbar_wait(bar(BB_REMPTY + s), ((v / kSweepSlots) - 1) & 1)) {
+        } else if (v >= kSweepSlots && !mbar_wait_lim(bar(BB_REMPTY + s), ((v / kSweepSlots) - 1) & 1, limit)) {
           *s_abort = 1;
           ok = 0;
         } else {
@@ -420,7 +424,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
       for (int t = 0; t < NV; ++t) {
         if (*s_abort) break;
         const int s = t % kSweepSlots;
-        if (t >= kSweepSlots && !mbar_wait(bar(BB_REMPTY + s), ((t / kSweepSlots) - 1) & 1)) {
+        if (t >= kSweepSlots && !mbar_wait_lim(bar(BB_REMPTY + s), ((t / kSweepSlots) - 1) & 1, limit)) {
           *s_abort = 1;
           break;
         }
@@ -451,7 +455,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
     const uint64_t dRingK = smem_desc(sbase + L::kRing, 16, 1024);
     const uint64_t dRingMN = smem_desc(sbase + L::kRing, 8192, 1024);
     auto wait_all = [&](int slot, uint32_t parity) -> bool {
-      return __all_sync(0xffffffffu, mbar_wait(bar(slot), parity));
+      return __all_sync(0xffffffffu, mbar_wait_lim(bar(slot), parity, limit));
     };
     auto issue_ss = [&](int t) -> bool {
       const int s = t % kSweepSlots, b = t & 1;

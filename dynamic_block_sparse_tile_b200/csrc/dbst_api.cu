@@ -7,8 +7,10 @@
 
 #include <cmath>
 #include <cstdint>
+#include <atomic>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/dbst.h"
 #include "attn_sweep.cuh"
@@ -47,15 +49,41 @@ long long tokens(const dbst_geom* g) { return static_cast<long long>(g->T) * g->
 int nblocks(const dbst_geom* g) { return static_cast<int>(tokens(g) / 64); }
 long long bh_count(const dbst_geom* g) { return static_cast<long long>(g->B) * g->H; }
 
+// Multiprocessors of the current device (the library may drive several devices from one process).
 int sm_count() {
-  static int n = 0;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      n = 148;
-  });
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      n < 1)
+    n = 148;
   return n;
+}
+
+// The opt-in to more than 48 KB of dynamic shared memory is a property of a kernel on one device:
+// it is set once per (device, kernel) and remembered.
+constexpr int kMaxDevices = 64;
+bool smem_opt_in(const void* kernel, int bytes) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  struct Entry { const void* fn; int bytes; };
+  static std::mutex mu;
+  static std::vector<Entry> done[kMaxDevices];
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry& e : done[dev])
+    if (e.fn == kernel && e.bytes >= bytes) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  done[dev].push_back({kernel, bytes});
+  return true;
+}
+template <typename K>
+bool smem_opt_in(K* kernel, int bytes) {
+  return smem_opt_in(reinterpret_cast<const void*>(kernel), bytes);
+}
+
+// Limit of the waits between a kernel's roles, in SM clock cycles (dbst_set_wait_limit); 0 = default.
+std::atomic<long long> g_wait_limit{0};
+long long wait_limit() {
+  const long long v = g_wait_limit.load(std::memory_order_relaxed);
+  return v > 0 ? v : dbst::kWaitLimitCycles;
 }
 
 dbst::TileGeo tile_geo(const dbst_geom* g) {
@@ -219,13 +247,9 @@ dbst_status launch_pair(const void* q, const void* k, const void* v, const dbst_
   p.pairs_per_head = pairs ? (p.NB + 1) / 2 : ((p.NB + 2 * p.pair_stride - 1) / (2 * p.pair_stride)) * p.pair_stride;
   const float sc = scale > 0.0f ? scale : 1.0f / std::sqrt(static_cast<float>(D));
   p.scale_log2 = sc * 1.4426950408889634f;
+  p.wait_limit = wait_limit();
   const int smem = dbst::PairSmem::kBytes + 1024;
-  static std::once_flag once;
-  static cudaError_t attr = cudaSuccess;
-  std::call_once(once, [&] {
-    attr = cudaFuncSetAttribute(dbst::pair_attn_kernel<D, RASTER>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  });
-  if (attr != cudaSuccess) return DBST_ECUDA;
+  if (!smem_opt_in(dbst::pair_attn_kernel<D, RASTER>, smem)) return DBST_ECUDA;
   const long long grid = bh_count(g) * p.pairs_per_head;
   if (grid >= (1ll << 31)) return DBST_EINVAL;
   dbst::pair_attn_kernel<D, RASTER><<<static_cast<unsigned>(grid), dbst::kPairThreads, smem, s>>>(tq, tk, tv, p);
@@ -280,15 +304,10 @@ dbst_status launch_bwd(const void* q, const void* k, const void* v, const float*
   const float sc = scale > 0.0f ? scale : 1.0f / std::sqrt(static_cast<float>(D));
   p.scale = sc;
   p.scale_log2 = sc * 1.4426950408889634f;
+  p.wait_limit = wait_limit();
   const int smem = dbst::SweepSmem::kBytes + 1024;
-  static std::once_flag once;
-  static cudaError_t attr = cudaSuccess;
-  std::call_once(once, [&] {
-    attr = cudaFuncSetAttribute(dbst::sweep_kernel<D, RASTER, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (attr == cudaSuccess)
-      attr = cudaFuncSetAttribute(dbst::sweep_kernel<D, RASTER, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  });
-  if (attr != cudaSuccess) return DBST_ECUDA;
+  if (!smem_opt_in(dbst::sweep_kernel<D, RASTER, 0>, smem) || !smem_opt_in(dbst::sweep_kernel<D, RASTER, 1>, smem))
+    return DBST_ECUDA;
   const long long grid = bh_count(g) * p.pairs_per_head;
   if (grid >= (1ll << 31)) return DBST_EINVAL;
   p.count = kv_count;
@@ -388,13 +407,9 @@ dbst_status launch_offset_attn(const void* q, const void* k, const void* v, cons
   const float sc = scale > 0.0f ? scale : 1.0f / std::sqrt(static_cast<float>(D));
   p.scale = sc;
   p.scale_log2 = sc * 1.4426950408889634f;
+  p.wait_limit = wait_limit();
   const int smem = dbst::SweepSmem::kBytes + 1024;
-  static std::once_flag once;
-  static cudaError_t attr = cudaSuccess;
-  std::call_once(once, [&] {
-    attr = cudaFuncSetAttribute(dbst::sweep_kernel<D, RASTER, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  });
-  if (attr != cudaSuccess) return DBST_ECUDA;
+  if (!smem_opt_in(dbst::sweep_kernel<D, RASTER, 2>, smem)) return DBST_ECUDA;
   const long long grid = bh_count(g) * p.pairs_per_head;
   if (grid >= (1ll << 31)) return DBST_EINVAL;
   // the second tensor-map argument (X2) is not read in this mode
@@ -427,13 +442,9 @@ dbst_status launch_gather_attn(const void* q, const void* k, const void* v, cons
   const float sc = scale > 0.0f ? scale : 1.0f / std::sqrt(static_cast<float>(D));
   p.scale = sc;
   p.scale_log2 = sc * 1.4426950408889634f;
+  p.wait_limit = wait_limit();
   const int smem = dbst::SweepLayout<3>::kBytes + 1024;
-  static std::once_flag once;
-  static cudaError_t attr = cudaSuccess;
-  std::call_once(once, [&] {
-    attr = cudaFuncSetAttribute(dbst::sweep_kernel<D, RASTER, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  });
-  if (attr != cudaSuccess) return DBST_ECUDA;
+  if (!smem_opt_in(dbst::sweep_kernel<D, RASTER, 3>, smem)) return DBST_ECUDA;
   const long long grid = bh_count(g) * p.pairs_per_head;
   if (grid >= (1ll << 31)) return DBST_EINVAL;
   // the second tensor-map argument (X2) is not read in this mode
@@ -480,9 +491,7 @@ template <int NPT>
 bool launch_select(const double* S, const dbst::SelectGeo& sg, long long rows, uint32_t* bits, int32_t* cnt,
                    int16_t* idx, cudaStream_t s) {
   const int smem = 256 * NPT * 16;   // sort keys + masses
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(dbst::select_kernel<NPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return false;
+  if (smem > 48 * 1024 && !smem_opt_in(dbst::select_kernel<NPT>, smem)) return false;
   dbst::select_kernel<NPT><<<static_cast<unsigned>(rows), 256, smem, s>>>(S, sg, bits, cnt, idx);
   return true;
 }
@@ -766,9 +775,7 @@ dbst_status dbst_pair_query_blocks(const uint32_t* mask_bits, const dbst_geom* g
   const bool stage = dbst::pairing_rows_bytes(pg.NB, pg.NW) <= static_cast<size_t>(dbst::kPairingStageBytes);
   const size_t smem = dbst::pairing_smem_bytes(pg.NB, pg.NW, stage);
   auto kern = stage ? dbst::pair_blocks_kernel<true> : dbst::pair_blocks_kernel<false>;
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
-    return DBST_ECUDA;
+  if (smem > 48 * 1024 && !smem_opt_in(kern, static_cast<int>(smem))) return DBST_ECUDA;
   kern<<<static_cast<unsigned>(bh), dbst::kPairingThreads, smem, static_cast<cudaStream_t>(stream)>>>(mask_bits, pg,
                                                                                                      pairs);
   return launch_status();
@@ -922,6 +929,8 @@ dbst_status dbst_squad_attn(const void* q, const void* k, const void* v, int B, 
   return window_transpose(o_loc, o, heads, w, m, D, s);
 }
 
+void dbst_set_wait_limit(long long cycles) { g_wait_limit.store(cycles > 0 ? cycles : 0, std::memory_order_relaxed); }
+
 dbst_status dbst_get_error(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DBST_ECUDA;
   unsigned int word = 0;
@@ -945,7 +954,6 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[DBST_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 

@@ -19,7 +19,9 @@
 // running them alone), with one single block when their count is odd.
 //
 // Output pairs[bh][e], e < ceil(NB/2): qa | qb << 16, qb = 0xFFFF for a single
-// block; matched pairs first (by lower block index), then the leftover pairs.
+// block, longest first: by the pair's tiles ceil(|A u B| / 2) descending, ties
+// by the order of construction (matched pairs by lower block index, then the
+// leftover pairs).  The attention kernel starts the longest items first.
 #pragma once
 #include <cstdint>
 #include "ptx.cuh"
@@ -192,6 +194,36 @@ __global__ void __launch_bounds__(kPairingThreads) pair_blocks_kernel(const uint
       }
       ++fi;
     }
+  }
+  __syncthreads();
+
+  // longest first: each pair's tiles, then its rank (tiles descending, construction order on ties)
+  const int npairs = (NB + 1) / 2;
+  int* ent = weight;              // the edge weights are no longer needed: 6 NB >= 2 npairs ints
+  int* cost = weight + npairs;
+  for (int e = tid; e < npairs; e += kPairingThreads) {
+    const int32_t x = out[e];
+    const int a = x & 0xFFFF, b = (x >> 16) & 0xFFFF;
+    int un = 0;
+    const uint32_t* ra = head + static_cast<long long>(a) * g.NW;
+    if (b == 0xFFFF) {
+      un = count[a];
+    } else {
+      const uint32_t* rb = head + static_cast<long long>(b) * g.NW;
+      for (int w = 0; w < g.NW; ++w) un += __popc(ra[w] | rb[w]);
+    }
+    ent[e] = x;
+    cost[e] = (un + 1) / 2;
+  }
+  __syncthreads();
+  for (int e = tid; e < npairs; e += kPairingThreads) {
+    const int c = cost[e];
+    int rank = 0;
+    for (int f = 0; f < npairs; ++f) {
+      const int cf = cost[f];
+      rank += (cf > c) || (cf == c && f < e);
+    }
+    out[rank] = ent[e];
   }
 }
 

@@ -164,10 +164,15 @@ dbst_status dbst_dense_attn_raster(const void* q, const void* k, const void* v, 
  *   mask_bits : [B,H,NB,ceil(NB/32)] uint32 as written by the mask builders
  *   pairs     : out, [B,H,ceil(NB/2)] int32, entry = qa | qb << 16 with
  *               qb = 0xFFFF for a single block; every block of a head appears
- *               exactly once.  4-byte aligned.
+ *               exactly once.  Each head's entries come longest first (by
+ *               the pair's tiles, ceil(|union| / 2), descending): the
+ *               attention kernel starts the longest pairs first.  4-byte
+ *               aligned.
  * Pass `pairs` to dbst_block_sparse_attn_raster (NULL there selects fixed
- * pairs of neighbours one tile step apart).  An entry naming a block outside
- * [0, NB) makes the attention skip that entry and report DBST_EBOUNDS.
+ * pairs of neighbours one tile step apart).  Any order of a head's entries
+ * gives the same results; the attention only schedules by it.  An entry
+ * naming a block outside [0, NB) makes the attention skip that entry and
+ * report DBST_EBOUNDS.
  */
 dbst_status dbst_pair_query_blocks(const uint32_t* mask_bits, const dbst_geom* g, int32_t* pairs, void* stream);
 
@@ -396,6 +401,18 @@ dbst_status dbst_squad_attn(const void* q, const void* k, const void* v, int B, 
  * CUDA error.  DBST_OK if there was none.
  */
 dbst_status dbst_get_error(void* stream);
+
+/*
+ * Diagnostic knob (no counterpart on the pages): the limit, in SM clock
+ * cycles, of the waits between the roles inside the attention kernels (forward
+ * and backward) launched after this call by this process.  A wait that runs
+ * out records DBST_ETIMEOUT, the kernel abandons its work (after waiting, with
+ * the default limit of about one second, for the copies and tensor-core
+ * products it has already issued) and its outputs are undefined.  cycles <= 0
+ * restores the default.  It exists so that tests can make a bounded wait
+ * expire without faulting anything; production callers leave it alone.
+ */
+void dbst_set_wait_limit(long long cycles);
 
 #ifdef __cplusplus
 }
