@@ -6,7 +6,8 @@ N=37632, 588 blocks; CDF threshold p=0.9; seeded synthetic q/k/v).  Default
 (`--path fused`): raster q, k, v in, raster o out, the tile reorder done by the
 kernels' own loads and stores:
     build_block_mask_raster(q, k) -> pair_query_blocks -> block_sparse_attn_raster(q, k, v, pairs) -> o
-(5 launches: pool, pooled logits, select, query-block pairing, attention).  `--path explicit` runs
+(6 launches: a memset and three kernels for the mask (block means, pooled logits on the tensor cores,
+row selection), the query-block pairing, the attention).  `--path explicit` runs
 the same steps as separate passes (8 launches):
     tile_reorder(q, k, v) -> build_block_mask -> block_sparse_attn -> tile_unreorder(o)
 
@@ -276,6 +277,11 @@ def timed_median(fn, steps: int, warmup: int) -> float:
 
 
 def run_sweep(args, w):
+    print(json.dumps(measure_sweep(args, w)), flush=True)
+    return 0
+
+
+def measure_sweep(args, w) -> dict:
     """Attention time and kept-block TFLOP/s against the kept fraction; dense attention at the same shape."""
     import torch
     import dynamic_block_sparse_tile_b200 as dbst
@@ -310,11 +316,11 @@ def run_sweep(args, w):
     for r in rows:
         r["speedup_vs_dense"] = dense_ref / r["sparse_attn_ms"]
     crossover = next((r["kept_fraction"] for r in rows if r["sparse_attn_ms"] >= dense_ref), None)
-    out = {"sweep": workload_desc(w, float("nan")), "dense_attn_ms": dense_ms, "dense_attn_ms_end": dense_end_ms,
-           "dense_tflops": dense_flops / (dense_ms * 1e-3) / 1e12, "peak_source": src, "points": rows,
-           "dense_crossover_kept_fraction": crossover}
-    print(json.dumps(out), flush=True)
-    return 0
+    return {"sweep": workload_desc(w, float("nan")), "dense_attn_ms": dense_ms, "dense_attn_ms_end": dense_end_ms,
+            "dense_tflops": dense_flops / (dense_ms * 1e-3) / 1e12, "peak_source": src, "points": rows,
+            "dense_crossover_kept_fraction": crossover,
+            "crossover_note": "kept fraction of the first p whose sparse attention is no faster than dense; "
+                              "null: sparse is faster at every p of the sweep, p = 1 (every block kept) included"}
 
 
 def measure_backward(args, w, p, qkv=None) -> dict:
@@ -416,20 +422,22 @@ def measure_step(args, name: str) -> dict:
     o = torch.empty_like(q)
     lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device="cuda")
 
-    def mask_and_pairs():
-        dbst.build_block_mask_raster(q, k, g, p, w.sta_radius, workspace=ws, out=mask)
-        dbst.pair_query_blocks(mask[0], g, out=pairs)
-
-    mask_ms = timed_median(mask_and_pairs, args.steps, args.warmup)
+    mask_ms = timed_median(lambda: dbst.build_block_mask_raster(q, k, g, p, w.sta_radius, workspace=ws, out=mask),
+                           args.steps, args.warmup)
+    pairing_ms = timed_median(lambda: dbst.pair_query_blocks(mask[0], g, out=pairs), args.steps, args.warmup)
     attn_ms = timed_median(lambda: dbst.block_sparse_attn_raster(q, k, v, g, mask[1], mask[2], 0.0, True, o, lse,
                                                                  pairs), args.steps, args.warmup)
     dbst.get_error()
     kept = int(mask[1].sum().item())
     flops = 4.0 * w.D * 64 * 64 * kept
+    hbm, bf16, _, src = peaks()
+    mask_gbs = 2 * w.B * w.H * w.N * w.D * 2 / (mask_ms * 1e-3) / 1e9
     return {"workload": workload_desc(w, p), "kept_fraction": kept / (g.B * g.H * g.NB * g.NB),
-            "mask_and_pairing_ms": mask_ms, "sparse_attn_ms": attn_ms,
+            "mask_build_ms": mask_ms, "mask_build_gbs": mask_gbs, "mask_frac_of_hbm": mask_gbs / hbm,
+            "pairing_ms": pairing_ms, "sparse_attn_ms": attn_ms,
             "sparse_attn_tflops": flops / (attn_ms * 1e-3) / 1e12,
-            "step_tflops": flops / ((mask_ms + attn_ms) * 1e-3) / 1e12}
+            "sparse_attn_frac_of_bf16_peak": flops / (attn_ms * 1e-3) / 1e12 / bf16, "peak_source": src,
+            "step_tflops": flops / ((mask_ms + pairing_ms + attn_ms) * 1e-3) / 1e12}
 
 
 def measure_fine(args, w, p, qkv=None) -> dict:
@@ -581,7 +589,7 @@ def main():
     stream = torch.cuda.current_stream()
     fused = args.path == "fused"
     # fused: pool + logits + select + pairing + attention; explicit: 3 reorders + 4 + unreorder
-    launches_per_step = 5 if fused else 8
+    launches_per_step = 5 if fused else 8   # kernels of this library (the memset is the runtime's)
     pairs = torch.empty((g.B, g.H, (g.NB + 1) // 2), dtype=torch.int32, device="cuda")
 
     ev = {}
@@ -598,9 +606,13 @@ def main():
             e0.record(stream)
         if fused:
             dbst.build_block_mask_raster(q_, k_, g, p, w.sta_radius, workspace=ws, out=(bits, cnt, idx))
-            dbst.pair_query_blocks(bits, g, out=pairs)
         else:
             dbst.build_block_mask(qt, kt, g, p, w.sta_radius, workspace=ws, out=(bits, cnt, idx))
+        if timed_parts:
+            em = torch.cuda.Event(enable_timing=True)
+            em.record(stream)
+        if fused:
+            dbst.pair_query_blocks(bits, g, out=pairs)
         if timed_parts:
             e1 = torch.cuda.Event(enable_timing=True)
             e1.record(stream)
@@ -611,7 +623,7 @@ def main():
         if timed_parts:
             e2 = torch.cuda.Event(enable_timing=True)
             e2.record(stream)
-            ev.setdefault("parts", []).append((e0, e1, e2))
+            ev.setdefault("parts", []).append((e0, e1, e2, em))
         if not fused:
             dbst.tile_unreorder(ot, g, out=o_)
 
@@ -639,8 +651,9 @@ def main():
     clk = clocks.stop()
     dbst.get_error()
     ms_total = start.elapsed_time(end)
-    mask_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev["parts"])
-    attn_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev["parts"])
+    mask_ms = statistics.mean(a.elapsed_time(m) for a, _, _, m in ev["parts"])      # mask build alone
+    pairing_ms = statistics.mean(m.elapsed_time(b) for _, b, _, m in ev["parts"])   # query-block pairing
+    attn_ms = statistics.mean(b.elapsed_time(c) for _, b, c, _ in ev["parts"])
 
     # End to end, as a serving loop runs it: every step copies its inputs in from pinned host
     # memory and its output back out, and the copies of neighbouring steps overlap this step's
@@ -695,7 +708,8 @@ def main():
     e2e_ms = s2.elapsed_time(e2)
     dbst.get_error()
 
-    ms_total, e2e_ms, attn_ms, mask_ms = max_over_ranks([ms_total, e2e_ms, attn_ms, mask_ms], world, "cuda")
+    ms_total, e2e_ms, attn_ms, mask_ms, pairing_ms = max_over_ranks([ms_total, e2e_ms, attn_ms, mask_ms, pairing_ms],
+                                                                    world, "cuda")
     ms_step = ms_total / args.steps
     value = job_tflops(world, flops, ms_step)
     e2e_value = job_tflops(world, flops, e2e_ms / args.steps)
@@ -713,6 +727,7 @@ def main():
                            "explicit tile_reorder / tile_unreorder passes"},
         "sparse_attn_ms_per_call": attn_ms, "sparse_attn_tflops": attn_tflops,
         "mask_build_ms_per_call": mask_ms, "mask_build_gbs": mask_bytes / (mask_ms * 1e-3) / 1e9,
+        "pairing_ms_per_call": pairing_ms,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": bf16, "unit": "TFLOP/s",
                      "frac": attn_tflops / bf16, "traffic": measured_traffic(w.name, p, "raster" if fused else "tiled"),
                      "peak_source": f"{src} bf16 burst; frac of sustained {attn_tflops / bf16_sus:.3f}",
@@ -734,7 +749,9 @@ def main():
                          ("backward", lambda: measure_backward(args, w, p, (q, k, v))),
                          ("sip", lambda: measure_sip(args, w, p, (q, k, v))),
                          ("squad", lambda: measure_squad(args)),
-                         ("wan_tiles_2x4x8", lambda: measure_step(args, "wan_2x4x8"))):
+                         ("wan_tiles_2x4x8", lambda: measure_step(args, "wan_2x4x8")),
+                         ("hunyuan", lambda: measure_step(args, "hunyuan")),
+                         ("sparsity_sweep", lambda: measure_sweep(args, S.workload("sweep")))):
             try:
                 ext[name] = fn()
             except Exception as e:   # noqa: BLE001 - reported, not raised

@@ -10,7 +10,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdbst.so")
 SOURCES = ["dbst_api.cu"]
-HEADERS = ["ptx.cuh", "reorder.cuh", "mask.cuh", "attn_pair.cuh", "pairing.cuh", "attn_sweep.cuh", "squad.cuh", "sip.cuh", "fine.cuh"]
+HEADERS = ["ptx.cuh", "reorder.cuh", "mask.cuh", "mask_tc.cuh", "attn_pair.cuh", "pairing.cuh", "attn_sweep.cuh", "squad.cuh", "sip.cuh", "fine.cuh"]
 
 
 def nvcc() -> str:

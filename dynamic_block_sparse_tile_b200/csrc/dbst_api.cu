@@ -18,6 +18,7 @@
 #include "attn_pair.cuh"
 #include "pairing.cuh"
 #include "mask.cuh"
+#include "mask_tc.cuh"
 #include "ptx.cuh"
 #include "reorder.cuh"
 #include "sip.cuh"
@@ -142,6 +143,31 @@ MaskWorkspace mask_workspace(const dbst_geom* g) {
   return w;
 }
 
+// Tensor-core mask build (rows of at most kMaskTcMaxNB blocks): pool counters, pieces, residuals, norms.
+constexpr int kMaskTcMaxNB = 1024;
+struct MaskTcWorkspace {
+  size_t kmax, pieces, resid, norm, s, total;
+};
+MaskTcWorkspace mask_tc_workspace(const dbst_geom* g) {
+  const size_t nb = static_cast<size_t>(nblocks(g));
+  const size_t bh = static_cast<size_t>(bh_count(g));
+  const size_t d = static_cast<size_t>(g->D);
+  MaskTcWorkspace w;
+  w.kmax = 0;                                             // kmax [BH]
+  w.pieces = align_up(bh * sizeof(unsigned int));
+  w.resid = w.pieces + align_up(6 * bh * nb * d * 2);
+  w.norm = w.resid + align_up(2 * bh * nb * d * sizeof(float));
+  w.s = w.norm + align_up(2 * bh * nb * sizeof(float));   // fast pooled logits [BH][NB][NB] float32
+  w.total = w.s + align_up(bh * nb * nb * sizeof(float));
+  return w;
+}
+// The workspace of every mask builder: the float64 layout of the SIP mask and of rows longer than
+// kMaskTcMaxNB blocks, or the tensor-core layout, whichever is larger.
+size_t mask_workspace_total(const dbst_geom* g) {
+  const size_t a = mask_workspace(g).total, b = mask_tc_workspace(g).total;
+  return a > b ? a : b;
+}
+
 // ---- TMA descriptors: a [rows, D] bf16 matrix, 64 x 64 boxes, 128-byte swizzle
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -167,6 +193,21 @@ bool make_tmap(CUtensorMap* m, const void* base, long long rows, int D) {
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// The mean pieces of the tensor-core mask build, [6][BH][NB][D] bf16, as a 4-D tensor (innermost
+// first); one box is `rows` blocks x 64 channels of one piece of one head; rows past NB read as 0.
+bool make_tmap_pieces(CUtensorMap* m, const void* base, long long BH, int NB, int D, int rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(NB), static_cast<cuuint64_t>(BH), 6};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(NB) * D * 2,
+                           static_cast<cuuint64_t>(BH) * NB * D * 2};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(rows), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Query blocks are paired with their neighbour one tile step along the slowest tile axis
@@ -536,6 +577,106 @@ dbst_status pool_and_logits(const void* q, const void* k, const dbst_geom* g, co
   return DBST_OK;
 }
 
+template <int D, int NPT>
+bool launch_select_rows(const dbst::SelRowsParams& prm, cudaStream_t s) {
+  const long long rows = prm.BH * prm.NB;
+  const long long grid = (rows + dbst::kSelRowsWarps - 1) / dbst::kSelRowsWarps;
+  dbst::select_rows_kernel<D, NPT><<<static_cast<unsigned>(grid), 32 * dbst::kSelRowsWarps, 0, s>>>(prm);
+  return cudaGetLastError() == cudaSuccess;
+}
+
+template <int D>
+bool launch_select_rows_npt(const dbst::SelRowsParams& prm, cudaStream_t s) {
+  const int NB = prm.NB;
+  if (NB <= 32) return launch_select_rows<D, 1>(prm, s);
+  if (NB <= 128) return launch_select_rows<D, 4>(prm, s);
+  if (NB <= 256) return launch_select_rows<D, 8>(prm, s);
+  if (NB <= 512) return launch_select_rows<D, 16>(prm, s);
+  if (NB <= 640) return launch_select_rows<D, 20>(prm, s);
+  return launch_select_rows<D, 32>(prm, s);
+}
+
+// Tensor-core mask build (NB <= kMaskTcMaxNB): the pool (HBM-bound), then the selection (persistent:
+// tensor cores for the logits, one warp per row for the CDF selection).
+dbst_status build_mask_tc(const void* q, const void* k, const dbst_geom* g, float p, int sta_radius,
+                          uint32_t* mask_bits, int32_t* kv_count, int16_t* kv_idx, char* ws, cudaStream_t s,
+                          bool raster) {
+  const MaskTcWorkspace w = mask_tc_workspace(g);
+  const int NB = nblocks(g), D = g->D;
+  const long long BH = bh_count(g);
+  dbst::MaskTcBuffers wb;
+  wb.kmax = reinterpret_cast<unsigned int*>(ws + w.kmax);
+  wb.pieces = reinterpret_cast<__nv_bfloat16*>(ws + w.pieces);
+  wb.resid = reinterpret_cast<float*>(ws + w.resid);
+  wb.norm = reinterpret_cast<float*>(ws + w.norm);
+  if (cudaMemsetAsync(ws + w.kmax, 0, BH * sizeof(unsigned int), s) != cudaSuccess) return DBST_ECUDA;
+  {  // 1. block means as pieces, residuals and norms
+    const long long warps = 2 * BH * NB;
+    long long grid = (warps * 32 + dbst::kPoolTcThreads - 1) / dbst::kPoolTcThreads;
+    const long long cap = static_cast<long long>(sm_count()) * 8;
+    if (grid > cap) grid = cap;
+    const auto* qa = static_cast<const uint4*>(q);
+    const auto* ka = static_cast<const uint4*>(k);
+    const unsigned gr = static_cast<unsigned>(grid);
+    const dbst::TileGeo tg = tile_geo(g);
+    if (D == 128) {
+      if (raster) dbst::pool_pieces_kernel<128, true><<<gr, dbst::kPoolTcThreads, 0, s>>>(qa, ka, wb, BH, NB, tg);
+      else dbst::pool_pieces_kernel<128, false><<<gr, dbst::kPoolTcThreads, 0, s>>>(qa, ka, wb, BH, NB, tg);
+    } else {
+      if (raster) dbst::pool_pieces_kernel<64, true><<<gr, dbst::kPoolTcThreads, 0, s>>>(qa, ka, wb, BH, NB, tg);
+      else dbst::pool_pieces_kernel<64, false><<<gr, dbst::kPoolTcThreads, 0, s>>>(qa, ka, wb, BH, NB, tg);
+    }
+    if (cudaGetLastError() != cudaSuccess) return DBST_ECUDA;
+  }
+  // 2. pooled logits on the tensor cores, into the float32 map S
+  float* S = reinterpret_cast<float*>(ws + w.s);
+  dbst::LogTcParams lp;
+  lp.wb = wb;
+  lp.S = S;
+  lp.BH = BH;
+  lp.NB = NB;
+  lp.ntiles = (NB + 127) / 128;
+  lp.R = lp.ntiles <= 3 ? 64 : lp.ntiles <= 5 ? 48 : 32;
+  lp.chunks = (NB + lp.R - 1) / lp.R;
+  const double scale = 1.0 / std::sqrt(static_cast<double>(D));
+  lp.scale_f = static_cast<float>(scale);
+  lp.wait_limit = wait_limit();
+  {
+    CUtensorMap tq, tk;
+    if (!make_tmap_pieces(&tq, wb.pieces, BH, NB, D, lp.R) || !make_tmap_pieces(&tk, wb.pieces, BH, NB, D, 128))
+      return DBST_ECUDA;
+    const long long items = BH * lp.chunks;
+    const unsigned grid = static_cast<unsigned>(items < sm_count() ? items : sm_count());
+    const int smem = (D == 128 ? dbst::LogTcSmem<128>::bytes(lp.R) : dbst::LogTcSmem<64>::bytes(lp.R)) + 1024;
+    if (D == 128) {
+      if (!smem_opt_in(dbst::pooled_logits_tc_kernel<128>, smem)) return DBST_ECUDA;
+      dbst::pooled_logits_tc_kernel<128><<<grid, dbst::kLogTcThreads, smem, s>>>(tq, tk, lp);
+    } else {
+      if (!smem_opt_in(dbst::pooled_logits_tc_kernel<64>, smem)) return DBST_ECUDA;
+      dbst::pooled_logits_tc_kernel<64><<<grid, dbst::kLogTcThreads, smem, s>>>(tq, tk, lp);
+    }
+    if (cudaGetLastError() != cudaSuccess) return DBST_ECUDA;
+  }
+  // 3. CDF selection, exactness band, sliding-tile union, lists: one warp per row
+  dbst::SelRowsParams prm;
+  prm.wb = wb;
+  prm.S = S;
+  prm.bits = mask_bits;
+  prm.count = kv_count;
+  prm.idx = kv_idx;
+  prm.BH = BH;
+  prm.NB = NB;
+  prm.NW = (NB + 31) / 32;
+  prm.nX = g->X / g->tx;
+  prm.nY = g->Y / g->ty;
+  prm.sta_radius = sta_radius;
+  prm.p = static_cast<double>(p);
+  prm.scale = scale;
+  prm.scale_f = static_cast<float>(scale);
+  const bool ok = D == 128 ? launch_select_rows_npt<128>(prm, s) : launch_select_rows_npt<64>(prm, s);
+  return ok ? launch_status() : DBST_ECUDA;
+}
+
 // Mask build over tile-ordered (raster = false) or raster-ordered (raster = true) q and k.
 dbst_status build_mask(const void* q_tiled, const void* k_tiled, const dbst_geom* g, float p, int sta_radius,
                        uint32_t* mask_bits, int32_t* kv_count, int16_t* kv_idx, void* workspace,
@@ -546,10 +687,12 @@ dbst_status build_mask(const void* q_tiled, const void* k_tiled, const dbst_geom
     return DBST_EINVAL;
   if (!(p > 0.0f && p <= 1.0f)) return DBST_EINVAL;   // also rejects NaN
   const MaskWorkspace w = mask_workspace(g);
-  if (workspace_bytes < w.total) return DBST_EINVAL;
+  if (workspace_bytes < mask_workspace_total(g)) return DBST_EINVAL;
   if (bh_count(g) > 65535) return DBST_EINVAL;        // grid.z of the pooled-logits launch
   auto s = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
+  if (nblocks(g) <= kMaskTcMaxNB)
+    return build_mask_tc(q_tiled, k_tiled, g, p, sta_radius, mask_bits, kv_count, kv_idx, ws, s, raster);
   double* S = reinterpret_cast<double*>(ws + w.s);
   const int NB = nblocks(g);
   const long long nblk = bh_count(g) * NB;
@@ -662,7 +805,7 @@ dbst_status build_sip_mask(const void* q, const void* k, const dbst_geom* g, dou
     return DBST_EINVAL;
   if (!(budget > 0.0) || !std::isfinite(budget)) return DBST_EINVAL;
   const MaskWorkspace w = mask_workspace(g);
-  if (workspace_bytes < w.total) return DBST_EINVAL;
+  if (workspace_bytes < mask_workspace_total(g)) return DBST_EINVAL;
   if (bh_count(g) > 65535) return DBST_EINVAL;
   auto s = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
@@ -705,7 +848,7 @@ dbst_status dbst_tile_unreorder(const void* y, void* x, const dbst_geom* g, void
 
 size_t dbst_mask_workspace_bytes(const dbst_geom* g) {
   if (!geom_ok(g)) return 0;
-  return mask_workspace(g).total;
+  return mask_workspace_total(g);
 }
 
 dbst_status dbst_build_block_mask(const void* q_tiled, const void* k_tiled, const dbst_geom* g, float p,
@@ -978,7 +1121,7 @@ extern "C" dbst_status dbst_build_block_mask_noalloc(const void* q_tiled, const 
                                                      float p, int sta_radius, uint32_t* mask_bits,
                                                      int32_t* kv_count, int16_t* kv_idx, void* stream) {
   if (!geom_ok(g)) return DBST_EINVAL;
-  if (mask_workspace(g).total > static_cast<size_t>(DBST_NOALLOC_SCRATCH_BYTES)) return DBST_ETOOLARGE;
+  if (mask_workspace_total(g) > static_cast<size_t>(DBST_NOALLOC_SCRATCH_BYTES)) return DBST_ETOOLARGE;
   void* scratch = scratch_for_current_device();
   if (scratch == nullptr) return DBST_ECUDA;
   return dbst_build_block_mask(q_tiled, k_tiled, g, p, sta_radius, mask_bits, kv_count, kv_idx, scratch,

@@ -4,9 +4,12 @@
 //
 // Precision: the pooled means are exact (64 bf16 values summed in float64) and
 // the pooled logits are float64.  The order of a row's blocks comes from those
-// logits; the masses are float32 exponentials summed in float64 for rows of at
-// most 1024 blocks, float64 for longer rows.  The kept set agrees with a
-// float64 reference except where a cumulative mass sits within rounding of p.
+// logits; the masses are float32 exponentials summed in float32 for rows of at
+// most 1024 blocks (one warp per row), float64 exponentials and sums for longer
+// rows.  The kept set agrees with a float64 reference except where a
+// cumulative mass sits within rounding of p.  (Rows of at most 1024 blocks are
+// built by the tensor-core path of mask_tc.cuh; these kernels serve the longer
+// rows and the SIP mask.)
 #pragma once
 #include <cstdint>
 #include "ptx.cuh"
@@ -415,6 +418,7 @@ __global__ void __launch_bounds__(128) select_warp_kernel(const double* __restri
   unsigned long long thr = 0ull;   // keep key >= thr (0 keeps all)
   if (g.p < 1.0) {
     unsigned long long lo = 0ull, hi = ~0ull;   // the answer lies in (lo, hi]
+    unsigned long long cand = 0ull;             // smallest key above hi (see below)
     float above = 0.0f;                         // mass of keys > hi
     for (int round = 0; round < 4 * 32 * NPT; ++round) {
       int mycnt = 0;
@@ -426,7 +430,13 @@ __global__ void __launch_bounds__(128) select_warp_kernel(const double* __restri
         if (live) mine = key[u];
       }
       const unsigned holders = __ballot_sync(0xffffffffu, mycnt > 0);
-      if (holders == 0u) break;                 // total mass below p (rounding): keep every block
+      if (holders == 0u) {
+        // The float32 sums of different orders left no key between "mass above hi < target" and
+        // "mass above lo >= target": the crossing is, within rounding, the smallest key above hi
+        // (0 keeps every block when hi never moved).
+        thr = cand;
+        break;
+      }
       const int nh = __popc(holders);
       const int pick = __fns(holders, 0, 1 + (round * 7) % nh);
       const unsigned long long pivot = __shfl_sync(0xffffffffu, mine, pick);
@@ -447,6 +457,7 @@ __global__ void __launch_bounds__(128) select_warp_kernel(const double* __restri
           break;
         }
         hi = pivot - 1ull;                      // below the pivot; everything >= pivot counts as above
+        cand = pivot;
         above = f;
       }
     }

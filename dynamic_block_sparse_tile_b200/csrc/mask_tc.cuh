@@ -1,0 +1,637 @@
+// Adaptive block mask with the pooled logits on the tensor cores (NABLA page,
+// "Construction de Masque Adaptatif": block mean-pool, reduced attention map,
+// CDF threshold; "Intégration Hybride avec STA": the sliding-tile union).
+//
+// Three kernels:
+//
+//   pool_pieces_kernel (HBM-bound) averages every 64-token block of q and k
+//   exactly (64 bf16 values summed in float64) and stores each mean x as three
+//   bf16 pieces b1 + b2 + b3 (round to nearest, each piece the rounded
+//   remainder of the previous ones, together the float32 value of x) plus the
+//   float32 residual x - (b1 + b2 + b3), and the block's norm.
+//
+//   pooled_logits_tc_kernel (persistent) takes items of R consecutive query
+//   blocks of one head.  tcgen05 computes the pooled logits of the R rows
+//   against every key block as S^T = Kp . Qp^T (M = 128 key blocks per tile,
+//   N = R rows), from the pieces: D1 = b1 b1 and D2 = b1 b2 + b2 b1 + b1 b3 +
+//   b2 b2 + b3 b1 in two fp32 accumulators; s = (D1 + D2) * scale goes to a
+//   float32 map in the workspace (small enough to stay in L2 for the next
+//   kernel).
+//
+//   select_rows_kernel, one warp per row and many rows in flight per SM, takes
+//   the CDF selection by a radix select on the row's keys with integer masses
+//   and writes bits and lists.
+//
+// Exactness.  The order of a row's blocks must be the order of the exact
+// (float64) logits.  The fast logits carry an error below E = 2^-15 * scale *
+// |Qp_i| * max_j |Kp_j| (Cauchy-Schwarz on the neglected piece products, the
+// representation errors and eight fp32 accumulation steps of D1, with a margin
+// of four).  After the fast selection, every key whose fast logit lies within
+// 4E of the boundary key's is recomputed exactly in float64 from the pieces and
+// residuals, and the selection is repeated with those keys ordered exactly and
+// all other keys placed above or below the band.  The result stands if the new
+// boundary lies within 2E of the old one; otherwise the band doubles and the
+// step repeats.  Masses are float32 exponentials of the fast logits, rounded to
+// integers of 2^-26 of the row's largest and summed exactly; a kept set can therefore differ from a
+// float64 reference only where a cumulative mass lies within rounding of p.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include "mask.cuh"
+#include "ptx.cuh"
+#include "reorder.cuh"
+
+namespace dbst {
+
+// ---------------------------------------------------------------------------
+// Workspace of the tensor-core mask build (all offsets 256-byte aligned).
+// ---------------------------------------------------------------------------
+struct MaskTcBuffers {
+  unsigned int* kmax;       // [BH] float bits of max_j |Kp_j| (zeroed before the pool kernel)
+  __nv_bfloat16* pieces;    // [6][BH][NB][D]: q pieces 1..3, then k pieces 1..3
+  float* resid;             // [2][BH][NB][D]: q, k residuals
+  float* norm;              // [2][BH][NB]: q, k block norms (rounded up)
+};
+
+constexpr int kPoolTcThreads = 256;
+
+template <int D, bool RASTER>
+__global__ void __launch_bounds__(kPoolTcThreads) pool_pieces_kernel(const uint4* __restrict__ q,
+                                                                     const uint4* __restrict__ k, MaskTcBuffers wb,
+                                                                     long long BH, int NB, TileGeo tg) {
+  constexpr int CPR = D / 8;            // 16-byte chunks per token row
+  constexpr int RPW = 32 / CPR;         // token rows covered by one warp pass
+  const int lane = threadIdx.x & 31;
+  const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  const int ch = lane % CPR;
+  const int r0 = lane / CPR;
+  __shared__ int row_off[64];             // raster offset of tile row r from the tile's first token
+  if (RASTER) {
+    if (threadIdx.x < 64) row_off[threadIdx.x] = tiled_to_raster(threadIdx.x, tg);   // tile 0 starts at token 0
+    __syncthreads();
+  }
+  const long long total = 2 * BH * NB;   // the q blocks of a head, then its k blocks
+  const long long plane = BH * NB * static_cast<long long>(D);
+  for (long long w = warp; w < total; w += nwarps) {
+    const long long bh = w / (2 * NB);
+    const int rem = static_cast<int>(w - bh * 2 * NB);
+    const bool isk = rem >= NB;
+    const int blk = isk ? rem - NB : rem;
+    const uint4* src = (isk ? k : q) +
+                       (bh * tg.N + (RASTER ? tiled_to_raster(blk * 64, tg) : static_cast<long long>(blk) * 64)) * CPR;
+    double acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.0;
+#pragma unroll 8
+    for (int r = r0; r < 64; r += RPW) {
+      const uint4 v = ld_stream(src + (RASTER ? row_off[r] : r) * CPR + ch);
+      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[2 * e] += static_cast<double>(__uint_as_float(u[e] << 16));
+        acc[2 * e + 1] += static_cast<double>(__uint_as_float(u[e] & 0xFFFF0000u));
+      }
+    }
+#pragma unroll
+    for (int off = CPR; off < 32; off <<= 1) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+    }
+    // every lane now holds the sums of channels 8ch .. 8ch+7
+    uint32_t pw[3][4];
+    float res[8];
+    double n2 = 0.0;
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      uint32_t pr[3] = {0u, 0u, 0u};
+#pragma unroll
+      for (int f = 0; f < 2; ++f) {
+        const double x = acc[e + f] * (1.0 / 64.0);
+        n2 = fma(x, x, n2);
+        const float hi = __double2float_rn(x);
+        const __nv_bfloat16 b1 = __float2bfloat16_rn(hi);
+        const float r1 = hi - __bfloat162float(b1);
+        const __nv_bfloat16 b2 = __float2bfloat16_rn(r1);
+        const float r2 = r1 - __bfloat162float(b2);
+        const __nv_bfloat16 b3 = __float2bfloat16_rn(r2);
+        const double rep = static_cast<double>(__bfloat162float(b1)) + static_cast<double>(__bfloat162float(b2)) +
+                           static_cast<double>(__bfloat162float(b3));
+        res[e + f] = __double2float_rn(x - rep);
+        pr[0] |= static_cast<uint32_t>(__bfloat16_as_ushort(b1)) << (16 * f);
+        pr[1] |= static_cast<uint32_t>(__bfloat16_as_ushort(b2)) << (16 * f);
+        pr[2] |= static_cast<uint32_t>(__bfloat16_as_ushort(b3)) << (16 * f);
+      }
+      pw[0][e / 2] = pr[0];
+      pw[1][e / 2] = pr[1];
+      pw[2][e / 2] = pr[2];
+    }
+#pragma unroll
+    for (int off = 1; off < CPR; off <<= 1) n2 += __shfl_xor_sync(0xffffffffu, n2, off);
+    const long long row = (bh * NB + blk) * static_cast<long long>(D);
+    if (r0 == 0) {
+#pragma unroll
+      for (int pc = 0; pc < 3; ++pc) {
+        uint4* dst = reinterpret_cast<uint4*>(wb.pieces + (isk ? 3 + pc : pc) * plane + row + ch * 8);
+        *dst = make_uint4(pw[pc][0], pw[pc][1], pw[pc][2], pw[pc][3]);
+      }
+      float4* rd = reinterpret_cast<float4*>(wb.resid + (isk ? plane : 0) + row + ch * 8);
+      rd[0] = make_float4(res[0], res[1], res[2], res[3]);
+      rd[1] = make_float4(res[4], res[5], res[6], res[7]);
+    }
+    if (lane == 0) {
+      const float nrm = __double2float_ru(__dsqrt_ru(n2));
+      wb.norm[(isk ? BH * NB : 0) + bh * NB + blk] = nrm;
+      if (isk) atomicMax(wb.kmax + bh, __float_as_uint(nrm));   // non-negative floats order as their bits
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Selection kernel.
+// ---------------------------------------------------------------------------
+constexpr int kLogTcThreads = 192;       // warp 0 TMA, warp 1 MMA, warps 2..5 drain
+constexpr int kLogTcDrain = 4;
+constexpr int kLogTcStages = 3;          // K ring: one piece of one 64-channel half of one key tile
+
+struct LogTcParams {
+  MaskTcBuffers wb;
+  float* S;            // out: [BH][NB][NB] fast pooled logits, already scaled
+  long long BH;
+  int NB;
+  int ntiles;          // key tiles of 128 blocks: ceil(NB / 128)
+  int R;               // query blocks per item (a multiple of 16)
+  int chunks;          // items per head: ceil(NB / R)
+  float scale_f;
+  long long wait_limit;
+};
+
+// dynamic shared memory layout (bytes, from a 1024-aligned base)
+template <int D>
+struct LogTcSmem {
+  static constexpr int kDH = D / 64;
+  static __host__ __device__ constexpr int q_bytes(int R) { return 3 * kDH * R * 128; }
+  static __host__ __device__ constexpr int ring(int R) { return q_bytes(R); }
+  static __host__ __device__ constexpr int stage_bytes() { return 128 * 128; }
+  static __host__ __device__ constexpr int bars(int R) { return ring(R) + kLogTcStages * stage_bytes(); }
+  static __host__ __device__ constexpr int bytes(int R) { return bars(R) + 256; }
+};
+
+enum {
+  SB_QFULL = 0,
+  SB_QFREE = 1,
+  SB_KFULL = 2,
+  SB_KEMPTY = SB_KFULL + kLogTcStages,
+  SB_ACC = SB_KEMPTY + kLogTcStages,     // the item's logits are complete in TMEM
+  SB_TFREE = SB_ACC + 1,                 // the drain warps have read TMEM out
+  SB_DRAIN = SB_TFREE + 1,               // every product issued has completed (before TMEM is freed)
+  SB_COUNT = SB_DRAIN + 1
+};
+
+// Row selection: one warp per query-block row.
+constexpr int kSelRowsWarps = 4;
+constexpr int kHistStride = 17;          // words per lane of a warp's radix-select histogram rows
+
+struct SelRowsParams {
+  MaskTcBuffers wb;
+  const float* S;      // [BH][NB][NB] fast pooled logits
+  uint32_t* bits;
+  int32_t* count;
+  int16_t* idx;
+  long long BH;
+  int NB, NW;
+  int nX, nY;          // tile grid
+  int sta_radius;      // < 0: none
+  double p;            // CDF threshold; >= 1 keeps all
+  double scale;        // 1 / sqrt(D)
+  float scale_f;
+};
+
+// Order-preserving maps of float and double onto unsigned integers.
+__device__ __forceinline__ uint32_t ord32(float x) {
+  const uint32_t b = __float_as_uint(x);
+  return (b >> 31) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ unsigned long long ord64(double x) {
+  const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(x));
+  return (b >> 63) ? ~b : (b | (1ull << 63));
+}
+// Selection key: class (2 bits) | order value (46 bits) | 0xFFFF - j.  Larger = earlier in the order.
+__device__ __forceinline__ unsigned long long sel_key(unsigned cls, unsigned long long sub46, int j) {
+  return (static_cast<unsigned long long>(cls) << 62) | ((sub46 & ((1ull << 46) - 1)) << 16) |
+         static_cast<unsigned long long>(0xFFFF - j);
+}
+
+// Radix select over 64-bit keys (unique: they carry the block index) with integer masses: the key
+// whose cumulative mass in descending key order first reaches `tgt`.  Passes of 4-bit digits,
+// starting at the highest bit where the candidates differ.  Each pass builds a 16-bin mass histogram
+// of the candidates (the keys that agree with the digits fixed so far): every lane sums its own
+// entries into a private row of the warp's shared-memory area `h` (17 words per lane, so the lanes'
+// rows fall in different banks), then lane b adds up column b.  The bin where the cumulative mass
+// crosses `tgt` fixes the next digit; the select ends once a single candidate is left.  Masses are
+// integers and every sum is exact, so the result does not depend on the order of the additions.
+// Entries with key 0 are not part of the row.  Per-lane sums must fit 32 bits: NPT masses of at
+// most 2^26.
+template <int NPT>
+__device__ __forceinline__ unsigned long long radix_select(const unsigned long long (&key)[NPT],
+                                                          const uint32_t (&M)[NPT], unsigned long long tgt,
+                                                          uint32_t* h) {
+  const int lane = threadIdx.x & 31;
+  // highest bit where the row's keys differ
+  unsigned long long first = 0ull, diff = 0ull;
+#pragma unroll
+  for (int u = 0; u < NPT; ++u)
+    if (first == 0ull && key[u] != 0ull) first = key[u];
+  {
+    const unsigned own = __ballot_sync(0xffffffffu, first != 0ull);
+    if (own == 0u) return 0ull;
+    first = __shfl_sync(0xffffffffu, first, __ffs(own) - 1);
+  }
+#pragma unroll
+  for (int u = 0; u < NPT; ++u)
+    if (key[u] != 0ull) diff |= key[u] ^ first;
+  const unsigned dlo = __reduce_or_sync(0xffffffffu, static_cast<unsigned>(diff));
+  const unsigned dhi = __reduce_or_sync(0xffffffffu, static_cast<unsigned>(diff >> 32));
+  const unsigned long long alld = (static_cast<unsigned long long>(dhi) << 32) | dlo;
+  if (alld == 0ull) return first;        // a single entry
+  int hi = 63 - __clzll(static_cast<long long>(alld));
+  unsigned long long pmask = ~((2ull << hi) - 1ull);   // bits above hi: equal for every entry
+  unsigned long long prefix = first & pmask;
+  unsigned long long above = 0ull;
+  uint32_t* mine = h + lane * kHistStride;
+  for (;; hi -= 4) {
+    const int lo = hi >= 3 ? hi - 3 : 0;   // digit bits [lo, hi]
+    const unsigned long long dmask = (1ull << (hi - lo + 1)) - 1ull;
+#pragma unroll
+    for (int b = 0; b < 16; ++b) mine[b] = 0u;
+    int ncand = 0;
+    unsigned long long last = 0ull;
+#pragma unroll
+    for (int u = 0; u < NPT; ++u) {
+      if (key[u] != 0ull && (key[u] & pmask) == prefix) {
+        mine[(key[u] >> lo) & dmask] += M[u];
+        ++ncand;
+        last = key[u];
+      }
+    }
+    // a single candidate left: it is the answer
+    const int total_cand = __reduce_add_sync(0xffffffffu, ncand);
+    if (total_cand <= 1) {
+      const unsigned own = __ballot_sync(0xffffffffu, ncand > 0);
+      return own ? __shfl_sync(0xffffffffu, last, __ffs(own) - 1) : 0ull;
+    }
+    __syncwarp();
+    // lanes 0..15 hold the bins in descending digit order: lane i sums column 15 - i
+    unsigned long long v = 0ull;
+    if (lane < 16) {
+      const int d = 15 - lane;
+#pragma unroll 8
+      for (int l = 0; l < 32; ++l) v += h[l * kHistStride + d];
+    }
+    __syncwarp();
+    unsigned long long incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const unsigned long long o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    // the mass above the candidates plus the candidates' mass reaches tgt, so some bin crosses
+    const unsigned hit = __ballot_sync(0xffffffffu, lane < 16 && above + incl >= tgt);
+    if (hit == 0u) return 0ull;           // not reached
+    const int b = __ffs(hit) - 1;
+    above += __shfl_sync(0xffffffffu, incl - v, b);
+    prefix |= static_cast<unsigned long long>(15 - b) << lo;
+    pmask |= dmask << lo;
+    if (lo == 0) {                        // every bit fixed: the unique key with this value
+      unsigned long long k = 0ull;
+#pragma unroll
+      for (int u = 0; u < NPT; ++u)
+        if (key[u] != 0ull && key[u] == prefix) k = key[u];
+      const unsigned own = __ballot_sync(0xffffffffu, k != 0ull);
+      return own ? __shfl_sync(0xffffffffu, k, __ffs(own) - 1) : 0ull;
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kLogTcThreads, 1)
+    pooled_logits_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                            const LogTcParams prm) {
+  using L = LogTcSmem<D>;
+  constexpr int DH = D / 64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(sm);
+  const int R = prm.R, ntiles = prm.ntiles, NB = prm.NB;
+  uint32_t* s_misc = reinterpret_cast<uint32_t*>(sm + L::bars(R) + 8 * SB_COUNT);
+  volatile uint32_t* s_abort = s_misc + 1;
+  auto bar = [&](int slot) -> uint32_t { return sbase + L::bars(R) + 8u * slot; };
+  const long long limit = prm.wait_limit > 0 ? prm.wait_limit : kWaitLimitCycles;
+  auto wait_live = [&](uint32_t mb, uint32_t parity, bool& live) {
+    if (!live || mbar_try(mb, parity)) return;
+    const long long t0 = clock64();
+    while (!mbar_try(mb, parity)) {
+      if (*s_abort) { live = false; return; }
+      if (clock64() - t0 > limit) {
+        record_error(kErrTimeout);
+        *s_abort = 1;
+        live = false;
+        return;
+      }
+    }
+  };
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long items = prm.BH * prm.chunks;
+  const int tcols = 2 * ntiles * R;
+  const uint32_t tmem_cols = tcols <= 32 ? 32u : tcols <= 64 ? 64u : tcols <= 128 ? 128u : tcols <= 256 ? 256u : 512u;
+  if (tid == 0) {
+    for (int b = 0; b < SB_COUNT; ++b) mbar_init(bar(b), b == SB_TFREE ? kLogTcDrain : 1u);
+    fence_mbar_init();
+    s_misc[1] = 0;
+  }
+  if (warp == 1) {
+    tmem_alloc(sbase + L::bars(R) + 8 * SB_COUNT, tmem_cols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_misc[0];
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (lane 0)
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      bool live = true;
+      int n = 0;                 // items of this CTA so far
+      long long gst = 0;         // K stages issued
+      int armed[kLogTcStages] = {0, 0, 0};
+      int qarmed = 0;
+      for (long long it = blockIdx.x; it < items && live; it += gridDim.x, ++n) {
+        const long long bh = it / prm.chunks;
+        const int i0 = static_cast<int>(it - bh * prm.chunks) * R;
+        if (n >= 1) wait_live(bar(SB_QFREE), (n - 1) & 1, live);
+        if (!live) break;
+        mbar_expect_tx(bar(SB_QFULL), 3 * DH * R * 128);
+        for (int pc = 0; pc < 3; ++pc)
+          for (int h = 0; h < DH; ++h)
+            tma_load_4d(sbase + (pc * DH + h) * R * 128, &tmQ, bar(SB_QFULL), 64 * h, i0, static_cast<int>(bh), pc);
+        qarmed = n + 1;
+        for (int m = 0; m < ntiles && live; ++m)
+          for (int h = 0; h < DH && live; ++h)
+            for (int pc = 0; pc < 3; ++pc, ++gst) {
+              const int s = static_cast<int>(gst % kLogTcStages);
+              if (gst >= kLogTcStages)
+                wait_live(bar(SB_KEMPTY + s), static_cast<uint32_t>((gst / kLogTcStages) - 1) & 1u, live);
+              if (!live) break;
+              mbar_expect_tx(bar(SB_KFULL + s), 128 * 128);
+              tma_load_4d(sbase + L::ring(R) + s * L::stage_bytes(), &tmK, bar(SB_KFULL + s), 64 * h, 128 * m,
+                          static_cast<int>(bh), 3 + pc);
+              armed[s] = static_cast<int>(gst / kLogTcStages) + 1;
+            }
+      }
+      // no copy may still be landing when the CTA exits
+      for (int s = 0; s < kLogTcStages; ++s)
+        if (armed[s] > 0) mbar_wait(bar(SB_KFULL + s), (armed[s] - 1) & 1);
+      if (qarmed > 0) mbar_wait(bar(SB_QFULL), (qarmed - 1) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (whole warp)
+    const uint32_t idesc = idesc_bf16(128, R, 0, 0);   // A = key tile piece (K-major), B = query rows piece
+    bool ok = true;
+    int n = 0;
+    long long gst = 0;
+    auto wait_all = [&](int slot, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait_lim(bar(slot), parity, limit));
+    };
+    for (long long it = blockIdx.x; it < items && ok; it += gridDim.x, ++n) {
+      if (!wait_all(SB_QFULL, n & 1)) { ok = false; break; }
+      if (n >= 1 && !wait_all(SB_TFREE, (n - 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      for (int m = 0; m < ntiles && ok; ++m)
+        for (int h = 0; h < DH && ok; ++h)
+          for (int pc = 0; pc < 3; ++pc, ++gst) {
+            const int s = static_cast<int>(gst % kLogTcStages);
+            if (__any_sync(0xffffffffu, *s_abort != 0) ||
+                !wait_all(SB_KFULL + s, static_cast<uint32_t>(gst / kLogTcStages) & 1u)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t a0 = smem_desc(sbase + L::ring(R) + s * L::stage_bytes(), 16, 1024);
+            // key piece pc+1 meets the query pieces whose order sum is at most 4:
+            //   D1: (1, 1);  D2: (1, 2), (1, 3), (2, 1), (2, 2), (3, 1)
+            const int nq = pc == 0 ? 3 : pc == 1 ? 2 : 1;
+            for (int pq = 0; pq < nq; ++pq) {
+              const bool d1 = pc == 0 && pq == 0;
+              const uint32_t dcol = static_cast<uint32_t>((d1 ? 0 : ntiles) + m) * static_cast<uint32_t>(R);
+              const uint64_t b0 = smem_desc(sbase + (pq * DH + h) * R * 128, 16, 1024);
+              // first product into D1: (h 0, pc 0, pq 0); into D2: (h 0, pc 0, pq 1)
+              const bool first = h == 0 && pc == 0 && pq <= 1;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                umma_f16_elect(tmem + dcol, a0 + static_cast<uint64_t>(kk * 2), b0 + static_cast<uint64_t>(kk * 2),
+                               idesc, (first && kk == 0) ? 0u : 1u);
+            }
+            umma_commit_elect(bar(SB_KEMPTY + s));
+          }
+      if (!ok) break;
+      umma_commit_elect(bar(SB_ACC));
+      umma_commit_elect(bar(SB_QFREE));
+    }
+    if (!ok && lane == 0) *s_abort = 1;
+    // every product issued has completed before TMEM is freed
+    umma_commit_elect(bar(SB_DRAIN));
+    mbar_wait(bar(SB_DRAIN), 0);
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ drain (4 warps): TMEM -> S
+    const int qtr = warp & 3;                  // TMEM lane quarter: key blocks 32 qtr .. +31 of each tile
+    const uint32_t lrow = static_cast<uint32_t>(32 * qtr) << 16;
+    const float scale_f = prm.scale_f;
+    bool live = true;
+    int n = 0;
+    for (long long it = blockIdx.x; it < items; it += gridDim.x, ++n) {
+      const long long bh = it / prm.chunks;
+      const int i0 = static_cast<int>(it - bh * prm.chunks) * R;
+      wait_live(bar(SB_ACC), n & 1, live);
+      tc_fence_after();
+      // S[bh][i0 + c][j] = (D1 + D2) * scale for key block j = 128 m + 32 qtr + lane: each store of a
+      // warp covers 32 consecutive keys of one row
+      for (int m = 0; m < ntiles; ++m) {
+        const int j = m * 128 + 32 * qtr + lane;
+        for (int c0 = 0; c0 < R; c0 += 8) {
+          uint32_t a[8], b[8];
+          tmem_ld8(tmem + lrow + static_cast<uint32_t>(m * R + c0), a);
+          tmem_ld8(tmem + lrow + static_cast<uint32_t>((ntiles + m) * R + c0), b);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const int i = i0 + c0 + c;
+            if (i < NB && j < NB)
+              prm.S[(bh * NB + i) * static_cast<long long>(NB) + j] =
+                  (__uint_as_float(a[c]) + __uint_as_float(b[c])) * scale_f;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(SB_TFREE));
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tmem_cols);
+  }
+}
+
+
+// One warp per query-block row of the fast pooled logits: integer masses, radix select of the CDF
+// boundary, the exactness band around it, the sliding-tile union, bits and lists.
+// At least four blocks (16 warps) per SM: the rows are latency-bound, so rows in flight matter.
+template <int D, int NPT>
+__global__ void __launch_bounds__(32 * kSelRowsWarps, 4) select_rows_kernel(const SelRowsParams prm) {
+  __shared__ uint32_t s_hist[kSelRowsWarps][32 * kHistStride];
+  const int lane = threadIdx.x & 31, wk = threadIdx.x >> 5;
+  const long long rows = prm.BH * prm.NB;
+  const long long row = static_cast<long long>(blockIdx.x) * kSelRowsWarps + wk;
+  if (row >= rows) return;                       // whole warps only
+  const int NB = prm.NB, NW = prm.NW;
+  const long long bh = row / NB;
+  const int i = static_cast<int>(row - bh * NB);
+  uint32_t* hist = s_hist[wk];
+  const float scale_f = prm.scale_f;
+  const float kmax = __uint_as_float(prm.wb.kmax[bh]);
+  const float* srow = prm.S + row * NB;
+        // fast logits, masses and keys
+        // the row is read through L1 wherever it is needed
+        auto sv = [&](int u) -> float { return __ldg(srow + lane + 32 * u); };   // valid for j = lane + 32u < NB
+        uint32_t mass[NPT];               // e^(s - max) in units of 2^-26
+        unsigned long long key[NPT];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < NPT; ++u)
+          if (lane + 32 * u < NB) mx = fmaxf(mx, sv(u));
+        mx = warp_max_f32(mx);
+        unsigned long long total = 0ull;
+#pragma unroll
+        for (int u = 0; u < NPT; ++u) {
+          const int j = lane + 32 * u;
+          const float x = (j < NB) ? sv(u) : 0.0f;
+          mass[u] = (j < NB) ? __float2uint_rn(fast_exp2((x - mx) * 1.4426950408889634f) * 67108864.0f) : 0u;
+          total += mass[u];
+          key[u] = (j < NB) ? sel_key(1u, static_cast<unsigned long long>(ord32(x)) << 14, j) : 0ull;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) total += __shfl_xor_sync(0xffffffffu, total, off);
+        // cumulative mass to reach: p of the total, rounded up
+        const unsigned long long target = static_cast<unsigned long long>(ceil(prm.p * static_cast<double>(total)));
+        unsigned long long thr = 0ull;   // keep key >= thr (0 keeps all)
+        if (prm.p < 1.0) {
+          thr = radix_select<NPT>(key, mass, target, hist);
+          if (thr != 0ull) {
+            // ---- exactness band around the boundary block
+            const float E = 3.0517578125e-05f * scale_f * prm.wb.norm[row] * kmax * 1.001f;   // 2^-15 ...
+            const int jb = 0xFFFF - static_cast<int>(thr & 0xFFFFull);
+            const float sb = __ldg(srow + jb);
+            uint32_t exact = 0u;          // bit u: key[u] holds the exact order value
+            double qx[D / 32];            // this lane's channels of Qp_i, exact, loaded on first use
+            bool have_q = false;
+            for (float W = 4.0f * E;; W *= 2.0f) {
+              bool any = false;
+#pragma unroll
+              for (int u = 0; u < NPT; ++u) {
+                const int j = lane + 32 * u;
+                any |= (j < NB) && j != jb && fabsf(sv(u) - sb) <= W;
+              }
+              if (!__any_sync(0xffffffffu, any)) break;   // the fast order is exact around the boundary
+              if (!have_q) {
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                  const long long o = row * D + lane * (D / 32) + c;
+                  const long long plane = prm.BH * NB * static_cast<long long>(D);
+                  qx[c] = static_cast<double>(__bfloat162float(prm.wb.pieces[o])) +
+                          static_cast<double>(__bfloat162float(prm.wb.pieces[plane + o])) +
+                          static_cast<double>(__bfloat162float(prm.wb.pieces[2 * plane + o])) +
+                          static_cast<double>(prm.wb.resid[o]);
+                }
+                have_q = true;
+              }
+              // exact logits for the band (and the boundary block), warp-cooperatively
+#pragma unroll
+              for (int u = 0; u < NPT; ++u) {
+                const int j = lane + 32 * u;
+                const bool need = (j < NB) && !((exact >> u) & 1u) && (j == jb || fabsf(sv(u) - sb) <= W);
+                unsigned todo = __ballot_sync(0xffffffffu, need);
+                while (todo) {
+                  const int src = __ffs(todo) - 1;
+                  todo &= todo - 1u;
+                  const int jj = src + 32 * u;
+                  const long long plane = prm.BH * NB * static_cast<long long>(D);
+                  double part = 0.0;
+#pragma unroll
+                  for (int c = 0; c < D / 32; ++c) {
+                    const long long o = (bh * NB + jj) * static_cast<long long>(D) + lane * (D / 32) + c;
+                    const double kx = static_cast<double>(__bfloat162float(prm.wb.pieces[3 * plane + o])) +
+                                      static_cast<double>(__bfloat162float(prm.wb.pieces[4 * plane + o])) +
+                                      static_cast<double>(__bfloat162float(prm.wb.pieces[5 * plane + o])) +
+                                      static_cast<double>(prm.wb.resid[plane + o]);
+                    part = fma(qx[c], kx, part);
+                  }
+                  part = warp_sum_f64(part) * prm.scale;
+                  if (lane == src) {
+                    key[u] = sel_key(1u, ord64(part) >> 18, jj);
+                    exact |= 1u << u;
+                  }
+                }
+              }
+              // keys: exact inside the band, above or below it elsewhere
+#pragma unroll
+              for (int u = 0; u < NPT; ++u) {
+                const int j = lane + 32 * u;
+                if (j >= NB) continue;
+                const float x = sv(u);
+                const bool in = j == jb || fabsf(x - sb) <= W;
+                if (!in) {
+                  key[u] = sel_key(x > sb ? 2u : 0u, static_cast<unsigned long long>(ord32(x)) << 14, j);
+                } else if (!((exact >> u) & 1u)) {
+                  key[u] = sel_key(1u, 0ull, j);   // not reached: every band member is exact by now
+                }
+              }
+              thr = radix_select<NPT>(key, mass, target, hist);
+              if (thr == 0ull) break;
+              const int j2 = 0xFFFF - static_cast<int>(thr & 0xFFFFull);
+              if (fabsf(__ldg(srow + j2) - sb) <= 0.5f * W) break;   // the boundary stayed inside the band
+              // restore the fast keys of the elements outside the wider band next round (done above)
+            }
+          }
+        }
+        // ---- keep set, sliding-tile union, bits and lists
+        const int qx_ = i % prm.nX, qy_ = (i / prm.nX) % prm.nY, qt_ = i / (prm.nX * prm.nY);
+        uint32_t* brow = prm.bits + row * NW;
+        int16_t* irow = prm.idx + row * NB;
+        int base = 0;
+#pragma unroll
+        for (int u = 0; u < NPT; ++u) {
+          const int j = lane + 32 * u;
+          bool keep = false;
+          if (j < NB) {
+            keep = key[u] >= thr;
+            if (prm.sta_radius >= 0) {
+              const int kx = j % prm.nX, ky = (j / prm.nX) % prm.nY, kt = j / (prm.nX * prm.nY);
+              const int dmax = max(abs(kt - qt_), max(abs(ky - qy_), abs(kx - qx_)));
+              keep = keep || (dmax <= prm.sta_radius);
+            }
+          }
+          const unsigned w = __ballot_sync(0xffffffffu, keep);
+          if (u < NW && lane == 0) brow[u] = w;
+          if (keep) irow[base + __popc(w & ((1u << lane) - 1u))] = static_cast<int16_t>(j);
+          base += __popc(w);
+        }
+        if (lane == 0) prm.count[row] = base;
+}
+
+}  // namespace dbst

@@ -71,14 +71,19 @@ dbst_status dbst_tile_reorder(const void* x_bf16, void* y_bf16, const dbst_geom*
 /* Inverse of dbst_tile_reorder: tiled [B,H,N,D] -> raster [B,H,N,D]. */
 dbst_status dbst_tile_unreorder(const void* y_bf16, void* x_bf16, const dbst_geom* g, void* stream);
 
-/* Bytes of device scratch that dbst_build_block_mask needs for geometry g. */
+/* Bytes of device scratch that the mask builders (dbst_build_block_mask[_raster],
+ * dbst_build_sip_mask[_raster]) need for geometry g. */
 size_t dbst_mask_workspace_bytes(const dbst_geom* g);
 
 /*
  * Adaptive block mask (NABLA page, "Construction de Masque Adaptatif" and
  * "Intégration Hybride avec STA").
  *   1. Qp, Kp = mean of each block's 64 tiled tokens (float64, exact).
- *   2. A[i,:] = softmax_j(<Qp_i, Kp_j> / sqrt(D)) per (b, h), float64.
+ *   2. A[i,:] = softmax_j(<Qp_i, Kp_j> / sqrt(D)) per (b, h).  Rows of at most
+ *      1024 blocks take the logits from the tensor cores (three bf16 pieces of
+ *      each mean) and recompute in float64 every key whose logit lies within
+ *      the error bound of the selection boundary's, so the order matches the
+ *      float64 one; longer rows use float64 logits throughout.
  *   3. Row i keeps the smallest set of key blocks whose mass reaches p:
  *      blocks sorted by A descending (ties: lower index first), keep the
  *      shortest prefix whose cumulative sum is >= p; p == 1 keeps all.

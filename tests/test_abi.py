@@ -118,8 +118,12 @@ def test_workspace_size_formula(lib):
 
     def up(x):
         return (x + 255) // 256 * 256
-    expect = 2 * up(bh * nb * 64 * 8) + up(bh * nb * nb * 8)
-    assert lib.dbst_mask_workspace_bytes(ctypes.byref(g)) == expect
+    # float64 layout (SIP mask, rows of more than 1024 blocks): block means of q and k, pooled logits
+    f64 = 2 * up(bh * nb * 64 * 8) + up(bh * nb * nb * 8)
+    # tensor-core layout: per-head max key norm, 6 bf16 pieces and 2 float32 residuals of the means,
+    # 2 norms per block, the float32 pooled logits
+    tc = up(bh * 4) + up(6 * bh * nb * 64 * 2) + up(2 * bh * nb * 64 * 4) + up(2 * bh * nb * 4) + up(bh * nb * nb * 4)
+    assert lib.dbst_mask_workspace_bytes(ctypes.byref(g)) == max(f64, tc)
 
 
 def test_python_binding_validates_shapes_before_calling():
