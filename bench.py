@@ -6,8 +6,8 @@ N=37632, 588 blocks; CDF threshold p=0.9; seeded synthetic q/k/v).  Default
 (`--path fused`): raster q, k, v in, raster o out, the tile reorder done by the
 kernels' own loads and stores:
     build_block_mask_raster(q, k) -> pair_query_blocks -> block_sparse_attn_raster(q, k, v, pairs) -> o
-(6 launches: a memset and three kernels for the mask (block means, pooled logits on the tensor cores,
-row selection), the query-block pairing, the attention).  `--path explicit` runs
+(7 launches: a memset and four kernels for the mask (block means, pooled logits on the tensor cores,
+row selection, float64 refinement of the rows that need it), the query-block pairing, the attention).  `--path explicit` runs
 the same steps as separate passes (8 launches):
     tile_reorder(q, k, v) -> build_block_mask -> block_sparse_attn -> tile_unreorder(o)
 
@@ -589,7 +589,7 @@ def main():
     stream = torch.cuda.current_stream()
     fused = args.path == "fused"
     # fused: pool + logits + select + pairing + attention; explicit: 3 reorders + 4 + unreorder
-    launches_per_step = 5 if fused else 8   # kernels of this library (the memset is the runtime's)
+    launches_per_step = 6 if fused else 9   # kernels of this library (the memset is the runtime's)
     pairs = torch.empty((g.B, g.H, (g.NB + 1) // 2), dtype=torch.int32, device="cuda")
 
     ev = {}

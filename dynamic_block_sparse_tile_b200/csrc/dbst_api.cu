@@ -146,19 +146,20 @@ MaskWorkspace mask_workspace(const dbst_geom* g) {
 // Tensor-core mask build (rows of at most kMaskTcMaxNB blocks): pool counters, pieces, residuals, norms.
 constexpr int kMaskTcMaxNB = 1024;
 struct MaskTcWorkspace {
-  size_t kmax, pieces, resid, norm, s, total;
+  size_t kmax, pieces, resid, norm, s, refine, total;
 };
 MaskTcWorkspace mask_tc_workspace(const dbst_geom* g) {
   const size_t nb = static_cast<size_t>(nblocks(g));
   const size_t bh = static_cast<size_t>(bh_count(g));
   const size_t d = static_cast<size_t>(g->D);
   MaskTcWorkspace w;
-  w.kmax = 0;                                             // kmax [BH]
-  w.pieces = align_up(bh * sizeof(unsigned int));
+  w.kmax = 0;                                             // kmax [BH], then the refine-list length
+  w.pieces = align_up((bh + 1) * sizeof(unsigned int));
   w.resid = w.pieces + align_up(6 * bh * nb * d * 2);
   w.norm = w.resid + align_up(2 * bh * nb * d * sizeof(float));
   w.s = w.norm + align_up(2 * bh * nb * sizeof(float));   // fast pooled logits [BH][NB][NB] float32
-  w.total = w.s + align_up(bh * nb * nb * sizeof(float));
+  w.refine = w.s + align_up(bh * nb * nb * sizeof(float)); // rows for the float64 refinement [BH * NB] int2
+  w.total = w.refine + align_up(bh * nb * 8);
   return w;
 }
 // The workspace of every mask builder: the float64 layout of the SIP mask and of rows longer than
@@ -582,6 +583,11 @@ bool launch_select_rows(const dbst::SelRowsParams& prm, cudaStream_t s) {
   const long long rows = prm.BH * prm.NB;
   const long long grid = (rows + dbst::kSelRowsWarps - 1) / dbst::kSelRowsWarps;
   dbst::select_rows_kernel<D, NPT><<<static_cast<unsigned>(grid), 32 * dbst::kSelRowsWarps, 0, s>>>(prm);
+  if (cudaGetLastError() != cudaSuccess) return false;
+  // the listed rows (a small share): persistent warps walk the list
+  long long rgrid = static_cast<long long>(sm_count()) * 4;
+  if (rgrid > grid) rgrid = grid;
+  dbst::refine_rows_kernel<D, NPT><<<static_cast<unsigned>(rgrid), 32 * dbst::kSelRowsWarps, 0, s>>>(prm);
   return cudaGetLastError() == cudaSuccess;
 }
 
@@ -609,7 +615,7 @@ dbst_status build_mask_tc(const void* q, const void* k, const dbst_geom* g, floa
   wb.pieces = reinterpret_cast<__nv_bfloat16*>(ws + w.pieces);
   wb.resid = reinterpret_cast<float*>(ws + w.resid);
   wb.norm = reinterpret_cast<float*>(ws + w.norm);
-  if (cudaMemsetAsync(ws + w.kmax, 0, BH * sizeof(unsigned int), s) != cudaSuccess) return DBST_ECUDA;
+  if (cudaMemsetAsync(ws + w.kmax, 0, (BH + 1) * sizeof(unsigned int), s) != cudaSuccess) return DBST_ECUDA;
   {  // 1. block means as pieces, residuals and norms
     const long long warps = 2 * BH * NB;
     long long grid = (warps * 32 + dbst::kPoolTcThreads - 1) / dbst::kPoolTcThreads;
@@ -661,6 +667,8 @@ dbst_status build_mask_tc(const void* q, const void* k, const dbst_geom* g, floa
   dbst::SelRowsParams prm;
   prm.wb = wb;
   prm.S = S;
+  prm.refine_count = wb.kmax + BH;
+  prm.refine = reinterpret_cast<int2*>(ws + w.refine);
   prm.bits = mask_bits;
   prm.count = kv_count;
   prm.idx = kv_idx;

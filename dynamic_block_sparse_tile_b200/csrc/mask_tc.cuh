@@ -18,9 +18,10 @@
 //   float32 map in the workspace (small enough to stay in L2 for the next
 //   kernel).
 //
-//   select_rows_kernel, one warp per row and many rows in flight per SM, takes
-//   the CDF selection by a radix select on the row's keys with integer masses
-//   and writes bits and lists.
+//   select_rows_kernel, one warp per row and many rows in flight per SM, finds
+//   the CDF boundary by bisection on the logit value with exact integer mass
+//   sums (one warp reduction per step), settles the order near the boundary
+//   (below) with a radix select on exact keys, and writes bits and lists.
 //
 // Exactness.  The order of a row's blocks must be the order of the exact
 // (float64) logits.  The fast logits carry an error below E = 2^-15 * scale *
@@ -32,7 +33,7 @@
 // all other keys placed above or below the band.  The result stands if the new
 // boundary lies within 2E of the old one; otherwise the band doubles and the
 // step repeats.  Masses are float32 exponentials of the fast logits, rounded to
-// integers of 2^-26 of the row's largest and summed exactly; a kept set can therefore differ from a
+// integers of 2^-21 of the row's largest and summed exactly; a kept set can therefore differ from a
 // float64 reference only where a cumulative mass lies within rounding of p.
 #pragma once
 #include <cstdint>
@@ -195,6 +196,8 @@ constexpr int kHistStride = 17;          // words per lane of a warp's radix-sel
 struct SelRowsParams {
   MaskTcBuffers wb;
   const float* S;      // [BH][NB][NB] fast pooled logits
+  unsigned int* refine_count;   // rows listed for refine_rows_kernel (zeroed before the selection)
+  int2* refine;        // [BH * NB] listed rows: (row, float bits of the boundary's fast logit)
   uint32_t* bits;
   int32_t* count;
   int16_t* idx;
@@ -489,149 +492,250 @@ __global__ void __launch_bounds__(kLogTcThreads, 1)
 }
 
 
-// One warp per query-block row of the fast pooled logits: integer masses, radix select of the CDF
-// boundary, the exactness band around it, the sliding-tile union, bits and lists.
+// ---------------------------------------------------------------------------
+// Row selection.  select_rows_kernel (one warp per row) finds the CDF boundary of every row by
+// bisection on its fast logits; a row whose boundary has other blocks within the error band goes to
+// a list that refine_rows_kernel settles with float64 logits.  Both write bits, lists and counts
+// through emit_row.
+// ---------------------------------------------------------------------------
+
+// Bits, list and count of one row from this lane's keep flags (bit u: block lane + 32u), with the
+// sliding-tile neighbourhood added.
+template <int NPT>
+__device__ __forceinline__ void emit_row(const SelRowsParams& prm, long long row, int i, uint32_t keepm) {
+  const int lane = threadIdx.x & 31;
+  const int NB = prm.NB, NW = prm.NW;
+  const int qx_ = i % prm.nX, qy_ = (i / prm.nX) % prm.nY, qt_ = i / (prm.nX * prm.nY);
+  uint32_t* brow = prm.bits + row * NW;
+  int16_t* irow = prm.idx + row * NB;
+  int base = 0;
+#pragma unroll
+  for (int u = 0; u < NPT; ++u) {
+    const int j = lane + 32 * u;
+    bool keep = false;
+    if (j < NB) {
+      keep = (keepm >> u) & 1u;
+      if (prm.sta_radius >= 0) {
+        const int kx = j % prm.nX, ky = (j / prm.nX) % prm.nY, kt = j / (prm.nX * prm.nY);
+        const int dmax = max(abs(kt - qt_), max(abs(ky - qy_), abs(kx - qx_)));
+        keep = keep || (dmax <= prm.sta_radius);
+      }
+    }
+    const unsigned w = __ballot_sync(0xffffffffu, keep);
+    if (u < NW && lane == 0) brow[u] = w;
+    if (keep) irow[base + __popc(w & ((1u << lane) - 1u))] = static_cast<int16_t>(j);
+    base += __popc(w);
+  }
+  if (lane == 0) prm.count[row] = base;
+}
+
+// A row's fast logits (-inf past NB), max and min, masses e^(s - max) as integers in units of 2^-21
+// of the row's largest (a row of at most 1024 blocks sums below 2^31, so every sum is exact in 32 bits
+// and independent of its order), and the cumulative mass to reach: p of the total, rounded up.
+template <int NPT>
+__device__ __forceinline__ void load_row(const SelRowsParams& prm, const float* srow, float (&s)[NPT],
+                                         uint32_t (&mass)[NPT], float& mx, float& mn, unsigned long long& target) {
+  const int lane = threadIdx.x & 31;
+  mx = -INFINITY;
+  mn = INFINITY;
+#pragma unroll
+  for (int u = 0; u < NPT; ++u) {
+    const bool v = lane + 32 * u < prm.NB;
+    s[u] = v ? __ldg(srow + lane + 32 * u) : -INFINITY;
+    mx = fmaxf(mx, s[u]);
+    if (v) mn = fminf(mn, s[u]);
+  }
+  mx = warp_max_f32(mx);
+  mn = -warp_max_f32(-mn);
+  uint32_t lsum = 0u;
+#pragma unroll
+  for (int u = 0; u < NPT; ++u) {
+    mass[u] = (s[u] != -INFINITY) ? __float2uint_rn(fast_exp2((s[u] - mx) * 1.4426950408889634f) * 2097152.0f) : 0u;
+    lsum += mass[u];
+  }
+  const uint32_t total = __reduce_add_sync(0xffffffffu, lsum);
+  target = static_cast<unsigned long long>(ceil(prm.p * static_cast<double>(total)));
+}
+
+// Bound of the fast logits' error for row `row` (see the file header).
+__device__ __forceinline__ float logit_error_bound(const SelRowsParams& prm, long long row, long long bh) {
+  return 3.0517578125e-05f * prm.scale_f * prm.wb.norm[row] * __uint_as_float(prm.wb.kmax[bh]) * 1.001f;
+}
+
 // At least four blocks (16 warps) per SM: the rows are latency-bound, so rows in flight matter.
 template <int D, int NPT>
 __global__ void __launch_bounds__(32 * kSelRowsWarps, 4) select_rows_kernel(const SelRowsParams prm) {
-  __shared__ uint32_t s_hist[kSelRowsWarps][32 * kHistStride];
   const int lane = threadIdx.x & 31, wk = threadIdx.x >> 5;
   const long long rows = prm.BH * prm.NB;
   const long long row = static_cast<long long>(blockIdx.x) * kSelRowsWarps + wk;
   if (row >= rows) return;                       // whole warps only
-  const int NB = prm.NB, NW = prm.NW;
+  const int NB = prm.NB;
   const long long bh = row / NB;
   const int i = static_cast<int>(row - bh * NB);
-  uint32_t* hist = s_hist[wk];
-  const float scale_f = prm.scale_f;
-  const float kmax = __uint_as_float(prm.wb.kmax[bh]);
   const float* srow = prm.S + row * NB;
-        // fast logits, masses and keys
-        // the row is read through L1 wherever it is needed
-        auto sv = [&](int u) -> float { return __ldg(srow + lane + 32 * u); };   // valid for j = lane + 32u < NB
-        uint32_t mass[NPT];               // e^(s - max) in units of 2^-26
-        unsigned long long key[NPT];
-        float mx = -INFINITY;
+  float s[NPT];
+  uint32_t mass[NPT];
+  float mx, mn;
+  unsigned long long target;
+  load_row<NPT>(prm, srow, s, mass, mx, mn, target);
+  if (!(prm.p < 1.0)) {                          // p = 1 keeps every block
+    emit_row<NPT>(prm, row, i, 0xFFFFFFFFu);
+    return;
+  }
+  // mass of the blocks whose fast logit is at least t
+  auto mass_from = [&](float t) -> unsigned long long {
+    uint32_t acc = 0u;
 #pragma unroll
-        for (int u = 0; u < NPT; ++u)
-          if (lane + 32 * u < NB) mx = fmaxf(mx, sv(u));
-        mx = warp_max_f32(mx);
-        unsigned long long total = 0ull;
+    for (int u = 0; u < NPT; ++u) acc += (s[u] >= t) ? mass[u] : 0u;
+    return __reduce_add_sync(0xffffffffu, acc);
+  };
+  const float E = logit_error_bound(prm, row, bh);
+  float sb = mx;                                 // fast logit of the boundary block
+  if (mass_from(mx) < target) {
+    // bisection on the logit value: mass_from(lo) >= target > mass_from(hi) throughout; the boundary
+    // block's fast logit lies in [lo, hi), and once that interval is narrower than E / 2 the band
+    // settles the order inside it
+    float lo = mn, hi = mx;
+    for (int it = 0; it < 64 && hi - lo > 0.5f * E; ++it) {
+      const float mid = 0.5f * (lo + hi);
+      if (!(mid > lo && mid < hi)) break;
+      if (mass_from(mid) >= target) lo = mid;
+      else hi = mid;
+    }
+    float c = -INFINITY;
 #pragma unroll
-        for (int u = 0; u < NPT; ++u) {
-          const int j = lane + 32 * u;
-          const float x = (j < NB) ? sv(u) : 0.0f;
-          mass[u] = (j < NB) ? __float2uint_rn(fast_exp2((x - mx) * 1.4426950408889634f) * 67108864.0f) : 0u;
-          total += mass[u];
-          key[u] = (j < NB) ? sel_key(1u, static_cast<unsigned long long>(ord32(x)) << 14, j) : 0ull;
-        }
+    for (int u = 0; u < NPT; ++u)
+      if (s[u] >= lo && s[u] < hi) c = fmaxf(c, s[u]);
+    sb = warp_max_f32(c);
+  }
+  // another block within the error band of the boundary: the order there needs float64 logits
+  int inband = 0;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) total += __shfl_xor_sync(0xffffffffu, total, off);
-        // cumulative mass to reach: p of the total, rounded up
-        const unsigned long long target = static_cast<unsigned long long>(ceil(prm.p * static_cast<double>(total)));
-        unsigned long long thr = 0ull;   // keep key >= thr (0 keeps all)
-        if (prm.p < 1.0) {
+  for (int u = 0; u < NPT; ++u) inband += (s[u] != -INFINITY && fabsf(s[u] - sb) <= 4.0f * E) ? 1 : 0;
+  if (__reduce_add_sync(0xffffffffu, inband) > 1) {
+    if (lane == 0) {
+      const unsigned k = atomicAdd(prm.refine_count, 1u);
+      prm.refine[k] = make_int2(static_cast<int>(row), __float_as_int(sb));
+    }
+    return;
+  }
+  uint32_t keepm = 0u;
+#pragma unroll
+  for (int u = 0; u < NPT; ++u) keepm |= (s[u] >= sb ? 1u : 0u) << u;
+  emit_row<NPT>(prm, row, i, keepm);
+}
+
+// The listed rows: exact order inside the error band of the boundary (see the file header).
+// Persistent: warps walk the list.
+template <int D, int NPT>
+__global__ void __launch_bounds__(32 * kSelRowsWarps) refine_rows_kernel(const SelRowsParams prm) {
+  __shared__ uint32_t s_hist[kSelRowsWarps][32 * kHistStride];
+  const int lane = threadIdx.x & 31, wk = threadIdx.x >> 5;
+  uint32_t* hist = s_hist[wk];
+  const int NB = prm.NB;
+  const unsigned n = *prm.refine_count;
+  for (long long e = static_cast<long long>(blockIdx.x) * kSelRowsWarps + wk; e < n;
+       e += static_cast<long long>(gridDim.x) * kSelRowsWarps) {
+    const int2 ent = prm.refine[e];
+    const long long row = ent.x;
+    const float sb = __int_as_float(ent.y);
+    const long long bh = row / NB;
+    const int i = static_cast<int>(row - bh * NB);
+    const float* srow = prm.S + row * NB;
+    float s[NPT];
+    uint32_t mass[NPT];
+    float mx, mn;
+    unsigned long long target;
+    load_row<NPT>(prm, srow, s, mass, mx, mn, target);
+    auto sv = [&](int u) -> float { return s[u]; };
+    const float E = logit_error_bound(prm, row, bh);
+    int jb = -1;                                 // the boundary block: the lowest index with the boundary logit
+#pragma unroll
+    for (int u = NPT - 1; u >= 0; --u) {
+      const unsigned eqm = __ballot_sync(0xffffffffu, s[u] == sb);
+      if (eqm) jb = 32 * u + __ffs(eqm) - 1;
+    }
+    unsigned long long key[NPT];
+#pragma unroll
+    for (int u = 0; u < NPT; ++u) {
+      const int j = lane + 32 * u;
+      key[u] = (j < NB) ? sel_key(1u, static_cast<unsigned long long>(ord32(s[u])) << 14, j) : 0ull;
+    }
+    unsigned long long thr = sel_key(1u, static_cast<unsigned long long>(ord32(sb)) << 14, jb);
+        uint32_t exact = 0u;          // bit u: key[u] holds the exact order value
+        double qx[D / 32];            // this lane's channels of Qp_i, exact, loaded on first use
+        bool have_q = false;
+        for (float W = 4.0f * E;; W *= 2.0f) {
+          bool any = false;
+#pragma unroll
+          for (int u = 0; u < NPT; ++u) {
+            const int j = lane + 32 * u;
+            any |= (j < NB) && j != jb && fabsf(sv(u) - sb) <= W;
+          }
+          if (!__any_sync(0xffffffffu, any)) break;   // the fast order is exact around the boundary
+          if (!have_q) {
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              const long long o = row * D + lane * (D / 32) + c;
+              const long long plane = prm.BH * NB * static_cast<long long>(D);
+              qx[c] = static_cast<double>(__bfloat162float(prm.wb.pieces[o])) +
+                      static_cast<double>(__bfloat162float(prm.wb.pieces[plane + o])) +
+                      static_cast<double>(__bfloat162float(prm.wb.pieces[2 * plane + o])) +
+                      static_cast<double>(prm.wb.resid[o]);
+            }
+            have_q = true;
+          }
+          // exact logits for the band (and the boundary block), warp-cooperatively
+#pragma unroll
+          for (int u = 0; u < NPT; ++u) {
+            const int j = lane + 32 * u;
+            const bool need = (j < NB) && !((exact >> u) & 1u) && (j == jb || fabsf(sv(u) - sb) <= W);
+            unsigned todo = __ballot_sync(0xffffffffu, need);
+            while (todo) {
+              const int src = __ffs(todo) - 1;
+              todo &= todo - 1u;
+              const int jj = src + 32 * u;
+              const long long plane = prm.BH * NB * static_cast<long long>(D);
+              double part = 0.0;
+#pragma unroll
+              for (int c = 0; c < D / 32; ++c) {
+                const long long o = (bh * NB + jj) * static_cast<long long>(D) + lane * (D / 32) + c;
+                const double kx = static_cast<double>(__bfloat162float(prm.wb.pieces[3 * plane + o])) +
+                                  static_cast<double>(__bfloat162float(prm.wb.pieces[4 * plane + o])) +
+                                  static_cast<double>(__bfloat162float(prm.wb.pieces[5 * plane + o])) +
+                                  static_cast<double>(prm.wb.resid[plane + o]);
+                part = fma(qx[c], kx, part);
+              }
+              part = warp_sum_f64(part) * prm.scale;
+              if (lane == src) {
+                key[u] = sel_key(1u, ord64(part) >> 18, jj);
+                exact |= 1u << u;
+              }
+            }
+          }
+          // keys: exact inside the band, above or below it elsewhere
+#pragma unroll
+          for (int u = 0; u < NPT; ++u) {
+            const int j = lane + 32 * u;
+            if (j >= NB) continue;
+            const float x = sv(u);
+            const bool in = j == jb || fabsf(x - sb) <= W;
+            if (!in) {
+              key[u] = sel_key(x > sb ? 2u : 0u, static_cast<unsigned long long>(ord32(x)) << 14, j);
+            } else if (!((exact >> u) & 1u)) {
+              key[u] = sel_key(1u, 0ull, j);   // not reached: every band member is exact by now
+            }
+          }
           thr = radix_select<NPT>(key, mass, target, hist);
-          if (thr != 0ull) {
-            // ---- exactness band around the boundary block
-            const float E = 3.0517578125e-05f * scale_f * prm.wb.norm[row] * kmax * 1.001f;   // 2^-15 ...
-            const int jb = 0xFFFF - static_cast<int>(thr & 0xFFFFull);
-            const float sb = __ldg(srow + jb);
-            uint32_t exact = 0u;          // bit u: key[u] holds the exact order value
-            double qx[D / 32];            // this lane's channels of Qp_i, exact, loaded on first use
-            bool have_q = false;
-            for (float W = 4.0f * E;; W *= 2.0f) {
-              bool any = false;
-#pragma unroll
-              for (int u = 0; u < NPT; ++u) {
-                const int j = lane + 32 * u;
-                any |= (j < NB) && j != jb && fabsf(sv(u) - sb) <= W;
-              }
-              if (!__any_sync(0xffffffffu, any)) break;   // the fast order is exact around the boundary
-              if (!have_q) {
-#pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                  const long long o = row * D + lane * (D / 32) + c;
-                  const long long plane = prm.BH * NB * static_cast<long long>(D);
-                  qx[c] = static_cast<double>(__bfloat162float(prm.wb.pieces[o])) +
-                          static_cast<double>(__bfloat162float(prm.wb.pieces[plane + o])) +
-                          static_cast<double>(__bfloat162float(prm.wb.pieces[2 * plane + o])) +
-                          static_cast<double>(prm.wb.resid[o]);
-                }
-                have_q = true;
-              }
-              // exact logits for the band (and the boundary block), warp-cooperatively
-#pragma unroll
-              for (int u = 0; u < NPT; ++u) {
-                const int j = lane + 32 * u;
-                const bool need = (j < NB) && !((exact >> u) & 1u) && (j == jb || fabsf(sv(u) - sb) <= W);
-                unsigned todo = __ballot_sync(0xffffffffu, need);
-                while (todo) {
-                  const int src = __ffs(todo) - 1;
-                  todo &= todo - 1u;
-                  const int jj = src + 32 * u;
-                  const long long plane = prm.BH * NB * static_cast<long long>(D);
-                  double part = 0.0;
-#pragma unroll
-                  for (int c = 0; c < D / 32; ++c) {
-                    const long long o = (bh * NB + jj) * static_cast<long long>(D) + lane * (D / 32) + c;
-                    const double kx = static_cast<double>(__bfloat162float(prm.wb.pieces[3 * plane + o])) +
-                                      static_cast<double>(__bfloat162float(prm.wb.pieces[4 * plane + o])) +
-                                      static_cast<double>(__bfloat162float(prm.wb.pieces[5 * plane + o])) +
-                                      static_cast<double>(prm.wb.resid[plane + o]);
-                    part = fma(qx[c], kx, part);
-                  }
-                  part = warp_sum_f64(part) * prm.scale;
-                  if (lane == src) {
-                    key[u] = sel_key(1u, ord64(part) >> 18, jj);
-                    exact |= 1u << u;
-                  }
-                }
-              }
-              // keys: exact inside the band, above or below it elsewhere
-#pragma unroll
-              for (int u = 0; u < NPT; ++u) {
-                const int j = lane + 32 * u;
-                if (j >= NB) continue;
-                const float x = sv(u);
-                const bool in = j == jb || fabsf(x - sb) <= W;
-                if (!in) {
-                  key[u] = sel_key(x > sb ? 2u : 0u, static_cast<unsigned long long>(ord32(x)) << 14, j);
-                } else if (!((exact >> u) & 1u)) {
-                  key[u] = sel_key(1u, 0ull, j);   // not reached: every band member is exact by now
-                }
-              }
-              thr = radix_select<NPT>(key, mass, target, hist);
-              if (thr == 0ull) break;
-              const int j2 = 0xFFFF - static_cast<int>(thr & 0xFFFFull);
-              if (fabsf(__ldg(srow + j2) - sb) <= 0.5f * W) break;   // the boundary stayed inside the band
-              // restore the fast keys of the elements outside the wider band next round (done above)
-            }
-          }
+          if (thr == 0ull) break;
+          const int j2 = 0xFFFF - static_cast<int>(thr & 0xFFFFull);
+          if (fabsf(__ldg(srow + j2) - sb) <= 0.5f * W) break;   // the boundary stayed inside the band
         }
-        // ---- keep set, sliding-tile union, bits and lists
-        const int qx_ = i % prm.nX, qy_ = (i / prm.nX) % prm.nY, qt_ = i / (prm.nX * prm.nY);
-        uint32_t* brow = prm.bits + row * NW;
-        int16_t* irow = prm.idx + row * NB;
-        int base = 0;
+    uint32_t keepm = 0u;
 #pragma unroll
-        for (int u = 0; u < NPT; ++u) {
-          const int j = lane + 32 * u;
-          bool keep = false;
-          if (j < NB) {
-            keep = key[u] >= thr;
-            if (prm.sta_radius >= 0) {
-              const int kx = j % prm.nX, ky = (j / prm.nX) % prm.nY, kt = j / (prm.nX * prm.nY);
-              const int dmax = max(abs(kt - qt_), max(abs(ky - qy_), abs(kx - qx_)));
-              keep = keep || (dmax <= prm.sta_radius);
-            }
-          }
-          const unsigned w = __ballot_sync(0xffffffffu, keep);
-          if (u < NW && lane == 0) brow[u] = w;
-          if (keep) irow[base + __popc(w & ((1u << lane) - 1u))] = static_cast<int16_t>(j);
-          base += __popc(w);
-        }
-        if (lane == 0) prm.count[row] = base;
+    for (int u = 0; u < NPT; ++u) keepm |= (key[u] != 0ull && key[u] >= thr ? 1u : 0u) << u;
+    emit_row<NPT>(prm, row, i, keepm);
+  }
 }
 
 }  // namespace dbst

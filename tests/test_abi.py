@@ -120,9 +120,10 @@ def test_workspace_size_formula(lib):
         return (x + 255) // 256 * 256
     # float64 layout (SIP mask, rows of more than 1024 blocks): block means of q and k, pooled logits
     f64 = 2 * up(bh * nb * 64 * 8) + up(bh * nb * nb * 8)
-    # tensor-core layout: per-head max key norm, 6 bf16 pieces and 2 float32 residuals of the means,
-    # 2 norms per block, the float32 pooled logits
-    tc = up(bh * 4) + up(6 * bh * nb * 64 * 2) + up(2 * bh * nb * 64 * 4) + up(2 * bh * nb * 4) + up(bh * nb * nb * 4)
+    # tensor-core layout: per-head max key norm and the refine-list length, 6 bf16 pieces and 2 float32
+    # residuals of the means, 2 norms per block, the float32 pooled logits, the refine list
+    tc = (up((bh + 1) * 4) + up(6 * bh * nb * 64 * 2) + up(2 * bh * nb * 64 * 4) + up(2 * bh * nb * 4) +
+          up(bh * nb * nb * 4) + up(bh * nb * 8))
     assert lib.dbst_mask_workspace_bytes(ctypes.byref(g)) == max(f64, tc)
 
 
