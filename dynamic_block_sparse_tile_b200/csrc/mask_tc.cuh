@@ -316,6 +316,74 @@ __device__ __forceinline__ unsigned long long radix_select(const unsigned long l
   }
 }
 
+// The boundary on keys of the form class | order | index where class 2 (above the band) and class 0
+// (below it) are ordered only coarsely and class 1 (the band) exactly: the mass of class 2 comes
+// first, then the band's members in descending key order.  With at most 32 members they are gathered
+// one per lane (through `h`), sorted by a bitonic network of shuffles and prefix-summed; otherwise,
+// or if the crossing is not among them, radix_select decides.
+template <int NPT>
+__device__ __forceinline__ unsigned long long band_select(const unsigned long long (&key)[NPT],
+                                                         const uint32_t (&M)[NPT], unsigned long long tgt,
+                                                         uint32_t* h) {
+  const int lane = threadIdx.x & 31;
+  uint32_t above_l = 0u;
+  int nm_l = 0;
+#pragma unroll
+  for (int u = 0; u < NPT; ++u) {
+    const unsigned cls = static_cast<unsigned>(key[u] >> 62);
+    if (key[u] != 0ull && cls == 2u) above_l += M[u];
+    if (key[u] != 0ull && cls == 1u) ++nm_l;
+  }
+  const unsigned long long above = __reduce_add_sync(0xffffffffu, above_l);
+  const int nm = __reduce_add_sync(0xffffffffu, nm_l);
+  unsigned hit = 0u;
+  unsigned long long k = 0ull;
+  if (nm > 0 && nm <= 32) {
+    unsigned long long* hk = reinterpret_cast<unsigned long long*>(h);   // 32 keys, then 32 masses
+    uint32_t* hm = h + 64;
+    int off = 0;
+#pragma unroll
+    for (int u = 0; u < NPT; ++u) {
+      const bool mem = key[u] != 0ull && (key[u] >> 62) == 1ull;
+      const unsigned m = __ballot_sync(0xffffffffu, mem);
+      if (mem) {
+        const int slot = off + __popc(m & ((1u << lane) - 1u));
+        hk[slot] = key[u];
+        hm[slot] = M[u];
+      }
+      off += __popc(m);
+    }
+    __syncwarp();
+    k = lane < nm ? hk[lane] : 0ull;
+    uint32_t w = lane < nm ? hm[lane] : 0u;
+    __syncwarp();
+    // bitonic sort of the 32 lanes, descending by key (the empty lanes, key 0, sink to the end)
+#pragma unroll
+    for (int kk = 2; kk <= 32; kk <<= 1) {
+#pragma unroll
+      for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+        const unsigned long long ok = __shfl_xor_sync(0xffffffffu, k, jj);
+        const uint32_t ow = __shfl_xor_sync(0xffffffffu, w, jj);
+        const bool desc = (lane & kk) == 0;      // direction of this lane's sequence (the last: descending)
+        const bool lower = (lane & jj) == 0;
+        if (lower == desc ? (ok > k) : (ok < k)) {
+          k = ok;
+          w = ow;
+        }
+      }
+    }
+    uint32_t incl = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    hit = __ballot_sync(0xffffffffu, lane < nm && above + incl >= tgt);
+  }
+  if (hit == 0u) return radix_select<NPT>(key, M, tgt, h);   // a wide band, or a crossing outside it
+  return __shfl_sync(0xffffffffu, k, __ffs(hit) - 1);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kLogTcThreads, 1)
     pooled_logits_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -629,7 +697,7 @@ __global__ void __launch_bounds__(32 * kSelRowsWarps, 4) select_rows_kernel(cons
 // Persistent: warps walk the list.
 template <int D, int NPT>
 __global__ void __launch_bounds__(32 * kSelRowsWarps) refine_rows_kernel(const SelRowsParams prm) {
-  __shared__ uint32_t s_hist[kSelRowsWarps][32 * kHistStride];
+  __shared__ __align__(16) uint32_t s_hist[kSelRowsWarps][32 * kHistStride];   // rows of 8-byte multiples
   const int lane = threadIdx.x & 31, wk = threadIdx.x >> 5;
   uint32_t* hist = s_hist[wk];
   const int NB = prm.NB;
@@ -662,75 +730,75 @@ __global__ void __launch_bounds__(32 * kSelRowsWarps) refine_rows_kernel(const S
       key[u] = (j < NB) ? sel_key(1u, static_cast<unsigned long long>(ord32(s[u])) << 14, j) : 0ull;
     }
     unsigned long long thr = sel_key(1u, static_cast<unsigned long long>(ord32(sb)) << 14, jb);
-        uint32_t exact = 0u;          // bit u: key[u] holds the exact order value
-        double qx[D / 32];            // this lane's channels of Qp_i, exact, loaded on first use
-        bool have_q = false;
-        for (float W = 4.0f * E;; W *= 2.0f) {
-          bool any = false;
+    uint32_t exact = 0u;          // bit u: key[u] holds the exact order value
+    double qx[D / 32];            // this lane's channels of Qp_i, exact, loaded on first use
+    bool have_q = false;
+    for (float W = 4.0f * E;; W *= 2.0f) {
+      bool any = false;
 #pragma unroll
-          for (int u = 0; u < NPT; ++u) {
-            const int j = lane + 32 * u;
-            any |= (j < NB) && j != jb && fabsf(sv(u) - sb) <= W;
-          }
-          if (!__any_sync(0xffffffffu, any)) break;   // the fast order is exact around the boundary
-          if (!have_q) {
+      for (int u = 0; u < NPT; ++u) {
+        const int j = lane + 32 * u;
+        any |= (j < NB) && j != jb && fabsf(sv(u) - sb) <= W;
+      }
+      if (!__any_sync(0xffffffffu, any)) break;   // the fast order is exact around the boundary
+      if (!have_q) {
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              const long long o = row * D + lane * (D / 32) + c;
-              const long long plane = prm.BH * NB * static_cast<long long>(D);
-              qx[c] = static_cast<double>(__bfloat162float(prm.wb.pieces[o])) +
-                      static_cast<double>(__bfloat162float(prm.wb.pieces[plane + o])) +
-                      static_cast<double>(__bfloat162float(prm.wb.pieces[2 * plane + o])) +
-                      static_cast<double>(prm.wb.resid[o]);
-            }
-            have_q = true;
-          }
-          // exact logits for the band (and the boundary block), warp-cooperatively
-#pragma unroll
-          for (int u = 0; u < NPT; ++u) {
-            const int j = lane + 32 * u;
-            const bool need = (j < NB) && !((exact >> u) & 1u) && (j == jb || fabsf(sv(u) - sb) <= W);
-            unsigned todo = __ballot_sync(0xffffffffu, need);
-            while (todo) {
-              const int src = __ffs(todo) - 1;
-              todo &= todo - 1u;
-              const int jj = src + 32 * u;
-              const long long plane = prm.BH * NB * static_cast<long long>(D);
-              double part = 0.0;
-#pragma unroll
-              for (int c = 0; c < D / 32; ++c) {
-                const long long o = (bh * NB + jj) * static_cast<long long>(D) + lane * (D / 32) + c;
-                const double kx = static_cast<double>(__bfloat162float(prm.wb.pieces[3 * plane + o])) +
-                                  static_cast<double>(__bfloat162float(prm.wb.pieces[4 * plane + o])) +
-                                  static_cast<double>(__bfloat162float(prm.wb.pieces[5 * plane + o])) +
-                                  static_cast<double>(prm.wb.resid[plane + o]);
-                part = fma(qx[c], kx, part);
-              }
-              part = warp_sum_f64(part) * prm.scale;
-              if (lane == src) {
-                key[u] = sel_key(1u, ord64(part) >> 18, jj);
-                exact |= 1u << u;
-              }
-            }
-          }
-          // keys: exact inside the band, above or below it elsewhere
-#pragma unroll
-          for (int u = 0; u < NPT; ++u) {
-            const int j = lane + 32 * u;
-            if (j >= NB) continue;
-            const float x = sv(u);
-            const bool in = j == jb || fabsf(x - sb) <= W;
-            if (!in) {
-              key[u] = sel_key(x > sb ? 2u : 0u, static_cast<unsigned long long>(ord32(x)) << 14, j);
-            } else if (!((exact >> u) & 1u)) {
-              key[u] = sel_key(1u, 0ull, j);   // not reached: every band member is exact by now
-            }
-          }
-          thr = radix_select<NPT>(key, mass, target, hist);
-          if (thr == 0ull) break;
-          const int j2 = 0xFFFF - static_cast<int>(thr & 0xFFFFull);
-          if (fabsf(__ldg(srow + j2) - sb) <= 0.5f * W) break;   // the boundary stayed inside the band
+        for (int c = 0; c < D / 32; ++c) {
+          const long long o = row * D + lane * (D / 32) + c;
+          const long long plane = prm.BH * NB * static_cast<long long>(D);
+          qx[c] = static_cast<double>(__bfloat162float(prm.wb.pieces[o])) +
+                  static_cast<double>(__bfloat162float(prm.wb.pieces[plane + o])) +
+                  static_cast<double>(__bfloat162float(prm.wb.pieces[2 * plane + o])) +
+                  static_cast<double>(prm.wb.resid[o]);
         }
+        have_q = true;
+      }
+      // exact logits for the band (and the boundary block), warp-cooperatively
+#pragma unroll
+      for (int u = 0; u < NPT; ++u) {
+        const int j = lane + 32 * u;
+        const bool need = (j < NB) && !((exact >> u) & 1u) && (j == jb || fabsf(sv(u) - sb) <= W);
+        unsigned todo = __ballot_sync(0xffffffffu, need);
+        while (todo) {
+          const int src = __ffs(todo) - 1;
+          todo &= todo - 1u;
+          const int jj = src + 32 * u;
+          const long long plane = prm.BH * NB * static_cast<long long>(D);
+          double part = 0.0;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            const long long o = (bh * NB + jj) * static_cast<long long>(D) + lane * (D / 32) + c;
+            const double kx = static_cast<double>(__bfloat162float(prm.wb.pieces[3 * plane + o])) +
+                              static_cast<double>(__bfloat162float(prm.wb.pieces[4 * plane + o])) +
+                              static_cast<double>(__bfloat162float(prm.wb.pieces[5 * plane + o])) +
+                              static_cast<double>(prm.wb.resid[plane + o]);
+            part = fma(qx[c], kx, part);
+          }
+          part = warp_sum_f64(part) * prm.scale;
+          if (lane == src) {
+            key[u] = sel_key(1u, ord64(part) >> 18, jj);
+            exact |= 1u << u;
+          }
+        }
+      }
+      // keys: exact inside the band, above or below it elsewhere
+#pragma unroll
+      for (int u = 0; u < NPT; ++u) {
+        const int j = lane + 32 * u;
+        if (j >= NB) continue;
+        const float x = sv(u);
+        const bool in = j == jb || fabsf(x - sb) <= W;
+        if (!in) {
+          key[u] = sel_key(x > sb ? 2u : 0u, static_cast<unsigned long long>(ord32(x)) << 14, j);
+        } else if (!((exact >> u) & 1u)) {
+          key[u] = sel_key(1u, 0ull, j);   // not reached: every band member is exact by now
+        }
+      }
+      thr = band_select<NPT>(key, mass, target, hist);
+      if (thr == 0ull) break;
+      const int j2 = 0xFFFF - static_cast<int>(thr & 0xFFFFull);
+      if (fabsf(__ldg(srow + j2) - sb) <= 0.5f * W) break;   // the boundary stayed inside the band
+    }
     uint32_t keepm = 0u;
 #pragma unroll
     for (int u = 0; u < NPT; ++u) keepm |= (key[u] != 0ull && key[u] >= thr ? 1u : 0u) << u;
