@@ -584,10 +584,15 @@ bool launch_select_rows(const dbst::SelRowsParams& prm, cudaStream_t s) {
   const long long grid = (rows + dbst::kSelRowsWarps - 1) / dbst::kSelRowsWarps;
   dbst::select_rows_kernel<D, NPT><<<static_cast<unsigned>(grid), 32 * dbst::kSelRowsWarps, 0, s>>>(prm);
   if (cudaGetLastError() != cudaSuccess) return false;
-  // the listed rows (a small share): persistent warps walk the list
+  // the listed rows (a small share): persistent warps walk the list; those whose band does not fit a
+  // warp (rare) are flagged for the wide-band kernel, which otherwise only scans the list
   long long rgrid = static_cast<long long>(sm_count()) * 4;
   if (rgrid > grid) rgrid = grid;
   dbst::refine_rows_kernel<D, NPT><<<static_cast<unsigned>(rgrid), 32 * dbst::kSelRowsWarps, 0, s>>>(prm);
+  if (cudaGetLastError() != cudaSuccess) return false;
+  long long wgrid = static_cast<long long>(sm_count()) * 2;
+  if (wgrid > grid) wgrid = grid;
+  dbst::refine_wide_kernel<D, NPT><<<static_cast<unsigned>(wgrid), 32 * dbst::kSelRowsWarps, 0, s>>>(prm);
   return cudaGetLastError() == cudaSuccess;
 }
 

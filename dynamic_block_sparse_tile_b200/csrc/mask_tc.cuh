@@ -630,6 +630,117 @@ __device__ __forceinline__ float logit_error_bound(const SelRowsParams& prm, lon
   return 3.0517578125e-05f * prm.scale_f * prm.wb.norm[row] * __uint_as_float(prm.wb.kmax[bh]) * 1.001f;
 }
 
+// A row whose band (the blocks with a fast logit within 4E of the boundary block's) holds several
+// blocks, settled inside the selecting warp when the band fits it: the band's blocks are gathered one
+// per lane (through `gather`, 64 words of shared memory), their float64 logits are computed from the
+// pieces and residuals (one warp-wide dot product each), and the lanes are sorted by exact key with a
+// shuffle bitonic network and prefix-summed after the mass of the blocks above the band.  Returns
+// false, leaving the row to refine_wide_kernel, when the band is wider than a warp or the crossing
+// block's fast logit lies in the outer half of the band (a wider band might then reorder it).
+template <int D, int NPT>
+__device__ __forceinline__ bool band_in_warp(const SelRowsParams& prm, long long row, long long bh,
+                                             const float (&s)[NPT], const uint32_t (&mass)[NPT], float sb, float E,
+                                             unsigned long long target, uint32_t* gather, uint32_t& keepm) {
+  const int lane = threadIdx.x & 31;
+  const int NB = prm.NB;
+  const float W = 4.0f * E;
+  const unsigned lt = (1u << lane) - 1u;
+  uint32_t above_l = 0u;
+  int nm = 0;
+#pragma unroll
+  for (int u = 0; u < NPT; ++u) {
+    const bool valid = s[u] != -INFINITY;
+    const bool mem = valid && fabsf(s[u] - sb) <= W;
+    if (valid && !mem && s[u] > sb) above_l += mass[u];
+    const unsigned bal = __ballot_sync(0xffffffffu, mem);
+    const int slot = nm + __popc(bal & lt);
+    if (mem && slot < 32) {
+      gather[slot] = static_cast<uint32_t>(lane + 32 * u);
+      gather[32 + slot] = mass[u];
+    }
+    nm += __popc(bal);
+  }
+  if (nm > 32) return false;
+  __syncwarp();
+  const int jm = lane < nm ? static_cast<int>(gather[lane]) : 0;
+  uint32_t w = lane < nm ? gather[32 + lane] : 0u;
+  __syncwarp();
+  const unsigned long long above = __reduce_add_sync(0xffffffffu, above_l);
+  // float64 logits of the band's blocks, one warp-wide dot product each
+  const long long plane = prm.BH * NB * static_cast<long long>(D);
+  double qx[D / 32];
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    const long long o = row * D + lane * (D / 32) + c;
+    qx[c] = static_cast<double>(__bfloat162float(prm.wb.pieces[o])) +
+            static_cast<double>(__bfloat162float(prm.wb.pieces[plane + o])) +
+            static_cast<double>(__bfloat162float(prm.wb.pieces[2 * plane + o])) + static_cast<double>(prm.wb.resid[o]);
+  }
+  unsigned long long k = 0ull;
+  for (int m = 0; m < nm; ++m) {
+    const int jj = __shfl_sync(0xffffffffu, jm, m);
+    double part = 0.0;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      const long long o = (bh * NB + jj) * static_cast<long long>(D) + lane * (D / 32) + c;
+      const double kx = static_cast<double>(__bfloat162float(prm.wb.pieces[3 * plane + o])) +
+                        static_cast<double>(__bfloat162float(prm.wb.pieces[4 * plane + o])) +
+                        static_cast<double>(__bfloat162float(prm.wb.pieces[5 * plane + o])) +
+                        static_cast<double>(prm.wb.resid[plane + o]);
+      part = fma(qx[c], kx, part);
+    }
+    part = warp_sum_f64(part) * prm.scale;
+    if (lane == m) k = sel_key(1u, ord64(part) >> 18, jm);
+  }
+  const unsigned long long k0 = k;               // lane m: the key of the band's m-th block (gather order)
+  // bitonic sort of the lanes, descending by key (the empty lanes, key 0, sink to the end)
+#pragma unroll
+  for (int kk = 2; kk <= 32; kk <<= 1) {
+#pragma unroll
+    for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+      const unsigned long long ok = __shfl_xor_sync(0xffffffffu, k, jj);
+      const uint32_t ow = __shfl_xor_sync(0xffffffffu, w, jj);
+      const bool desc = (lane & kk) == 0;
+      const bool lower = (lane & jj) == 0;
+      if (lower == desc ? (ok > k) : (ok < k)) {
+        k = ok;
+        w = ow;
+      }
+    }
+  }
+  uint32_t incl = w;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const unsigned hit = __ballot_sync(0xffffffffu, lane < nm && above + incl >= target);
+  if (hit == 0u) return false;                   // not reached: the band and the blocks above it hold the target
+  const unsigned long long thr = __shfl_sync(0xffffffffu, k, __ffs(hit) - 1);
+  const int jc = 0xFFFF - static_cast<int>(thr & 0xFFFFull);
+  // the crossing block's fast logit (every lane finds it in its own registers, one lane owns it)
+  float xc = -INFINITY;
+#pragma unroll
+  for (int u = 0; u < NPT; ++u)
+    if (lane + 32 * u == jc) xc = s[u];
+  xc = warp_max_f32(xc);
+  if (!(fabsf(xc - sb) <= 0.5f * W)) return false;
+  // keep: above the band, or in the band at or before the crossing in the exact order
+  keepm = 0u;
+  int base = 0;
+#pragma unroll
+  for (int u = 0; u < NPT; ++u) {
+    const bool valid = s[u] != -INFINITY;
+    const bool mem = valid && fabsf(s[u] - sb) <= W;
+    const unsigned bal = __ballot_sync(0xffffffffu, mem);
+    const unsigned long long km = __shfl_sync(0xffffffffu, k0, (base + __popc(bal & lt)) & 31);
+    base += __popc(bal);
+    const bool keep = mem ? (km >= thr) : (valid && s[u] > sb);
+    keepm |= (keep ? 1u : 0u) << u;
+  }
+  return true;
+}
+
 // At least four blocks (16 warps) per SM: the rows are latency-bound, so rows in flight matter.
 template <int D, int NPT>
 __global__ void __launch_bounds__(32 * kSelRowsWarps, 4) select_rows_kernel(const SelRowsParams prm) {
@@ -693,10 +804,39 @@ __global__ void __launch_bounds__(32 * kSelRowsWarps, 4) select_rows_kernel(cons
   emit_row<NPT>(prm, row, i, keepm);
 }
 
-// The listed rows: exact order inside the error band of the boundary (see the file header).
-// Persistent: warps walk the list.
+// The listed rows whose band fits a warp (band_in_warp); the others are flagged in the list (bit 31
+// of the row) for refine_wide_kernel.  Persistent: warps walk the list.
 template <int D, int NPT>
-__global__ void __launch_bounds__(32 * kSelRowsWarps) refine_rows_kernel(const SelRowsParams prm) {
+__global__ void __launch_bounds__(32 * kSelRowsWarps, 4) refine_rows_kernel(const SelRowsParams prm) {
+  __shared__ uint32_t s_gather[kSelRowsWarps][64];
+  const int lane = threadIdx.x & 31, wk = threadIdx.x >> 5;
+  const int NB = prm.NB;
+  const unsigned n = *prm.refine_count;
+  for (long long e = static_cast<long long>(blockIdx.x) * kSelRowsWarps + wk; e < n;
+       e += static_cast<long long>(gridDim.x) * kSelRowsWarps) {
+    const int2 ent = prm.refine[e];
+    const long long row = ent.x;
+    const float sb = __int_as_float(ent.y);
+    const long long bh = row / NB;
+    const int i = static_cast<int>(row - bh * NB);
+    float s[NPT];
+    uint32_t mass[NPT];
+    float mx, mn;
+    unsigned long long target;
+    load_row<NPT>(prm, prm.S + row * NB, s, mass, mx, mn, target);
+    uint32_t km;
+    if (band_in_warp<D, NPT>(prm, row, bh, s, mass, sb, logit_error_bound(prm, row, bh), target, s_gather[wk], km))
+      emit_row<NPT>(prm, row, i, km);
+    else if (lane == 0)
+      prm.refine[e].x = ent.x | static_cast<int>(0x80000000u);
+  }
+}
+
+// The flagged rows of the list: exact order inside a band that is widened until the crossing stays in
+// its inner half (see the file header), with radix_select over keys of 64 bits.  Persistent: warps walk
+// the list and skip the rows refine_rows_kernel settled.
+template <int D, int NPT>
+__global__ void __launch_bounds__(32 * kSelRowsWarps) refine_wide_kernel(const SelRowsParams prm) {
   __shared__ __align__(16) uint32_t s_hist[kSelRowsWarps][32 * kHistStride];   // rows of 8-byte multiples
   const int lane = threadIdx.x & 31, wk = threadIdx.x >> 5;
   uint32_t* hist = s_hist[wk];
@@ -705,7 +845,8 @@ __global__ void __launch_bounds__(32 * kSelRowsWarps) refine_rows_kernel(const S
   for (long long e = static_cast<long long>(blockIdx.x) * kSelRowsWarps + wk; e < n;
        e += static_cast<long long>(gridDim.x) * kSelRowsWarps) {
     const int2 ent = prm.refine[e];
-    const long long row = ent.x;
+    if (ent.x >= 0) continue;                    // settled by refine_rows_kernel
+    const long long row = ent.x & 0x7FFFFFFF;
     const float sb = __int_as_float(ent.y);
     const long long bh = row / NB;
     const int i = static_cast<int>(row - bh * NB);
