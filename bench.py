@@ -6,9 +6,10 @@ N=37632, 588 blocks; CDF threshold p=0.9; seeded synthetic q/k/v).  Default
 (`--path fused`): raster q, k, v in, raster o out, the tile reorder done by the
 kernels' own loads and stores:
     build_block_mask_raster(q, k) -> pair_query_blocks -> block_sparse_attn_raster(q, k, v, pairs) -> o
-(7 launches: a memset and four kernels for the mask (block means, pooled logits on the tensor cores,
-row selection, float64 refinement of the rows that need it), the query-block pairing, the attention).  `--path explicit` runs
-the same steps as separate passes (8 launches):
+(8 launches: a memset and five kernels for the mask (block means, pooled logits on the tensor cores,
+row selection, float64 refinement of the rows whose error band holds several blocks, and of the
+rare rows whose band is wider than a warp), the query-block pairing, the attention).  `--path
+explicit` runs the same steps as separate passes (11 launches, no pairing):
     tile_reorder(q, k, v) -> build_block_mask -> block_sparse_attn -> tile_unreorder(o)
 
 `value` = kept-block TFLOP/s of the whole step (4*D*64*64 FLOP per kept
@@ -389,6 +390,9 @@ def measure_sip(args, w, p, qkv=None) -> dict:
                                                                   out=o, lse=lse), args.steps, args.warmup)
     plain_ms = timed_median(lambda: dbst.block_sparse_attn_offsets(q, k, v, g, cnt, idx, None, raster=True, out=o,
                                                                    lse=lse), args.steps, args.warmup)
+    pairs = dbst.pair_query_blocks(bits, g)
+    fwd_ms = timed_median(lambda: dbst.block_sparse_attn_raster(q, k, v, g, cnt, idx, 0.0, True, o, lse, pairs),
+                          args.steps, args.warmup)
     dbst.get_error()
     kept_sip = int(sip[1].sum().item())
     kept = int(cnt.sum().item())
@@ -396,9 +400,13 @@ def measure_sip(args, w, p, qkv=None) -> dict:
     return {"sip": workload_desc(w, p), "budget_blocks_per_row": budget,
             "kept_fraction_sip": kept_sip / (g.B * g.H * g.NB * g.NB), "sip_mask_ms": sel_ms,
             "sip_attn_ms": attn_ms, "sip_attn_tflops": unit * kept_sip / (attn_ms * 1e-3) / 1e12,
-            "two_sweep_attn_on_nabla_mask_ms": plain_ms,
-            "two_sweep_attn_tflops": unit * kept / (plain_ms * 1e-3) / 1e12,
-            "note": "TFLOP/s count the 2 products of attention per kept block pair; the two-sweep kernel runs 3"}
+            "offset_attn_on_nabla_mask_ms": plain_ms,
+            "offset_attn_on_nabla_mask_tflops": unit * kept / (plain_ms * 1e-3) / 1e12,
+            "forward_on_nabla_mask_ms": fwd_ms,
+            "sip_attn_over_forward": attn_ms / fwd_ms,
+            "note": "TFLOP/s count the 2 products of attention per kept block pair; the offsets ride in the "
+                    "forward kernel's exponent (query blocks paired one tile step apart; the forward here uses "
+                    "the pair list of dbst_pair_query_blocks)"}
 
 
 def run_sip(args, w, p):
@@ -588,8 +596,8 @@ def main():
     o_host = torch.empty_like(host[0]).pin_memory()
     stream = torch.cuda.current_stream()
     fused = args.path == "fused"
-    # fused: pool + logits + select + pairing + attention; explicit: 3 reorders + 4 + unreorder
-    launches_per_step = 6 if fused else 9   # kernels of this library (the memset is the runtime's)
+    # fused: 5 mask kernels + pairing + attention; explicit: 3 reorders + 5 + attention + unreorder
+    launches_per_step = 7 if fused else 10   # kernels of this library (the memset is the runtime's)
     pairs = torch.empty((g.B, g.H, (g.NB + 1) // 2), dtype=torch.int32, device="cuda")
 
     ev = {}

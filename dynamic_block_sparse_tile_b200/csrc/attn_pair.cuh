@@ -9,7 +9,10 @@
 //     S[128 queries x 128 keys] = Q[128 x D] . K_tile[128 x D]^T      (tcgen05 SS, M=128, N=128)
 //     O[128 queries x D]       += P[128 x 128 keys] . V_tile[128 x D]  (tcgen05 TS: P read from TMEM)
 // A key block kept by only one of the two query blocks is masked (P = 0) in
-// the other block's 64 rows.
+// the other block's 64 rows.  With a logit offset per (query block, key block) (SIP's log(1/pi) on
+// the AB-Attention page, section "Les trois techniques"), x = s * scale + offset enters the row max
+// and the exponent in place of s * scale: the exponential warps fold it into the constant of their
+// fused multiply-add, so offsets cost two loads per warp per tile, fetched a tile ahead.
 //
 // TMEM (512 columns): O at 0..D-1, S buffers at 128 and 256, P buffers (bf16
 // pairs, 64 columns each) at 384 and 448.  Because P has its own buffers, S(t+2)
@@ -55,6 +58,8 @@ constexpr float kPairRescale = 16.0f;
 struct PairParams {
   const int32_t* kv_count;   // [BH*NB]; null => dense (every list is 0..NB-1)
   const int16_t* kv_idx;     // [BH*NB*NB]
+  const float* offsets;      // [BH][NB][NB] logit offset (natural log) per (query block, key block), read at
+                             // kept blocks only; null => none
   __nv_bfloat16* o;          // [BH, N, D], tile or raster order (RASTER)
   float* lse;                // [BH, N] in the same order, or null
   int NB, N;
@@ -75,8 +80,8 @@ struct PairSmem {
   static constexpr int kWords = kUnion + 16384;           // u32 [2][128] bitmasks of the two lists
   static constexpr int kScan = kWords + 1024;             // int [128] word offsets
   static constexpr int kRing = kScan + 512;               // float2 [2 tile parities][128 rows]: (m, a)
-  static constexpr int kLsum = kRing + 2048;              // float [2 halves][128 rows]
-  static constexpr int kBars = kLsum + 1024;
+  static constexpr int kLsum = kRing + 2048;              // float [2 sums][2 halves][128 rows]
+  static constexpr int kBars = kLsum + 2048;
   static constexpr int kMisc = kBars + 256;
   static constexpr int kBytes = kMisc + 64;
 };
@@ -115,7 +120,9 @@ __device__ __forceinline__ void umma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, 
 // by the loads themselves (5-D boxes tx x ty x tt tokens x 64 channels land in shared memory in
 // exactly the tile-ordered layout) and by the epilogue, which writes o and lse rows in raster
 // order.  Both produce bit-identical results.
-template <int D, bool RASTER>
+// OFFSETS: the kernel reads PairParams::offsets (compiled apart so that the common case carries no
+// offset bookkeeping).
+template <int D, bool RASTER, bool OFFSETS = false>
 __global__ void __launch_bounds__(kPairThreads, 1)
     pair_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const PairParams prm) {
@@ -294,6 +301,17 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     return;
   }
   const int T = (nu + 1) >> 1;
+  // Logit offsets: the row of offsets of query block qa (side 0) or qb (side 1), null without offsets
+  // (or for the absent second block); offset_of(row, e) is union entry e's offset in log2 units, 0 past
+  // the union's end or without offsets.
+  auto offset_row = [&](int side) -> const float* {
+    if (!OFFSETS || prm.offsets == nullptr || (side == 1 && !has_b)) return nullptr;
+    return prm.offsets + (bh * NB + (side ? qb : qa)) * static_cast<long long>(NB);
+  };
+  auto offset_of = [&](const float* orow, int e) -> float {
+    if constexpr (!OFFSETS) return 0.0f;
+    return (orow != nullptr && e < nu) ? __ldg(orow + (s_union[e] & 0xFFFF)) * 1.4426950408889634f : 0.0f;
+  };
 
   if (warp == 13 || warp == 14) {
     // ------------------------------------------------------------ TMA producers
@@ -388,13 +406,18 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const float sc = prm.scale_log2;
     float m = -INFINITY;                      // running reference max (log2 units) of this row
     bool live = true;
+    const float* orow = offset_row(side);
+    float o0 = offset_of(orow, 0), o1 = offset_of(orow, 1);   // this tile's offsets, fetched a tile ahead
     for (int t = 0; t < T; ++t) {
       const int b = t & 1;
+      const float c0 = o0, c1 = o1;
+      o0 = offset_of(orow, 2 * t + 2);
+      o1 = offset_of(orow, 2 * t + 3);
       wait_live(bar(PB_SFULL + b), (t >> 1) & 1, live);
       tc_fence_after();
       const bool v0 = (s_union[2 * t] >> (16 + side)) & 1;
       const bool v1 = (2 * t + 1 < nu) && ((s_union[2 * t + 1] >> (16 + side)) & 1);
-      float m0 = -INFINITY, m1 = -INFINITY;
+      float tmax = -INFINITY;                 // max over the tile's kept columns of x * scale + offset
 #pragma unroll
       for (int hb = 0; hb < 2; ++hb) {
         if (hb == 0 ? v0 : v1) {
@@ -402,16 +425,18 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           tmem_ld32(tmem + kTmemS + 128u * b + 64u * hb + lrow, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
           tmem_ld32(tmem + kTmemS + 128u * b + 64u * hb + 32u + lrow, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
           tmem_wait_ld();
+          float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
           for (int c = 0; c < 64; c += 4) {
             m0 = fmax3(m0, __uint_as_float(u[c]), __uint_as_float(u[c + 1]));
             m1 = fmax3(m1, __uint_as_float(u[c + 2]), __uint_as_float(u[c + 3]));
           }
+          const float hm = fmaxf(m0, m1) * sc;
+          tmax = fmaxf(tmax, OFFSETS ? hm + (hb == 0 ? c0 : c1) : hm);
         }
       }
       tc_fence_before();
       mbar_arrive(bar(PB_SEMPTY + b));
-      const float tmax = fmaxf(m0, m1) * sc;
       float a = 1.0f;
       if (tmax > m + kPairRescale) {   // also the row's first kept tile (m = -inf)
         if (m != -INFINITY) a = fast_exp2(m - tmax);
@@ -453,10 +478,15 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const float2 sc2 = make_float2(sc, sc);
     float m = -INFINITY;                      // this row's reference for the current tile
     float2 l2 = make_float2(0.0f, 0.0f);      // partial row sum of 2^(x - m) over this warp's columns
+    float2 lb2 = make_float2(0.0f, 0.0f);     // the same sum over the bf16-rounded weights that enter P . V
     bool live = true;
     int ent = (hc < nu) ? s_union[hc] : 0;    // union entry of this warp's key block, one tile ahead
+    const float* orow = offset_row(side);
+    float offn = offset_of(orow, hc);         // its offset (log2 units), one tile ahead
     for (int t = 0; t < T; ++t) {
       const int b = t & 1;
+      const float offc = offn;
+      offn = offset_of(orow, 2 * t + 2 + hc);
       wait_live(bar(PB_MREADY + 4 * b + q), (t >> 1) & 1, live);
       const float2 ma = s_ring[b * 128 + r];
       const bool vh = (2 * t + hc < nu) && ((ent >> (16 + side)) & 1);   // uniform per warp
@@ -464,6 +494,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       m = ma.x;
       l2.x *= ma.y;
       l2.y *= ma.y;
+      lb2.x *= ma.y;
+      lb2.y *= ma.y;
       tc_fence_after();
       uint32_t u[64];
       if (vh) {
@@ -476,13 +508,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       // P = 2^(x*scale - m) on kept columns, 0 elsewhere; bf16 pairs (keys 2c, 2c+1)
       uint32_t pk[32];
       if (vh) {
-        const float2 nm = make_float2(-m, -m);
+        const float2 nm = make_float2(offc - m, offc - m);
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const float2 x = ffma2(make_float2(__uint_as_float(u[2 * c]), __uint_as_float(u[2 * c + 1])), sc2, nm);
           const float2 p = make_float2(fast_exp2(x.x), fast_exp2(x.y));
           l2 = fadd2(l2, p);
           pk[c] = pack_bf16x2(p.x, p.y);
+          lb2 = fadd2(lb2, make_float2(__uint_as_float(pk[c] << 16), __uint_as_float(pk[c] & 0xFFFF0000u)));
         }
       } else {
 #pragma unroll
@@ -496,14 +529,18 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     }
 
     // ---- epilogue: O / l, bf16 store (this warp's half of the columns), log-sum-exp
-    const float lpart = l2.x + l2.y;
+    // o is normalised by the sum of the weights it was accumulated with (the bf16-rounded P), so a row
+    // whose attention sits on one key errs only by o's own rounding; lse takes the float32 sum.
+    const float lpart = l2.x + l2.y, lbpart = lb2.x + lb2.y;
     if (!mbar_wait(bar(PB_DRAIN), 0)) *s_abort = 1;   // every MMA of the CTA has completed
     tc_fence_after();
     s_lsum[hc * 128 + r] = lpart;
+    s_lsum[256 + hc * 128 + r] = lbpart;
     named_bar_sync(1u + static_cast<uint32_t>(q), 64);
     const float lt = lpart + s_lsum[(hc ^ 1) * 128 + r];
+    const float ltb = lbpart + s_lsum[256 + (hc ^ 1) * 128 + r];
     if (side == 0 || has_b) {
-      const float inv = (lt > 0.0f) ? 1.0f / lt : 0.0f;
+      const float inv = (ltb > 0.0f) ? 1.0f / ltb : 0.0f;
       const long long orow = out_row(side ? qb : qa, r & 63);
       uint4* dst = reinterpret_cast<uint4*>(prm.o + orow * D + (D / 2) * hc);
 #pragma unroll

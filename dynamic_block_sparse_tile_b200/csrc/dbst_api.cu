@@ -268,7 +268,8 @@ bool make_tmap_raster_group(CUtensorMap* m, const void* base, const dbst_geom* g
 
 template <int D, bool RASTER>
 dbst_status launch_pair(const void* q, const void* k, const void* v, const dbst_geom* g, const int32_t* cnt,
-                        const int16_t* idx, const int32_t* pairs, float scale, void* o, float* lse, cudaStream_t s) {
+                        const int16_t* idx, const int32_t* pairs, float scale, void* o, float* lse, cudaStream_t s,
+                        const float* offsets = nullptr) {
   const long long rows = bh_count(g) * tokens(g);
   CUtensorMap tq, tk, tv;
   if (RASTER) {
@@ -280,6 +281,7 @@ dbst_status launch_pair(const void* q, const void* k, const void* v, const dbst_
   p.tg = tile_geo(g);
   p.kv_count = cnt;
   p.kv_idx = idx;
+  p.offsets = offsets;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.NB = nblocks(g);
@@ -291,10 +293,15 @@ dbst_status launch_pair(const void* q, const void* k, const void* v, const dbst_
   p.scale_log2 = sc * 1.4426950408889634f;
   p.wait_limit = wait_limit();
   const int smem = dbst::PairSmem::kBytes + 1024;
-  if (!smem_opt_in(dbst::pair_attn_kernel<D, RASTER>, smem)) return DBST_ECUDA;
   const long long grid = bh_count(g) * p.pairs_per_head;
   if (grid >= (1ll << 31)) return DBST_EINVAL;
-  dbst::pair_attn_kernel<D, RASTER><<<static_cast<unsigned>(grid), dbst::kPairThreads, smem, s>>>(tq, tk, tv, p);
+  if (offsets != nullptr) {
+    if (!smem_opt_in(dbst::pair_attn_kernel<D, RASTER, true>, smem)) return DBST_ECUDA;
+    dbst::pair_attn_kernel<D, RASTER, true><<<static_cast<unsigned>(grid), dbst::kPairThreads, smem, s>>>(tq, tk, tv, p);
+  } else {
+    if (!smem_opt_in(dbst::pair_attn_kernel<D, RASTER>, smem)) return DBST_ECUDA;
+    dbst::pair_attn_kernel<D, RASTER><<<static_cast<unsigned>(grid), dbst::kPairThreads, smem, s>>>(tq, tk, tv, p);
+  }
   return launch_status();
 }
 
@@ -522,6 +529,13 @@ dbst_status offset_attn_common(const void* q, const void* k, const void* v, cons
     return DBST_EINVAL;
   if (!std::isfinite(scale)) return DBST_EINVAL;
   auto s = static_cast<cudaStream_t>(stream);
+  if (gmask == nullptr) {   // offsets only: the forward kernel, with the offsets in its exponent
+    if (raster)
+      return g->D == 128 ? launch_pair<128, true>(q, k, v, g, cnt, idx, nullptr, scale, o, lse, s, offsets)
+                         : launch_pair<64, true>(q, k, v, g, cnt, idx, nullptr, scale, o, lse, s, offsets);
+    return g->D == 128 ? launch_pair<128, false>(q, k, v, g, cnt, idx, nullptr, scale, o, lse, s, offsets)
+                       : launch_pair<64, false>(q, k, v, g, cnt, idx, nullptr, scale, o, lse, s, offsets);
+  }
   if (raster)
     return g->D == 128 ? launch_offset_attn<128, true>(q, k, v, g, cnt, idx, offsets, gmask, scale, o, lse, s)
                        : launch_offset_attn<64, true>(q, k, v, g, cnt, idx, offsets, gmask, scale, o, lse, s);
@@ -829,7 +843,9 @@ dbst_status build_sip_mask(const void* q, const void* k, const dbst_geom* g, dou
   long long grid = (rows + dbst::kSipWarps - 1) / dbst::kSipWarps;
   const long long cap = static_cast<long long>(sm_count()) * 16;
   if (grid > cap) grid = cap;
-  dbst::sip_select_kernel<<<static_cast<unsigned>(grid), 32 * dbst::kSipWarps, 0, s>>>(
+  const int smem = dbst::kSipWarps * NB * static_cast<int>(sizeof(double));   // each warp's row of a_j
+  if (smem > 48 * 1024 && !smem_opt_in(dbst::sip_select_kernel, smem)) return DBST_ECUDA;
+  dbst::sip_select_kernel<<<static_cast<unsigned>(grid), 32 * dbst::kSipWarps, smem, s>>>(
       reinterpret_cast<const double*>(ws + w.s), NB, (NB + 31) / 32, rows, budget, uniforms, mask_bits, kv_count,
       kv_idx, offsets);
   return launch_status();

@@ -13,8 +13,10 @@
 //   keep  = u_ij < pi_j for the caller's uniforms u (float64)
 //   offset_ij = log(1 / pi_j) (float32) for kept blocks, 0 elsewhere
 // and the same bitmask and ascending lists as the CDF selection.  Rows longer
-// than 32 blocks are walked in strides of 32; the certainty flags of a row live
-// in shared memory (one bit per block).
+// than 32 blocks are walked in strides of 32; the row's map a_j (one exponential
+// per block) and its certainty flags (one bit per block) live in shared memory
+// (kSipWarps * NB doubles of dynamic shared memory), so the fixed-point rounds
+// only read them.
 #pragma once
 #include <cstdint>
 #include "mask.cuh"
@@ -39,8 +41,10 @@ __global__ void __launch_bounds__(32 * kSipWarps) sip_select_kernel(const double
                                                                     int16_t* __restrict__ idx,
                                                                     float* __restrict__ offsets) {
   __shared__ uint32_t s_cert[kSipWarps][kSipMaxWords];
+  extern __shared__ double s_a[];              // [kSipWarps][NB]
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   uint32_t* cert = s_cert[wib];
+  double* arow = s_a + static_cast<long long>(wib) * NB;
   const long long warp0 = static_cast<long long>(blockIdx.x) * kSipWarps + wib;
   const long long nwarps = static_cast<long long>(gridDim.x) * kSipWarps;
   for (long long row = warp0; row < rows; row += nwarps) {
@@ -51,9 +55,14 @@ __global__ void __launch_bounds__(32 * kSipWarps) sip_select_kernel(const double
     for (int j = lane; j < NB; j += 32) mx = fmax(mx, srow[j]);
     mx = warp_max_f64(mx);
     double sum = 0.0;
-    for (int j = lane; j < NB; j += 32) sum += exp(srow[j] - mx);
+    for (int j = lane; j < NB; j += 32) {
+      const double e = exp(srow[j] - mx);
+      arow[j] = e;
+      sum += e;
+    }
     sum = warp_sum_f64(sum);
-    auto a_of = [&](int j) -> double { return exp(srow[j] - mx) / sum; };
+    for (int j = lane; j < NB; j += 32) arow[j] /= sum;   // each lane rereads only its own entries
+    auto a_of = [&](int j) -> double { return arow[j]; };
     int npos = 0;
     for (int j = lane; j < NB; j += 32) npos += a_of(j) > 0.0;
     npos = warp_sum_i32(npos);
@@ -112,7 +121,7 @@ __global__ void __launch_bounds__(32 * kSipWarps) sip_select_kernel(const double
       base += __popc(m);
     }
     if (lane == 0) count[row] = base;
-    __syncwarp();
+    __syncwarp();   // the next row overwrites cert and arow
   }
 }
 

@@ -201,8 +201,11 @@ dbst_status dbst_pair_query_blocks(const uint32_t* mask_bits, const dbst_geom* g
  *
  * Set-up: the first call on each device (with that device current) looks up
  * the array's device address once; make that first call before any stream
- * capture begins.  All calls share the one array and it keeps the last call's
- * contents; nothing in it needs to start at zero.  Two calls whose kernels
+ * capture begins.  The address is kept for the life of the process, so a
+ * cudaDeviceReset (or any other re-creation of the device's primary context)
+ * invalidates it: do not call this entry point after one.  All calls share
+ * the one array and it keeps the last call's contents; nothing in it needs to
+ * start at zero.  Two calls whose kernels
  * overlap on the GPU (different streams without ordering between them) race
  * on the array and produce undefined masks: order them on one stream.
  */
@@ -307,11 +310,12 @@ dbst_status dbst_build_sip_mask_raster(const void* q, const void* k, const dbst_
  *   o[n]   = sum_{m in tokens(S_i)} softmax_m(scale <q_n, k_m> + off[i, block(m)]) v[m]
  *   lse[n] = log sum_{m in tokens(S_i)} exp(scale <q_n, k_m> + off[i, block(m)])
  * offsets is [B,H,NB,NB] float32 (natural log; read only at kept blocks) or
- * NULL for none.  The kernel walks the kept blocks twice (row statistics, then
- * normalised P times V), so it forms S three times per two products of
- * dbst_block_sparse_attn.  An empty row gives o = 0, lse = -inf.  Other
- * arguments as for dbst_block_sparse_attn (the _raster form: raster q, k, v, o,
- * lse); lse may be NULL.
+ * NULL for none.  Runs the kernel of dbst_block_sparse_attn (query blocks
+ * paired one tile step apart) with the offset added to the logits before the
+ * row max and the exponent, so it costs what the plain forward costs.  An
+ * empty row gives o = 0, lse = -inf.  Other arguments as for
+ * dbst_block_sparse_attn (the _raster form: raster q, k, v, o, lse); lse may
+ * be NULL.
  */
 dbst_status dbst_block_sparse_attn_offsets(const void* q, const void* k, const void* v, const dbst_geom* g,
                                            const int32_t* kv_count, const int16_t* kv_idx, const float* offsets,
@@ -350,8 +354,8 @@ dbst_status dbst_build_fine_mask_raster(const void* q, const void* k, const dbst
  * Attention over the kept 4-token groups: for query block i, the keys are the
  * tokens of the groups that group_mask[b,h,i,:] keeps in the blocks listed by
  * (kv_count, kv_idx); exact softmax over those tokens, o bf16, lse float32
- * (NULL allowed).  Runs the two-sweep kernel of dbst_block_sparse_attn_offsets
- * over the listed blocks with the other groups' columns masked, so it costs
+ * (NULL allowed).  Runs a two-sweep kernel (row statistics, then normalised P
+ * times V) over the listed blocks with the other groups' columns masked, so it costs
  * whole blocks; gathering the kept groups into full tiles is not done here.
  * group_mask must be 2-byte aligned and is required.  The _raster form takes
  * raster q, k, v, o, lse.

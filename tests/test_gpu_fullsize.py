@@ -139,7 +139,8 @@ def test_hunyuan_like_full_size(built):
     assert 0.03 < kept < 0.15
 
 
-@pytest.mark.parametrize("p", [0.5, 0.9, 1.0])
+# every p of the sparsity sweep
+@pytest.mark.parametrize("p", S.workload("sweep").p_list)
 def test_sweep_full_size(built, p):
     kept, excused = check_full("sweep", p, per_head=8)
     if p >= 1.0:

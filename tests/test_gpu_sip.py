@@ -8,7 +8,7 @@ disagreement is excused only where the uniform lies within 1e-9 of the
 oracle's pi (the two sides sum the pooled map in different orders, so pi agrees
 to about 1e-15).  Offsets log(1/pi) agree to float32 rounding.
 
-Attention with offsets: the two-sweep kernel against ``oracle.sip_attention``
+Attention with offsets: the forward kernel, offsets in its exponent, against ``oracle.sip_attention``
 on the oracle's own kept set and pi, with the forward's bounds (max-abs 2e-2,
 relative L2 5e-3 on o, 2e-3 on lse); without offsets it must match the plain
 masked attention oracle to the same bounds.
@@ -120,7 +120,7 @@ def run_offset_attn(w, q, k, v, keep, off, raster=False):
 
 
 @pytest.mark.parametrize("name,D", [("tiny", 64), ("small", 64), ("small", 128)])
-def test_offset_free_two_sweep_attention_matches_masked_attention(built, name, D):
+def test_offset_free_attention_matches_masked_attention(built, name, D):
     w = dataclasses.replace(S.workload(name), D=D)
     og = P.geometry(w)
     q, k, v = S.make_qkv(w)
