@@ -144,7 +144,7 @@ MaskWorkspace mask_workspace(const dbst_geom* g) {
 }
 
 // Tensor-core mask build (rows of at most kMaskTcMaxNB blocks): pool counters, pieces, residuals, norms.
-constexpr int kMaskTcMaxNB = 1024;
+constexpr int kMaskTcMaxNB = 2048;
 struct MaskTcWorkspace {
   size_t kmax, pieces, resid, norm, s, refine, total;
 };
@@ -618,7 +618,8 @@ bool launch_select_rows_npt(const dbst::SelRowsParams& prm, cudaStream_t s) {
   if (NB <= 256) return launch_select_rows<D, 8>(prm, s);
   if (NB <= 512) return launch_select_rows<D, 16>(prm, s);
   if (NB <= 640) return launch_select_rows<D, 20>(prm, s);
-  return launch_select_rows<D, 32>(prm, s);
+  if (NB <= 1024) return launch_select_rows<D, 32>(prm, s);
+  return launch_select_rows<D, 64>(prm, s);
 }
 
 // Tensor-core mask build (NB <= kMaskTcMaxNB): the pool (HBM-bound), then the selection (persistent:
@@ -661,7 +662,8 @@ dbst_status build_mask_tc(const void* q, const void* k, const dbst_geom* g, floa
   lp.BH = BH;
   lp.NB = NB;
   lp.ntiles = (NB + 127) / 128;
-  lp.R = lp.ntiles <= 3 ? 64 : lp.ntiles <= 5 ? 48 : 32;
+  // rows per item: the two accumulators of every key tile, 2 * ntiles * R columns, fit TMEM's 512
+  lp.R = lp.ntiles <= 3 ? 64 : lp.ntiles <= 5 ? 48 : lp.ntiles <= 8 ? 32 : 16;
   lp.chunks = (NB + lp.R - 1) / lp.R;
   const double scale = 1.0 / std::sqrt(static_cast<double>(D));
   lp.scale_f = static_cast<float>(scale);

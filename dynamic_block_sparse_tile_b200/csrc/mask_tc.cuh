@@ -570,7 +570,7 @@ __global__ void __launch_bounds__(kLogTcThreads, 1)
 // Bits, list and count of one row from this lane's keep flags (bit u: block lane + 32u), with the
 // sliding-tile neighbourhood added.
 template <int NPT>
-__device__ __forceinline__ void emit_row(const SelRowsParams& prm, long long row, int i, uint32_t keepm) {
+__device__ __forceinline__ void emit_row(const SelRowsParams& prm, long long row, int i, unsigned long long keepm) {
   const int lane = threadIdx.x & 31;
   const int NB = prm.NB, NW = prm.NW;
   const int qx_ = i % prm.nX, qy_ = (i / prm.nX) % prm.nY, qt_ = i / (prm.nX * prm.nY);
@@ -582,7 +582,7 @@ __device__ __forceinline__ void emit_row(const SelRowsParams& prm, long long row
     const int j = lane + 32 * u;
     bool keep = false;
     if (j < NB) {
-      keep = (keepm >> u) & 1u;
+      keep = (keepm >> u) & 1ull;
       if (prm.sta_radius >= 0) {
         const int kx = j % prm.nX, ky = (j / prm.nX) % prm.nY, kt = j / (prm.nX * prm.nY);
         const int dmax = max(abs(kt - qt_), max(abs(ky - qy_), abs(kx - qx_)));
@@ -597,9 +597,14 @@ __device__ __forceinline__ void emit_row(const SelRowsParams& prm, long long row
   if (lane == 0) prm.count[row] = base;
 }
 
-// A row's fast logits (-inf past NB), max and min, masses e^(s - max) as integers in units of 2^-21
-// of the row's largest (a row of at most 1024 blocks sums below 2^31, so every sum is exact in 32 bits
-// and independent of its order), and the cumulative mass to reach: p of the total, rounded up.
+// Units of the integer masses: 2^21 per the row's largest for rows of at most 1024 blocks, 2^20 for
+// rows of at most 2048, so that a row's total stays below 2^32.
+template <int NPT>
+__device__ __forceinline__ constexpr float mass_unit() { return NPT > 32 ? 1048576.0f : 2097152.0f; }
+
+// A row's fast logits (-inf past NB), max and min, masses e^(s - max) as integers in mass_unit<NPT>()
+// of the row's largest (a row sums to at most 2^31, so every sum is exact in 32 bits and independent
+// of its order), and the cumulative mass to reach: p of the total, rounded up.
 template <int NPT>
 __device__ __forceinline__ void load_row(const SelRowsParams& prm, const float* srow, float (&s)[NPT],
                                          uint32_t (&mass)[NPT], float& mx, float& mn, unsigned long long& target) {
@@ -618,7 +623,7 @@ __device__ __forceinline__ void load_row(const SelRowsParams& prm, const float* 
   uint32_t lsum = 0u;
 #pragma unroll
   for (int u = 0; u < NPT; ++u) {
-    mass[u] = (s[u] != -INFINITY) ? __float2uint_rn(fast_exp2((s[u] - mx) * 1.4426950408889634f) * 2097152.0f) : 0u;
+    mass[u] = (s[u] != -INFINITY) ? __float2uint_rn(fast_exp2((s[u] - mx) * 1.4426950408889634f) * mass_unit<NPT>()) : 0u;
     lsum += mass[u];
   }
   const uint32_t total = __reduce_add_sync(0xffffffffu, lsum);
@@ -640,7 +645,7 @@ __device__ __forceinline__ float logit_error_bound(const SelRowsParams& prm, lon
 template <int D, int NPT>
 __device__ __forceinline__ bool band_in_warp(const SelRowsParams& prm, long long row, long long bh,
                                              const float (&s)[NPT], const uint32_t (&mass)[NPT], float sb, float E,
-                                             unsigned long long target, uint32_t* gather, uint32_t& keepm) {
+                                             unsigned long long target, uint32_t* gather, unsigned long long& keepm) {
   const int lane = threadIdx.x & 31;
   const int NB = prm.NB;
   const float W = 4.0f * E;
@@ -726,7 +731,7 @@ __device__ __forceinline__ bool band_in_warp(const SelRowsParams& prm, long long
   xc = warp_max_f32(xc);
   if (!(fabsf(xc - sb) <= 0.5f * W)) return false;
   // keep: above the band, or in the band at or before the crossing in the exact order
-  keepm = 0u;
+  keepm = 0ull;
   int base = 0;
 #pragma unroll
   for (int u = 0; u < NPT; ++u) {
@@ -736,14 +741,14 @@ __device__ __forceinline__ bool band_in_warp(const SelRowsParams& prm, long long
     const unsigned long long km = __shfl_sync(0xffffffffu, k0, (base + __popc(bal & lt)) & 31);
     base += __popc(bal);
     const bool keep = mem ? (km >= thr) : (valid && s[u] > sb);
-    keepm |= (keep ? 1u : 0u) << u;
+    keepm |= (keep ? 1ull : 0ull) << u;
   }
   return true;
 }
 
 // At least four blocks (16 warps) per SM: the rows are latency-bound, so rows in flight matter.
 template <int D, int NPT>
-__global__ void __launch_bounds__(32 * kSelRowsWarps, 4) select_rows_kernel(const SelRowsParams prm) {
+__global__ void __launch_bounds__(32 * kSelRowsWarps, NPT > 32 ? 2 : 4) select_rows_kernel(const SelRowsParams prm) {
   const int lane = threadIdx.x & 31, wk = threadIdx.x >> 5;
   const long long rows = prm.BH * prm.NB;
   const long long row = static_cast<long long>(blockIdx.x) * kSelRowsWarps + wk;
@@ -758,7 +763,7 @@ __global__ void __launch_bounds__(32 * kSelRowsWarps, 4) select_rows_kernel(cons
   unsigned long long target;
   load_row<NPT>(prm, srow, s, mass, mx, mn, target);
   if (!(prm.p < 1.0)) {                          // p = 1 keeps every block
-    emit_row<NPT>(prm, row, i, 0xFFFFFFFFu);
+    emit_row<NPT>(prm, row, i, ~0ull);
     return;
   }
   // mass of the blocks whose fast logit is at least t
@@ -798,16 +803,16 @@ __global__ void __launch_bounds__(32 * kSelRowsWarps, 4) select_rows_kernel(cons
     }
     return;
   }
-  uint32_t keepm = 0u;
+  unsigned long long keepm = 0ull;
 #pragma unroll
-  for (int u = 0; u < NPT; ++u) keepm |= (s[u] >= sb ? 1u : 0u) << u;
+  for (int u = 0; u < NPT; ++u) keepm |= (s[u] >= sb ? 1ull : 0ull) << u;
   emit_row<NPT>(prm, row, i, keepm);
 }
 
 // The listed rows whose band fits a warp (band_in_warp); the others are flagged in the list (bit 31
 // of the row) for refine_wide_kernel.  Persistent: warps walk the list.
 template <int D, int NPT>
-__global__ void __launch_bounds__(32 * kSelRowsWarps, 4) refine_rows_kernel(const SelRowsParams prm) {
+__global__ void __launch_bounds__(32 * kSelRowsWarps, NPT > 32 ? 2 : 4) refine_rows_kernel(const SelRowsParams prm) {
   __shared__ uint32_t s_gather[kSelRowsWarps][64];
   const int lane = threadIdx.x & 31, wk = threadIdx.x >> 5;
   const int NB = prm.NB;
@@ -824,7 +829,7 @@ __global__ void __launch_bounds__(32 * kSelRowsWarps, 4) refine_rows_kernel(cons
     float mx, mn;
     unsigned long long target;
     load_row<NPT>(prm, prm.S + row * NB, s, mass, mx, mn, target);
-    uint32_t km;
+    unsigned long long km;
     if (band_in_warp<D, NPT>(prm, row, bh, s, mass, sb, logit_error_bound(prm, row, bh), target, s_gather[wk], km))
       emit_row<NPT>(prm, row, i, km);
     else if (lane == 0)
@@ -940,9 +945,9 @@ __global__ void __launch_bounds__(32 * kSelRowsWarps) refine_wide_kernel(const S
       const int j2 = 0xFFFF - static_cast<int>(thr & 0xFFFFull);
       if (fabsf(__ldg(srow + j2) - sb) <= 0.5f * W) break;   // the boundary stayed inside the band
     }
-    uint32_t keepm = 0u;
+    unsigned long long keepm = 0ull;
 #pragma unroll
-    for (int u = 0; u < NPT; ++u) keepm |= (key[u] != 0ull && key[u] >= thr ? 1u : 0u) << u;
+    for (int u = 0; u < NPT; ++u) keepm |= (key[u] != 0ull && key[u] >= thr ? 1ull : 0ull) << u;
     emit_row<NPT>(prm, row, i, keepm);
   }
 }

@@ -80,7 +80,7 @@ size_t dbst_mask_workspace_bytes(const dbst_geom* g);
  * "Intégration Hybride avec STA").
  *   1. Qp, Kp = mean of each block's 64 tiled tokens (float64, exact).
  *   2. A[i,:] = softmax_j(<Qp_i, Kp_j> / sqrt(D)) per (b, h).  Rows of at most
- *      1024 blocks take the logits from the tensor cores (three bf16 pieces of
+ *      2048 blocks take the logits from the tensor cores (three bf16 pieces of
  *      each mean) and recompute in float64 every key whose logit lies within
  *      the error bound of the selection boundary's, so the order matches the
  *      float64 one; longer rows use float64 logits throughout.

@@ -118,7 +118,7 @@ def test_workspace_size_formula(lib):
 
     def up(x):
         return (x + 255) // 256 * 256
-    # float64 layout (SIP mask, rows of more than 1024 blocks): block means of q and k, pooled logits
+    # float64 layout (SIP mask, rows of more than 2048 blocks): block means of q and k, pooled logits
     f64 = 2 * up(bh * nb * 64 * 8) + up(bh * nb * nb * 8)
     # tensor-core layout: per-head max key norm and the refine-list length, 6 bf16 pieces and 2 float32
     # residuals of the means, 2 norms per block, the float32 pooled logits, the refine list

@@ -92,6 +92,22 @@ def test_mask_matches_oracle(built, name, p, sta):
         assert got.all()
 
 
+# Rows of more than 1024 blocks (the HunyuanVideo-like shape has 2040): the tensor-core path's longest
+# rows, with integer masses in coarser units; the whole mask against the oracle.
+@pytest.mark.parametrize("grid,p,sta", [((17, 64, 64), 0.9, -1), ((32, 64, 64), 0.8, 1)])
+def test_mask_long_rows_match_oracle(built, grid, p, sta):
+    w = dataclasses.replace(S.workload("small"), H=2, grid=grid, tile=(1, 8, 8))
+    g = P.geometry(w)
+    assert 1024 < g.NB <= 2048
+    q, k, _ = S.make_qkv(w)
+    qt, kt = O.tile_reorder(q, g), O.tile_reorder(k, g)
+    ref, A = P.oracle_mask_per_head(qt, kt, g, p, sta)
+    got, cnt, idx = gpu_mask(w, qt, kt, p, sta)
+    hard, excused = P.mask_mismatches(got, ref, A, p, O.sta_mask(g, sta))
+    assert not hard, f"{len(hard)} non-excused mask disagreements, first {hard[:5]}"
+    assert P.lists_match_bits(cnt, idx, got)
+
+
 # ---------------------------------------------------------------- attention
 def gpu_attention_from_mask(w, qt, kt, vt, mask, scale=0.0):
     g = gpu_geom(w, heads=qt.shape[1])
