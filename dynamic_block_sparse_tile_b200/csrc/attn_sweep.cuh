@@ -135,8 +135,7 @@ enum {
   BB_REMPTY = BB_RFULL + kSweepSlots,      // [kSweepSlots] ring slot's last reader (the TS products) done
   BB_SFULL = BB_REMPTY + kSweepSlots,      // [2] A and A2 of tile t in buffer t&1 complete
   BB_PFULL = BB_SFULL + 2,               // [2] 256 arrivals: P / dS of tile t written
-  BB_ACC = BB_PFULL + 2,                 // [2] TS products of tile t complete (buffer t&1 free)
-  BB_DRAIN = BB_ACC + 2,
+  BB_DRAIN = BB_PFULL + 2,
   BB_COUNT = BB_DRAIN + 1
 };
 static_assert(BB_COUNT * 8 <= 256, "barrier area");
@@ -499,7 +498,6 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
           }
         }
       }
-      umma_commit_elect(bar(BB_ACC + b));
       umma_commit_elect(bar(BB_REMPTY + s));
       return true;
     };
@@ -509,11 +507,10 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
     for (int u = 0; ok && u < NV; ++u) {
       if (__any_sync(0xffffffffu, *s_abort != 0)) { ok = false; break; }
       if (!issue_ts(u)) { ok = false; break; }
-      // buffer u&1 is rewritten by the products of tile u+2 only once the TS products of tile u,
-      // which read P and dS from it, have completed
-      if (u + 2 < NV) {
-        if (!wait_all(BB_ACC + (u & 1), (u >> 1) & 1) || !issue_ss(u + 2)) { ok = false; break; }
-      }
+      // The products of tile u+2 rewrite buffer u&1, which the TS products of tile u read (P and dS):
+      // tcgen05.mma operations issued by one thread execute in issue order, so they are queued right
+      // behind them, with no wait for their completion.
+      if (u + 2 < NV && !issue_ss(u + 2)) { ok = false; break; }
     }
     if (!ok && lane == 0) *s_abort = 1;
     umma_commit_elect(bar(BB_DRAIN));

@@ -103,25 +103,75 @@ __global__ void __launch_bounds__(kPairingThreads) pair_blocks_kernel(const uint
     __syncthreads();
   }
 
-  for (int v = tid; v < NB; v += kPairingThreads) {
+  // Rows in shared memory: one thread per block.  Rows in global memory (a head too large to stage):
+  // one warp per block, the lanes holding the row's words w = lane + 32 i (NW <= 128), so that every
+  // read of a row is one coalesced pass.  First the kept counts and each neighbour's union count,
+  // then the weights.
+  const int warp = tid >> 5, lane = tid & 31;
+  constexpr int kWarps = kPairingThreads / 32;
+  if constexpr (STAGE) {
+    for (int v = tid; v < NB; v += kPairingThreads) {
+      int c = 0;
+      for (int w = 0; w < g.NW; ++w) c += __popc(head[static_cast<long long>(v) * g.NW + w]);
+      count[v] = c;
+      partner[v] = -1;
+    }
+    __syncthreads();
+    for (int v = tid; v < NB; v += kPairingThreads) {
+      const uint32_t* a = head + static_cast<long long>(v) * g.NW;
+      for (int k = 0; k < 6; ++k) {
+        const int u = pairing_neighbour(v, k, g);
+        int un = -1;
+        if (u >= 0) {
+          const uint32_t* b = head + static_cast<long long>(u) * g.NW;
+          un = 0;
+          for (int w = 0; w < g.NW; ++w) un += __popc(a[w] | b[w]);
+        }
+        weight[v * 6 + k] = un;   // union count for now; -1: no neighbour
+      }
+    }
+  } else for (int v = warp; v < NB; v += kWarps) {
+    const uint32_t* a = head + static_cast<long long>(v) * g.NW;
+    uint32_t aw[4];
     int c = 0;
-    for (int w = 0; w < g.NW; ++w) c += __popc(head[static_cast<long long>(v) * g.NW + w]);
-    count[v] = c;
-    partner[v] = -1;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int w = lane + 32 * i;
+      aw[i] = w < g.NW ? a[w] : 0u;
+      c += __popc(aw[i]);
+    }
+    c = __reduce_add_sync(0xffffffffu, c);
+    int un[6];
+#pragma unroll
+    for (int k = 0; k < 6; ++k) {
+      const int u = pairing_neighbour(v, k, g);
+      int x = 0;
+      if (u >= 0) {
+        const uint32_t* b = head + static_cast<long long>(u) * g.NW;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int w = lane + 32 * i;
+          x += __popc(aw[i] | (w < g.NW ? b[w] : 0u));
+        }
+      }
+      un[k] = u >= 0 ? x : -1;
+    }
+#pragma unroll
+    for (int k = 0; k < 6; ++k) {
+      const int x = un[k] >= 0 ? __reduce_add_sync(0xffffffffu, un[k]) : -1;
+      if (lane == 0) weight[v * 6 + k] = x;   // union count for now; -1: no neighbour
+    }
+    if (lane == 0) {
+      count[v] = c;
+      partner[v] = -1;
+    }
   }
   __syncthreads();
   for (int v = tid; v < NB; v += kPairingThreads) {
-    const uint32_t* a = head + static_cast<long long>(v) * g.NW;
     for (int k = 0; k < 6; ++k) {
       const int u = pairing_neighbour(v, k, g);
-      int wt = -1;
-      if (u >= 0) {
-        const uint32_t* b = head + static_cast<long long>(u) * g.NW;
-        int un = 0;
-        for (int w = 0; w < g.NW; ++w) un += __popc(a[w] | b[w]);
-        wt = (count[v] + 1) / 2 + (count[u] + 1) / 2 - (un + 1) / 2;
-      }
-      weight[v * 6 + k] = wt;
+      const int x = weight[v * 6 + k];
+      weight[v * 6 + k] = u >= 0 ? (count[v] + 1) / 2 + (count[u] + 1) / 2 - (x + 1) / 2 : -1;
     }
   }
   __syncthreads();
@@ -201,19 +251,30 @@ __global__ void __launch_bounds__(kPairingThreads) pair_blocks_kernel(const uint
   const int npairs = (NB + 1) / 2;
   int* ent = weight;              // the edge weights are no longer needed: 6 NB >= 2 npairs ints
   int* cost = weight + npairs;
-  for (int e = tid; e < npairs; e += kPairingThreads) {
+  for (int e = STAGE ? tid : warp; e < npairs; e += STAGE ? kPairingThreads : kWarps) {
     const int32_t x = out[e];
     const int a = x & 0xFFFF, b = (x >> 16) & 0xFFFF;
     int un = 0;
-    const uint32_t* ra = head + static_cast<long long>(a) * g.NW;
     if (b == 0xFFFF) {
       un = count[a];
-    } else {
+    } else if (STAGE) {
+      const uint32_t* ra = head + static_cast<long long>(a) * g.NW;
       const uint32_t* rb = head + static_cast<long long>(b) * g.NW;
       for (int w = 0; w < g.NW; ++w) un += __popc(ra[w] | rb[w]);
+    } else {   // one warp per pair, coalesced rows
+      const uint32_t* ra = head + static_cast<long long>(a) * g.NW;
+      const uint32_t* rb = head + static_cast<long long>(b) * g.NW;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int w = lane + 32 * i;
+        un += w < g.NW ? __popc(ra[w] | rb[w]) : 0;
+      }
+      un = __reduce_add_sync(0xffffffffu, un);
     }
-    ent[e] = x;
-    cost[e] = (un + 1) / 2;
+    if (STAGE || lane == 0) {
+      ent[e] = x;
+      cost[e] = (un + 1) / 2;
+    }
   }
   __syncthreads();
   for (int e = tid; e < npairs; e += kPairingThreads) {
