@@ -386,8 +386,10 @@ def measure_sip(args, w, p, qkv=None) -> dict:
     lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device="cuda")
     sel_ms = timed_median(lambda: dbst.build_sip_mask(q, k, g, budget, u, raster=True, workspace=ws, out=sip),
                           args.steps, args.warmup)
+    sip_pairs = dbst.pair_query_blocks(sip[0], g)
     attn_ms = timed_median(lambda: dbst.block_sparse_attn_offsets(q, k, v, g, sip[1], sip[2], sip[3], raster=True,
-                                                                  out=o, lse=lse), args.steps, args.warmup)
+                                                                  out=o, lse=lse, pairs=sip_pairs),
+                           args.steps, args.warmup)
     plain_ms = timed_median(lambda: dbst.block_sparse_attn_offsets(q, k, v, g, cnt, idx, None, raster=True, out=o,
                                                                    lse=lse), args.steps, args.warmup)
     pairs = dbst.pair_query_blocks(bits, g)
@@ -405,8 +407,8 @@ def measure_sip(args, w, p, qkv=None) -> dict:
             "forward_on_nabla_mask_ms": fwd_ms,
             "sip_attn_over_forward": attn_ms / fwd_ms,
             "note": "TFLOP/s count the 2 products of attention per kept block pair; the offsets ride in the "
-                    "forward kernel's exponent (query blocks paired one tile step apart; the forward here uses "
-                    "the pair list of dbst_pair_query_blocks)"}
+                    "forward kernel's exponent; SIP attention and the forward run on the pair lists of "
+                    "dbst_pair_query_blocks for their masks, the offset kernel on the NABLA mask without one"}
 
 
 def run_sip(args, w, p):

@@ -38,7 +38,8 @@ EXPORTS = ("dbst_status_string", "dbst_tile_reorder", "dbst_tile_unreorder", "db
            "dbst_build_sip_mask", "dbst_build_sip_mask_raster", "dbst_block_sparse_attn_offsets",
            "dbst_block_sparse_attn_offsets_raster", "dbst_fine_mask_workspace_bytes", "dbst_build_fine_mask",
            "dbst_build_fine_mask_raster", "dbst_block_sparse_attn_groups", "dbst_block_sparse_attn_groups_raster",
-           "dbst_block_sparse_attn_gather", "dbst_block_sparse_attn_gather_raster", "dbst_set_wait_limit")
+           "dbst_block_sparse_attn_gather", "dbst_block_sparse_attn_gather_raster", "dbst_set_wait_limit",
+           "dbst_block_sparse_attn_offsets_paired", "dbst_block_sparse_attn_offsets_paired_raster")
 
 DBST_OK, DBST_EINVAL, DBST_ECUDA, DBST_ETIMEOUT, DBST_EBOUNDS, DBST_ETOOLARGE = 0, 1, 2, 3, 4, 5
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -121,6 +122,9 @@ def load() -> ctypes.CDLL:
         getattr(lib, name).restype = i32
     for name in ("dbst_block_sparse_attn_offsets", "dbst_block_sparse_attn_offsets_raster"):
         getattr(lib, name).argtypes = [vp, vp, vp, gp, vp, vp, vp, f32, vp, vp, vp]
+        getattr(lib, name).restype = i32
+    for name in ("dbst_block_sparse_attn_offsets_paired", "dbst_block_sparse_attn_offsets_paired_raster"):
+        getattr(lib, name).argtypes = [vp, vp, vp, gp, vp, vp, vp, vp, f32, vp, vp, vp]
         getattr(lib, name).restype = i32
     lib.dbst_fine_mask_workspace_bytes.argtypes = [gp]
     lib.dbst_fine_mask_workspace_bytes.restype = ctypes.c_size_t
@@ -399,9 +403,11 @@ def build_sip_mask(q, k, g: Geom, budget: float, uniforms: torch.Tensor, raster:
 
 def block_sparse_attn_offsets(q, k, v, g: Geom, kv_count, kv_idx, offsets: Optional[torch.Tensor] = None,
                               scale: float = 0.0, raster: bool = False, want_lse: bool = True,
-                              out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None):
+                              out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                              pairs: Optional[torch.Tensor] = None):
     """Attention over kept blocks with a logit offset per (query block, key block)
-    (``dbst_block_sparse_attn_offsets[_raster]``) -> (o, lse or None)."""
+    (``dbst_block_sparse_attn_offsets[_raster]``, or ``..._offsets_paired[_raster]`` on the schedule
+    ``pairs`` of :func:`pair_query_blocks`) -> (o, lse or None)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, torch.bfloat16, _qkv_shape(g), n)
     _need(kv_count, torch.int32, (g.B, g.H, g.NB), "kv_count")
@@ -411,6 +417,13 @@ def block_sparse_attn_offsets(q, k, v, g: Geom, kv_count, kv_idx, offsets: Optio
     o = torch.empty_like(q) if out is None else out
     if want_lse and lse is None:
         lse = torch.empty((g.B, g.H, g.N), dtype=torch.float32, device=q.device)
+    if pairs is not None:
+        _need(pairs, torch.int32, (g.B, g.H, (g.NB + 1) // 2), "pairs")
+        fn = "dbst_block_sparse_attn_offsets_paired_raster" if raster else "dbst_block_sparse_attn_offsets_paired"
+        _check(getattr(load(), fn)(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(g), _ptr(kv_count), _ptr(kv_idx),
+                                   _ptr(offsets), _ptr(pairs), float(scale), _ptr(o),
+                                   _ptr(lse if want_lse else None), _stream()), fn)
+        return o, (lse if want_lse else None)
     fn = "dbst_block_sparse_attn_offsets_raster" if raster else "dbst_block_sparse_attn_offsets"
     _check(getattr(load(), fn)(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(g), _ptr(kv_count), _ptr(kv_idx),
                                _ptr(offsets), float(scale), _ptr(o), _ptr(lse if want_lse else None), _stream()), fn)

@@ -520,7 +520,7 @@ dbst_status gather_common(const void* q, const void* k, const void* v, const dbs
 
 dbst_status offset_attn_common(const void* q, const void* k, const void* v, const dbst_geom* g, const int32_t* cnt,
                                const int16_t* idx, const float* offsets, const uint16_t* gmask, float scale, void* o,
-                               float* lse, void* stream, bool raster) {
+                               float* lse, void* stream, bool raster, const int32_t* pairs = nullptr) {
   if (!geom_ok(g) || !q || !k || !v || !o || !cnt || !idx) return DBST_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(cnt) || !aligned16(idx))
     return DBST_EINVAL;
@@ -528,13 +528,14 @@ dbst_status offset_attn_common(const void* q, const void* k, const void* v, cons
       (gmask && (reinterpret_cast<uintptr_t>(gmask) & 1u)))
     return DBST_EINVAL;
   if (!std::isfinite(scale)) return DBST_EINVAL;
+  if (pairs && (reinterpret_cast<uintptr_t>(pairs) & 3u)) return DBST_EINVAL;
   auto s = static_cast<cudaStream_t>(stream);
   if (gmask == nullptr) {   // offsets only: the forward kernel, with the offsets in its exponent
     if (raster)
-      return g->D == 128 ? launch_pair<128, true>(q, k, v, g, cnt, idx, nullptr, scale, o, lse, s, offsets)
-                         : launch_pair<64, true>(q, k, v, g, cnt, idx, nullptr, scale, o, lse, s, offsets);
-    return g->D == 128 ? launch_pair<128, false>(q, k, v, g, cnt, idx, nullptr, scale, o, lse, s, offsets)
-                       : launch_pair<64, false>(q, k, v, g, cnt, idx, nullptr, scale, o, lse, s, offsets);
+      return g->D == 128 ? launch_pair<128, true>(q, k, v, g, cnt, idx, pairs, scale, o, lse, s, offsets)
+                         : launch_pair<64, true>(q, k, v, g, cnt, idx, pairs, scale, o, lse, s, offsets);
+    return g->D == 128 ? launch_pair<128, false>(q, k, v, g, cnt, idx, pairs, scale, o, lse, s, offsets)
+                       : launch_pair<64, false>(q, k, v, g, cnt, idx, pairs, scale, o, lse, s, offsets);
   }
   if (raster)
     return g->D == 128 ? launch_offset_attn<128, true>(q, k, v, g, cnt, idx, offsets, gmask, scale, o, lse, s)
@@ -1067,6 +1068,23 @@ dbst_status dbst_block_sparse_attn_offsets_raster(const void* q, const void* k, 
                                                   const float* offsets, float scale, void* o, float* lse,
                                                   void* stream) {
   return offset_attn_common(q, k, v, g, kv_count, kv_idx, offsets, nullptr, scale, o, lse, stream, true);
+}
+
+dbst_status dbst_block_sparse_attn_offsets_paired(const void* q, const void* k, const void* v, const dbst_geom* g,
+                                                  const int32_t* kv_count, const int16_t* kv_idx,
+                                                  const float* offsets, const int32_t* pairs, float scale, void* o,
+                                                  float* lse, void* stream) {
+  if (!pairs) return DBST_EINVAL;
+  return offset_attn_common(q, k, v, g, kv_count, kv_idx, offsets, nullptr, scale, o, lse, stream, false, pairs);
+}
+
+dbst_status dbst_block_sparse_attn_offsets_paired_raster(const void* q, const void* k, const void* v,
+                                                         const dbst_geom* g, const int32_t* kv_count,
+                                                         const int16_t* kv_idx, const float* offsets,
+                                                         const int32_t* pairs, float scale, void* o, float* lse,
+                                                         void* stream) {
+  if (!pairs) return DBST_EINVAL;
+  return offset_attn_common(q, k, v, g, kv_count, kv_idx, offsets, nullptr, scale, o, lse, stream, true, pairs);
 }
 
 size_t dbst_squad_workspace_bytes(int B, int H, int N, int D, int w) {

@@ -324,6 +324,18 @@ dbst_status dbst_block_sparse_attn_offsets_raster(const void* q, const void* k, 
                                                   const int32_t* kv_count, const int16_t* kv_idx,
                                                   const float* offsets, float scale, void* o, float* lse,
                                                   void* stream);
+/* The same on the query-block schedule `pairs` written by dbst_pair_query_blocks
+ * for this mask's bits (required, 4-byte aligned; any order of a head's
+ * entries gives the same results, as for dbst_block_sparse_attn_raster). */
+dbst_status dbst_block_sparse_attn_offsets_paired(const void* q, const void* k, const void* v, const dbst_geom* g,
+                                                  const int32_t* kv_count, const int16_t* kv_idx,
+                                                  const float* offsets, const int32_t* pairs, float scale, void* o,
+                                                  float* lse, void* stream);
+dbst_status dbst_block_sparse_attn_offsets_paired_raster(const void* q, const void* k, const void* v,
+                                                         const dbst_geom* g, const int32_t* kv_count,
+                                                         const int16_t* kv_idx, const float* offsets,
+                                                         const int32_t* pairs, float scale, void* o, float* lse,
+                                                         void* stream);
 
 /*
  * Fine-grained mask with key groups of 4 tokens (AB-Attention page, section

@@ -149,6 +149,15 @@ def test_sip_attention_matches_oracle(built, name, budget, D):
     ro, rlse = run_offset_attn(w, q, k, v, keep, off, raster=True)
     assert torch.equal(ro.view(torch.int16), o.view(torch.int16).cpu())
     np.testing.assert_array_equal(rlse.numpy(), lse.cpu().numpy())
+    # on the pair schedule of the sampled mask: the same bounds
+    g = gpu_geom(w)
+    bits = torch.from_numpy(P.pack_mask(keep).view(np.int32)).cuda()
+    cnt, idx = dbst.mask_from_bits(bits, g)
+    pairs = dbst.pair_query_blocks(bits, g)
+    po, plse = dbst.block_sparse_attn_offsets(*(P.bits_to_torch(a) for a in (qt, kt, vt)), g, cnt, idx,
+                                              torch.from_numpy(off.astype(np.float32)).cuda(), pairs=pairs)
+    dbst.get_error()
+    check_attention(f"{name} K={budget} D={D} paired", po, plse, ref_o, ref_lse)
 
 
 def test_offset_attention_empty_head_and_repeat(built):
