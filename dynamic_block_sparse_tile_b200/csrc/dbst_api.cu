@@ -736,18 +736,8 @@ dbst_status build_mask(const void* q_tiled, const void* k_tiled, const dbst_geom
     sg.nY = g->Y / g->ty;
     sg.sta_radius = sta_radius;
     sg.p = static_cast<double>(p);
-    const long long rows = nblk;
-    bool ok = true;
-    const unsigned wgrid = static_cast<unsigned>((rows * 32 + 127) / 128);   // one warp per row
-    if (NB <= 256) dbst::select_warp_kernel<8><<<wgrid, 128, 0, s>>>(S, sg, rows, mask_bits, kv_count, kv_idx);
-    else if (NB <= 384) dbst::select_warp_kernel<12><<<wgrid, 128, 0, s>>>(S, sg, rows, mask_bits, kv_count, kv_idx);
-    else if (NB <= 512) dbst::select_warp_kernel<16><<<wgrid, 128, 0, s>>>(S, sg, rows, mask_bits, kv_count, kv_idx);
-    else if (NB <= 640) dbst::select_warp_kernel<20><<<wgrid, 128, 0, s>>>(S, sg, rows, mask_bits, kv_count, kv_idx);
-    else if (NB <= 768) dbst::select_warp_kernel<24><<<wgrid, 128, 0, s>>>(S, sg, rows, mask_bits, kv_count, kv_idx);
-    else if (NB <= 1024) dbst::select_warp_kernel<32><<<wgrid, 128, 0, s>>>(S, sg, rows, mask_bits, kv_count, kv_idx);
-    else if (NB <= 2048) ok = launch_select<8>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
-    else ok = launch_select<16>(S, sg, rows, mask_bits, kv_count, kv_idx, s);
-    if (!ok) return DBST_ECUDA;
+    // rows of 2049 .. kMaxNB blocks (shorter ones take the tensor-core path): one CTA per row
+    if (!launch_select<16>(S, sg, nblk, mask_bits, kv_count, kv_idx, s)) return DBST_ECUDA;
   }
   return launch_status();
 }

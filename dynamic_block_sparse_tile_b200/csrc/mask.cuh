@@ -4,12 +4,11 @@
 //
 // Precision: the pooled means are exact (64 bf16 values summed in float64) and
 // the pooled logits are float64.  The order of a row's blocks comes from those
-// logits; the masses are float32 exponentials summed in float32 for rows of at
-// most 1024 blocks (one warp per row), float64 exponentials and sums for longer
-// rows.  The kept set agrees with a float64 reference except where a
-// cumulative mass sits within rounding of p.  (Rows of at most 1024 blocks are
-// built by the tensor-core path of mask_tc.cuh; these kernels serve the longer
-// rows and the SIP mask.)
+// logits, with float64 exponentials and sums for the masses; the kept set agrees
+// with a float64 reference except where a cumulative mass sits within rounding
+// of p.  Rows of at most 2048 blocks are built by the tensor-core path of
+// mask_tc.cuh; these kernels serve longer rows, and the pool and logits serve the
+// SIP mask.
 #pragma once
 #include <cstdint>
 #include "ptx.cuh"
@@ -345,19 +344,7 @@ __global__ void __launch_bounds__(256) select_kernel(const double* __restrict__ 
   }
 }
 
-// ---------------------------------------------------------------------------
-// Same selection with one warp per row (rows of at most 32*NPT blocks): the
-// row lives in registers (lane l owns blocks j = l + 32u), and the threshold
-// key is found by a mass quickselect instead of a sort.  Each round picks a
-// live key as pivot and sums, over the warp, the mass of the live keys above
-// it; the answer lies above the pivot, is the pivot, or lies below it, and
-// the pivot always leaves the live set.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ float warp_sum_f32(float v) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-  return v;
-}
+// Warp reductions in float64 (the SIP selection and the tensor-core mask's band refinement).
 __device__ __forceinline__ double warp_sum_f64(double v) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
@@ -367,124 +354,6 @@ __device__ __forceinline__ double warp_max_f64(double v) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, off));
   return v;
-}
-
-// Order-preserving 64-bit key of a row entry: the float64 logit (the softmax
-// keeps its order), top 48 bits, then 0xFFFF - j so that ties go to the lower
-// index.  Logits equal in their top 48 bits (relative difference below
-// 2^-36) count as ties.
-__device__ __forceinline__ unsigned long long logit_key(double s, int j) {
-  unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(s));
-  b = (b >> 63) ? ~b : (b | (1ull << 63));
-  return ((b >> 16) << 16) | static_cast<unsigned long long>(0xFFFF - j);
-}
-
-template <int NPT>
-__global__ void __launch_bounds__(128) select_warp_kernel(const double* __restrict__ S, SelectGeo g, long long rows,
-                                                          uint32_t* __restrict__ bits, int32_t* __restrict__ count,
-                                                          int16_t* __restrict__ idx) {
-  const int lane = threadIdx.x & 31;
-  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (row >= rows) return;                      // whole warps only
-  const int i = static_cast<int>(row % g.NB);
-  const double* srow = S + row * g.NB;
-
-  // keys from the float64 logits; unnormalised masses e^(s - max) and their sums in float32.  A
-  // row of at most 1024 masses, each <= 1, sums with a relative error below 1024 * 2^-24 = 6e-5,
-  // so a kept set can differ from a float64 reference only where the cumulative mass lies that
-  // close to p; the order itself comes from the exact logits.
-  float m[NPT];
-  unsigned long long key[NPT];
-  double mx = -INFINITY;
-#pragma unroll
-  for (int u = 0; u < NPT; ++u) {
-    const int j = lane + 32 * u;
-    const double sj = (j < g.NB) ? srow[j] : -INFINITY;
-    key[u] = (j < g.NB) ? logit_key(sj, j) : 0ull;
-    mx = fmax(mx, sj);
-  }
-  mx = warp_max_f64(mx);
-  float total = 0.0f;
-#pragma unroll
-  for (int u = 0; u < NPT; ++u) {
-    const int j = lane + 32 * u;
-    const double sj = (j < g.NB) ? srow[j] : -INFINITY;
-    m[u] = (j < g.NB) ? fast_exp2(static_cast<float>((sj - mx) * 1.4426950408889634)) : 0.0f;
-    total += m[u];
-  }
-  total = warp_sum_f32(total);
-  const float target = static_cast<float>(g.p * static_cast<double>(total));   // cumulative mass to reach
-
-  unsigned long long thr = 0ull;   // keep key >= thr (0 keeps all)
-  if (g.p < 1.0) {
-    unsigned long long lo = 0ull, hi = ~0ull;   // the answer lies in (lo, hi]
-    unsigned long long cand = 0ull;             // smallest key above hi (see below)
-    float above = 0.0f;                         // mass of keys > hi
-    for (int round = 0; round < 4 * 32 * NPT; ++round) {
-      int mycnt = 0;
-      unsigned long long mine = 0ull;
-#pragma unroll
-      for (int u = 0; u < NPT; ++u) {
-        const bool live = key[u] > lo && key[u] <= hi;
-        mycnt += live;
-        if (live) mine = key[u];
-      }
-      const unsigned holders = __ballot_sync(0xffffffffu, mycnt > 0);
-      if (holders == 0u) {
-        // The float32 sums of different orders left no key between "mass above hi < target" and
-        // "mass above lo >= target": the crossing is, within rounding, the smallest key above hi
-        // (0 keeps every block when hi never moved).
-        thr = cand;
-        break;
-      }
-      const int nh = __popc(holders);
-      const int pick = __fns(holders, 0, 1 + (round * 7) % nh);
-      const unsigned long long pivot = __shfl_sync(0xffffffffu, mine, pick);
-      float gt = 0.0f, eq = 0.0f;
-#pragma unroll
-      for (int u = 0; u < NPT; ++u) {
-        const bool live = key[u] > lo && key[u] <= hi;
-        if (live && key[u] > pivot) gt += m[u];
-        if (key[u] == pivot) eq = m[u];
-      }
-      const float g_above = above + warp_sum_f32(gt);
-      if (g_above >= target) {
-        lo = pivot;                             // the k*-th key is above the pivot
-      } else {
-        const float f = g_above + warp_sum_f32(eq);
-        if (f >= target) {
-          thr = pivot;                          // the pivot is the k*-th key
-          break;
-        }
-        hi = pivot - 1ull;                      // below the pivot; everything >= pivot counts as above
-        cand = pivot;
-        above = f;
-      }
-    }
-  }
-
-  const int qx = i % g.nX, qy = (i / g.nX) % g.nY, qt = i / (g.nX * g.nY);
-  uint32_t* brow = bits + row * g.NW;
-  int16_t* irow = idx + row * g.NB;
-  int base = 0;
-#pragma unroll
-  for (int u = 0; u < NPT; ++u) {
-    const int j = lane + 32 * u;
-    bool keep = false;
-    if (j < g.NB) {
-      keep = key[u] >= thr;
-      if (g.sta_radius >= 0) {
-        const int kx = j % g.nX, ky = (j / g.nX) % g.nY, kt = j / (g.nX * g.nY);
-        const int dmax = max(abs(kt - qt), max(abs(ky - qy), abs(kx - qx)));
-        keep = keep || (dmax <= g.sta_radius);
-      }
-    }
-    const unsigned w = __ballot_sync(0xffffffffu, keep);
-    if (u < g.NW && lane == 0) brow[u] = w;
-    if (keep) irow[base + __popc(w & ((1u << lane) - 1u))] = static_cast<int16_t>(j);
-    base += __popc(w);
-  }
-  if (lane == 0) count[row] = base;
 }
 
 // ---------------------------------------------------------------------------

@@ -93,12 +93,13 @@ def test_mask_matches_oracle(built, name, p, sta):
 
 
 # Rows of more than 1024 blocks (the HunyuanVideo-like shape has 2040): the tensor-core path's longest
-# rows, with integer masses in coarser units; the whole mask against the oracle.
-@pytest.mark.parametrize("grid,p,sta", [((17, 64, 64), 0.9, -1), ((32, 64, 64), 0.8, 1)])
+# rows, with integer masses in coarser units, and beyond 2048 blocks the float64 path; the whole mask
+# against the oracle.
+@pytest.mark.parametrize("grid,p,sta", [((17, 64, 64), 0.9, -1), ((32, 64, 64), 0.8, 1), ((34, 64, 64), 0.9, -1)])
 def test_mask_long_rows_match_oracle(built, grid, p, sta):
     w = dataclasses.replace(S.workload("small"), H=2, grid=grid, tile=(1, 8, 8))
     g = P.geometry(w)
-    assert 1024 < g.NB <= 2048
+    assert 1024 < g.NB <= 4096
     q, k, _ = S.make_qkv(w)
     qt, kt = O.tile_reorder(q, g), O.tile_reorder(k, g)
     ref, A = P.oracle_mask_per_head(qt, kt, g, p, sta)
