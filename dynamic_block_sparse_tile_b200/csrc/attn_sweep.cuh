@@ -1,8 +1,9 @@
 // Block-sparse attention kernels built on one tile walk: a CTA keeps its own 128 rows (two
 // 64-token blocks) in shared memory while the 64-row blocks of the other side stream through a
-// ring, one block per tile, over the union of the two own blocks' lists.  Three uses:
+// ring, one block per tile, over the union of the two own blocks' lists.  Uses:
 //   MODE 0  backward, dq pass            MODE 1  backward, dk/dv pass
-//   MODE 2  forward with a logit offset per (query block, key block)
+//   MODE 2  forward with 4-token group masks (and optional logit offsets)
+//   MODE 3  forward over gathered 4-token key groups
 //
 // ---- Backward (MODES 0 and 1)
 // The NABLA page ("NABLA: Neighborhood Adaptive Block-Level Attention",
@@ -41,11 +42,12 @@
 //                 acc1 += dS^T . Y          (dk; Y = Q)
 // A row (or column) whose block does not keep the tile's block gets P = dS = 0.
 //
-// ---- Forward with logit offsets (MODE 2)
-// AB-Attention's SIP ("AB-Attention accélère la génération vidéo…", section "Les trois
-// techniques", second technique) keeps a sampled set of key blocks and adds log(1/pi) to the
-// logits of each kept block, pi being its inclusion probability.  Here the offset is any
-// per-(query block, key block) value the caller supplies.  One CTA per pair of query blocks
+// ---- Forward with logit offsets and group masks (MODE 2)
+// A forward for AB-Attention's finer selections ("AB-Attention accélère la génération vidéo…",
+// section "Les trois techniques"): the 4-token key groups of the third technique (a 16-bit mask
+// per (query block, key block) masks columns), with an optional logit offset per (query block,
+// key block).  (SIP's offsets alone run in pair_attn_kernel, which folds them into its exponent.)
+// One CTA per pair of query blocks
 // (X = Q), the ring brings K and V (Y, Y2), two sweeps over the union: the first only forms
 // S = Q K^T and keeps each row's running max and sum of 2^(x - max), x = s * scale * log2 e +
 // offset * log2 e; the two column halves are merged into the row max M and L = log2 of the

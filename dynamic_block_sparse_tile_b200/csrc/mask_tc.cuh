@@ -2,7 +2,7 @@
 // "Construction de Masque Adaptatif": block mean-pool, reduced attention map,
 // CDF threshold; "Intégration Hybride avec STA": the sliding-tile union).
 //
-// Three kernels:
+// Five kernels:
 //
 //   pool_pieces_kernel (HBM-bound) averages every 64-token block of q and k
 //   exactly (64 bf16 values summed in float64) and stores each mean x as three
@@ -20,8 +20,12 @@
 //
 //   select_rows_kernel, one warp per row and many rows in flight per SM, finds
 //   the CDF boundary by bisection on the logit value with exact integer mass
-//   sums (one warp reduction per step), settles the order near the boundary
-//   (below) with a radix select on exact keys, and writes bits and lists.
+//   sums (one warp reduction per step) and writes bits and lists, or lists the
+//   row when another block lies within the error band of its boundary (below).
+//
+//   refine_rows_kernel settles the listed rows whose band fits a warp (float64
+//   logits of the band's blocks, a shuffle sort), and refine_wide_kernel the rest
+//   (a band widened until the crossing stays inside, radix select on exact keys).
 //
 // Exactness.  The order of a row's blocks must be the order of the exact
 // (float64) logits.  The fast logits carry an error below E = 2^-15 * scale *
@@ -33,8 +37,9 @@
 // all other keys placed above or below the band.  The result stands if the new
 // boundary lies within 2E of the old one; otherwise the band doubles and the
 // step repeats.  Masses are float32 exponentials of the fast logits, rounded to
-// integers of 2^-21 of the row's largest and summed exactly; a kept set can therefore differ from a
-// float64 reference only where a cumulative mass lies within rounding of p.
+// integers of 2^-21 (2^-20 for rows of more than 1024 blocks) of the row's
+// largest and summed exactly; a kept set can therefore differ from a float64
+// reference only where a cumulative mass lies within rounding of p.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
