@@ -57,6 +57,23 @@ def test_reference_arm_non_zero_rank_exits_without_work():
     assert r.stdout.strip() == ""
 
 
+def test_reference_arm_rank_zero_prints_the_contract_line():
+    """The oracle arm on rank 0: one JSON line with the metric, a positive value, the oracle as its own
+    cpu_baseline and an end-to-end figure equal to the value with no host copies."""
+    import json
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "0", "--ref-budget", "0.5"], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "TFLOP/s" and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"] == {"value": d["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
 # ---------------------------------------------------------------- head split (shard.py)
 def _oracle_local(q, k, v, gl, p, sta):
     """The oracle on one rank's heads, in place of the CUDA path: raster bf16 q, k, v -> raster (o, lse), float64."""
